@@ -1,0 +1,444 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks the oracle against hand-worked fixtures (tests/golden/), exact
+rational arithmetic, closed forms, an independent brute-force implementation, or an
+invariant the KV4-RL pages state (exact regional merge, bounded protected set,
+INT8 tracking BF16).
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import kv4_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_fixture(name):
+    out = {}
+    for line in open(os.path.join(GOLD, name)):
+        if line.startswith("#") or ":" not in line:
+            continue
+        k, v = line.split(":", 1)
+        out[k.strip()] = v.split()
+    return out
+
+
+def _bf16(x):
+    """Round float32 to the nearest bf16 value (ties to even), returned as float32."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
+    return u.astype(np.uint32).view(np.float32)
+
+
+# --------------------------------------------------------------------------
+# fp16 rounding used for stored parameters
+# --------------------------------------------------------------------------
+
+def _f16_neighbours(fr: Fraction):
+    """All finite fp16 values as Fractions, nearest two around fr."""
+    allv = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    vals = np.concatenate([-allv[::-1], allv])
+    i = np.searchsorted(vals, float(fr))
+    cand = [vals[j] for j in (i - 1, i) if 0 <= j < len(vals)]
+    return [Fraction(c) for c in cand]
+
+
+def _exact_f16_rne(fr: Fraction) -> Fraction:
+    if abs(fr) > 65504:
+        return Fraction(65504) * (1 if fr > 0 else -1)
+    cands = _f16_neighbours(fr)
+    best = min(cands, key=lambda c: (abs(c - fr),))
+    ties = [c for c in cands if abs(c - fr) == abs(best - fr)]
+    if len(ties) > 1:  # tie: even significand (last mantissa bit 0)
+        ties.sort(key=lambda c: int(np.float16(float(c)).view(np.uint16)) & 1)
+        best = ties[0]
+    return best
+
+
+def test_to_f16_is_round_nearest_even_with_saturation():
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.normal(0, 3, 300), rng.normal(0, 1e-5, 100),
+                         rng.uniform(-7e4, 7e4, 50), [65504.0, 65519.0, 70000.0, -1e9,
+                                                       2.0 ** -24 * 1.5, 2.0 ** -25]]
+                        ).astype(np.float32)
+    got = O.to_f16(xs).astype(np.float64)
+    for x, g in zip(xs, got):
+        assert Fraction(float(g)) == _exact_f16_rne(Fraction(float(x))), x
+
+
+# --------------------------------------------------------------------------
+# INT4 quantiser
+# --------------------------------------------------------------------------
+
+def test_int4_golden_group_a():
+    fx = _read_fixture("int4_group_worked.txt")
+    x = np.array([float(v) for v in fx["values"]], dtype=np.float32)
+    assert np.array_equal(_bf16(x), x)  # every input is a bf16 value
+    x128 = np.zeros(128, np.float32)
+    x128[:32] = x
+    x128[32:] = 0.25  # other groups constant: scale 0
+    codes, sc, mn = O.quantize_int4(x128)
+    assert list(codes[:32]) == [int(c) for c in fx["codes"]]
+    assert sc[0].view(np.uint16) == int(fx["scale_bits"][0], 16)
+    assert mn[0].view(np.uint16) == int(fx["min_bits"][0], 16)
+    packed = O.pack_int4_token(codes)
+    assert [int(b) for b in packed[0]] == [int(b, 16) for b in fx["packed"]]
+    # constant groups: zero scale, zero codes, min is the value
+    assert np.all(sc[1:] == 0) and np.all(codes[32:] == 0) and np.all(mn[1:] == 0.25)
+    # dequantisation of group A by hand: -1 + 0.5 * code
+    deq = O.dequant_int4(codes, sc, mn)[:32]
+    assert np.array_equal(deq, -1.0 + 0.5 * np.array(codes[:32], np.float64))
+
+
+def test_int4_golden_group_b_rounded_scale():
+    fx = _read_fixture("int4_group_worked.txt")
+    xb = np.zeros(128, np.float32)
+    vals = [float(v) for v in fx["valuesB"]]
+    xb[:len(vals)] = vals
+    codes, sc, mn = O.quantize_int4(xb)
+    assert list(codes[:len(vals)]) == [int(c) for c in fx["codesB"]]
+    assert sc[0].view(np.uint16) == int(fx["scaleB_bits"][0], 16)
+    assert mn[0].view(np.uint16) == int(fx["minB_bits"][0], 16)
+
+
+def _round_half_even(fr: Fraction) -> int:
+    f = math.floor(fr)
+    r = fr - f
+    if r > Fraction(1, 2):
+        return f + 1
+    if r < Fraction(1, 2):
+        return f
+    return f if f % 2 == 0 else f + 1
+
+
+def _groups(rng, n):
+    """Varied bf16 groups of 32: normal, outliers, tiny, one-sided, heavy tails."""
+    out = []
+    for i in range(n):
+        kind = i % 6
+        if kind == 0:
+            g = rng.normal(0, 1, 32)
+        elif kind == 1:
+            g = rng.normal(0, 1, 32)
+            g[rng.integers(0, 32, 2)] *= 10
+        elif kind == 2:
+            g = rng.normal(0, 1e-4, 32)
+        elif kind == 3:
+            g = np.abs(rng.normal(3, 1, 32))
+        elif kind == 4:
+            g = rng.standard_t(3, 32) * 5
+        else:
+            g = rng.normal(-50, 0.01, 32)
+        out.append(_bf16(g.astype(np.float32)))
+    return np.stack(out)
+
+
+def test_int4_codes_are_the_exact_nearest_level():
+    """Exact rational check: each code is the nearest level of the stored (scale, min),
+    ties to even, clamped; the stored scale/min are correctly rounded fp16."""
+    rng = np.random.default_rng(1)
+    G = _groups(rng, 240)
+    x = G.reshape(-1, 128)
+    codes, sc, mn = O.quantize_int4(x)
+    codes = codes.reshape(-1, 32)
+    sc = sc.reshape(-1)
+    mn = mn.reshape(-1)
+    near_tie = 0
+    for gi in range(G.shape[0]):
+        g = [Fraction(float(v)) for v in G[gi]]
+        lo, hi = min(g), max(g)
+        min_h = Fraction(float(mn[gi]))
+        s_h = Fraction(float(sc[gi]))
+        assert min_h == _exact_f16_rne(lo)
+        exact_s = (hi - lo) / 15
+        # stored scale: a correct fp16 rounding of a value within fp32 error of exact
+        assert abs(s_h - exact_s) <= abs(_exact_f16_rne(exact_s) - exact_s) + exact_s * Fraction(1, 2 ** 21)
+        for t in range(32):
+            c = int(codes[gi, t])
+            assert 0 <= c <= 15
+            if s_h == 0:
+                assert c == 0
+                continue
+            Q = (g[t] - min_h) / s_h
+            want = min(15, max(0, _round_half_even(Q)))
+            dist = abs(Q - math.floor(Q) - Fraction(1, 2))
+            if dist > Fraction(1, 2 ** 18) * max(1, abs(Q)):
+                assert c == want, (gi, t, float(Q))
+            else:
+                near_tie += 1
+                assert c in (min(15, max(0, math.floor(Q))), min(15, max(0, math.ceil(Q))))
+    assert near_tie < 0.01 * codes.size
+
+
+def test_int4_reconstruction_bound_and_special_groups():
+    rng = np.random.default_rng(2)
+    G = _groups(rng, 120).reshape(-1, 128)
+    codes, sc, mn = O.quantize_int4(G)
+    deq = O.dequant_int4(codes, sc, mn).reshape(-1, 4, 32)
+    g = G.reshape(-1, 4, 32).astype(np.float64)
+    s = sc.astype(np.float64)
+    span = g.max(-1) - g.min(-1)
+    slack = np.maximum(0, span - 15 * s) + np.abs(g.min(-1) - mn.astype(np.float64))
+    err = np.abs(g - deq).max(-1)
+    assert np.all(err <= s / 2 * (1 + 2 ** -9) + slack + 1e-30)
+    # a group holding only its min and max maps to codes {0, 15}
+    two = np.where(np.arange(128) % 2 == 0, -2.0, 3.0).astype(np.float32)
+    c2, _, _ = O.quantize_int4(two)
+    assert set(c2.tolist()) == {0, 15}
+
+
+# --------------------------------------------------------------------------
+# INT8 quantiser
+# --------------------------------------------------------------------------
+
+def test_int8_golden_rows():
+    fx = _read_fixture("int8_row_worked.txt")
+    for tag in ("A", "B"):
+        vals = [float(v) for v in fx["values" + tag]]
+        x = np.zeros(128, np.float32)
+        x[:len(vals)] = vals
+        assert np.array_equal(_bf16(x), x)
+        codes, sc = O.quantize_int8(x)
+        assert list(codes[:len(vals)]) == [int(c) for c in fx["codes" + tag]]
+        assert np.all(codes[len(vals):] == 0)
+        assert sc.view(np.uint16) == int(fx["scale" + tag + "_bits"][0], 16)
+
+
+def test_int8_exact_nearest_and_symmetry():
+    rng = np.random.default_rng(3)
+    X = _groups(rng, 160).reshape(-1, 128)
+    codes, sc = O.quantize_int8(X)
+    for r in range(X.shape[0]):
+        s_h = Fraction(float(sc[r]))
+        amax = max(abs(Fraction(float(v))) for v in X[r])
+        assert s_h == _exact_f16_rne(amax / 127) or \
+            abs(s_h - amax / 127) <= abs(_exact_f16_rne(amax / 127) - amax / 127) + amax / 127 * Fraction(1, 2 ** 21)
+        for t in range(0, 128, 3):
+            Q = Fraction(float(X[r, t])) / s_h
+            want = min(127, max(-127, _round_half_even(Q)))
+            dist = abs(abs(Q) - math.floor(abs(Q)) - Fraction(1, 2))
+            if dist > Fraction(1, 2 ** 18) * max(1, abs(Q)):
+                assert int(codes[r, t]) == want
+    neg, sc2 = O.quantize_int8(-X)
+    assert np.array_equal(neg, -codes) and np.array_equal(sc2, sc)
+    deq = O.dequant_int8(codes, sc)
+    assert np.all(np.abs(deq - X) <= sc.astype(np.float64)[:, None] / 2 * (1 + 2 ** -9))
+    z, zs = O.quantize_int8(np.zeros((2, 128), np.float32))
+    assert np.all(z == 0) and np.all(zs == 0)
+
+
+# --------------------------------------------------------------------------
+# protected set and regions (bound from ai4snews "Interpretation" para. 3)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("S,R", [(0, 0), (4, 32), (16, 128), (0, 144), (144, 0), (7, 13)])
+def test_regions_partition_and_protected_bound(S, R):
+    for L in range(0, 420):
+        (a0, a1), (b0, b1), (c0, c1) = O.regions(L, S, R)
+        cover = np.zeros(L, int)
+        for lo, hi in ((a0, a1), (b0, b1), (c0, c1)):
+            assert 0 <= lo <= hi <= L
+            cover[lo:hi] += 1
+        assert np.all(cover == 1)
+        prot = O.protected_mask(L, S, R)
+        assert prot.sum() == min(L, S + R) <= 144
+        # protected positions are exactly the first S and the last R
+        idx = np.arange(L)
+        assert np.array_equal(prot, (idx < S) | (idx >= L - R))
+
+
+def test_protected_set_over_144_is_rejected():
+    with pytest.raises(ValueError):
+        O.regions(500, 16, 129)
+    with pytest.raises(ValueError):
+        O.check_protection(145, 0)
+
+
+def test_ring_window_matches_sequential_appends():
+    """expected_side's window formula equals literally appending tokens one by one."""
+    rng = np.random.default_rng(4)
+    for (S, R, L) in [(4, 32, 37), (4, 32, 20), (16, 128, 300), (0, 16, 50), (3, 5, 5), (2, 8, 9)]:
+        k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+        rec = O.token_records(k, k)
+        sim_sink, sim_ring = {}, {}
+        for pos in range(L):  # append procedure: sink slot pos, else ring slot pos mod R
+            if pos < S:
+                sim_sink[pos] = pos
+            else:
+                sim_ring[pos % R] = pos
+        sk, sks, _, _, rk, rks, _, _ = O.expected_side(rec, L, S, R)
+        for slot in range(sk.shape[1] * 16):
+            want = rec["k8"][sim_sink[slot]] if slot in sim_sink else 0
+            assert np.array_equal(sk[:, slot // 16, :, slot % 16, :], np.broadcast_to(want, (2, 8, 16)))
+        for slot in range(rk.shape[1] * 16):
+            want = rec["ks"][sim_ring[slot]] if slot in sim_ring else 0
+            assert np.array_equal(rks[:, slot], np.broadcast_to(want, (2,)))
+
+
+# --------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------
+
+def _loop_attention(q, K, V):
+    """Independent brute force: explicit loops, math.exp, math.fsum."""
+    Hq, D = q.shape
+    L, Hkv, _ = K.shape
+    G = Hq // Hkv
+    out = np.zeros((Hq, D))
+    for j in range(Hq):
+        h = j // G
+        s = [math.fsum(float(K[t, h, d]) * float(q[j, d]) for d in range(D)) / math.sqrt(D)
+             for t in range(L)]
+        m = max(s)
+        w = [math.exp(x - m) for x in s]
+        den = math.fsum(w)
+        for d in range(D):
+            out[j, d] = math.fsum(w[t] * float(V[t, h, d]) for t in range(L)) / den
+    return out
+
+
+def test_attention_brute_force_tiny():
+    rng = np.random.default_rng(5)
+    for L in (1, 2, 5, 8):
+        q = rng.normal(0, 1, (4, 128))
+        K = rng.normal(0, 1, (L, 2, 128))
+        V = rng.normal(0, 1, (L, 2, 128))
+        got, lse = O.attention(q, K, V)
+        assert np.max(np.abs(got - _loop_attention(q, K, V))) < 1e-12
+
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(6)
+    q = rng.normal(0, 1, (4, 128))
+    # identical keys -> uniform weights -> mean of values
+    K = np.repeat(rng.normal(0, 1, (1, 2, 128)), 7, axis=0)
+    V = rng.normal(0, 1, (7, 2, 128))
+    got, lse = O.attention(q, K, V)
+    for j in range(4):
+        assert np.allclose(got[j], V[:, j // 2].mean(0), atol=1e-13)
+        s0 = K[0, j // 2] @ q[j] / math.sqrt(128)
+        assert abs(lse[j] - (s0 + math.log(7))) < 1e-12
+    # two tokens: sigmoid weights
+    K2 = rng.normal(0, 1, (2, 2, 128))
+    V2 = rng.normal(0, 1, (2, 2, 128))
+    got, _ = O.attention(q, K2, V2)
+    for j in range(4):
+        h = j // 2
+        d = (K2[0, h] - K2[1, h]) @ q[j] / math.sqrt(128)
+        w0 = 1.0 / (1.0 + math.exp(-d))
+        assert np.allclose(got[j], w0 * V2[0, h] + (1 - w0) * V2[1, h], atol=1e-13)
+    # empty context
+    e, l = O.attention(q, np.zeros((0, 2, 128)), np.zeros((0, 2, 128)))
+    assert np.all(e == 0) and np.all(np.isneginf(l))
+
+
+def test_attention_gqa_mapping():
+    rng = np.random.default_rng(7)
+    q = rng.normal(0, 1, (8, 128))
+    K = rng.normal(0, 1, (6, 2, 128))
+    V = rng.normal(0, 1, (6, 2, 128))
+    got, _ = O.attention(q, K, V)
+    for h in range(2):
+        sub, _ = O.attention(q[4 * h:4 * h + 4], K[:, h:h + 1], V[:, h:h + 1])
+        assert np.array_equal(got[4 * h:4 * h + 4], sub)
+
+
+# --------------------------------------------------------------------------
+# the exact regional merge (ai4snews "Interpretation" para. 3)
+# --------------------------------------------------------------------------
+
+def test_regional_merge_equals_monolithic_softmax():
+    rng = np.random.default_rng(8)
+    for trial in range(60):
+        L = int(rng.integers(1, 300))
+        K = rng.normal(0, 2, (L, 128))
+        V = rng.normal(0, 1, (L, 128))
+        q = rng.normal(0, 1, 128)
+        mono, lse = O.attention(q[None], K[:, None], V[:, None])
+        nreg = int(rng.integers(1, 21))
+        cuts = np.sort(rng.integers(0, L + 1, nreg - 1))
+        bounds = np.concatenate([[0], cuts, [L]])
+        parts = [O.partial_state(q, K[a:b], V[a:b]) for a, b in zip(bounds[:-1], bounds[1:])]
+        got, glse = O.merge_partials(parts)
+        assert np.max(np.abs(got - mono[0])) <= 1e-12 * max(1, np.abs(mono).max())
+        assert abs(glse - lse[0]) <= 1e-12 * max(1, abs(lse[0]))
+        perm = rng.permutation(len(parts))
+        got2, _ = O.merge_partials([parts[i] for i in perm])
+        assert np.max(np.abs(got2 - got)) <= 1e-12
+
+
+def test_merge_of_empty_regions():
+    D = 128
+    empty = (-np.inf, 0.0, np.zeros(D))
+    o, l = O.merge_partials([empty, empty])
+    assert np.all(o == 0) and np.isneginf(l)
+    one = (1.5, 2.0, np.full(D, 4.0))
+    o, l = O.merge_partials([empty, one, empty])
+    assert np.allclose(o, 2.0) and abs(l - (1.5 + math.log(2.0))) < 1e-15
+
+
+# --------------------------------------------------------------------------
+# the cache as a whole
+# --------------------------------------------------------------------------
+
+def test_decode_reference_partition_special_cases():
+    rng = np.random.default_rng(9)
+    L = 40
+    k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    v = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    q = _bf16(rng.normal(0, 1, (8, 128)).astype(np.float32))
+    # S = R = 0: plain INT4 everywhere
+    c, s, m = O.quantize_int4(k)
+    cv, sv, mv = O.quantize_int4(v)
+    want, _ = O.attention(q, O.dequant_int4(c, s, m), O.dequant_int4(cv, sv, mv))
+    got, _ = O.decode_reference(q, k, v, 0, 0)
+    assert np.array_equal(got, want)
+    # L <= S + R: plain INT8 everywhere
+    c8, s8 = O.quantize_int8(k)
+    cv8, sv8 = O.quantize_int8(v)
+    want8, _ = O.attention(q, O.dequant_int8(c8, s8), O.dequant_int8(cv8, sv8))
+    got8, _ = O.decode_reference(q, k, v, 8, 32)
+    assert np.array_equal(got8, want8)
+
+
+def test_all_int8_tracks_bf16_within_derived_bound():
+    """KV8 tracks BF16 (ai4snews "Interpretation" para. 2): with every position
+    protected, |O_int8 - O_bf16| <= (e^(2 delta) - 1) max|v| + max scale_v / 2,
+    delta = max_t sum_d |q_d| scale_k,t / (2 sqrt d)."""
+    rng = np.random.default_rng(10)
+    for L in (5, 60, 144):
+        k = _bf16(rng.normal(0, 1, (L, 1, 128)).astype(np.float32))
+        v = _bf16(rng.normal(0, 1, (L, 1, 128)).astype(np.float32))
+        q = _bf16(rng.normal(0, 1, (4, 128)).astype(np.float32))
+        got, _ = O.decode_reference(q, k, v, 16, 128)
+        ref, _ = O.attention(q, k.astype(np.float64), v.astype(np.float64))
+        _, sk = O.quantize_int8(k)
+        _, sv = O.quantize_int8(v)
+        for j in range(4):
+            delta = (np.abs(q[j]).sum() * sk.astype(np.float64).max() / 2) / math.sqrt(128)
+            bound = (math.exp(2 * delta) - 1) * np.abs(v).max() + sv.astype(np.float64).max() / 2
+            err = np.abs(got[j] - ref[j]).max()
+            assert err <= bound
+        assert np.abs(got - ref).max() < 0.05  # and it is small in absolute terms
+
+
+def test_expected_pages_layout():
+    rng = np.random.default_rng(11)
+    L = 21
+    k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    rec = O.token_records(k, k)
+    pages = O.expected_pages(rec, L, np.array([7, 3]))
+    assert set(pages) == {7, 3}
+    kc, kp, _, _ = pages[3]
+    # page 3 holds positions 16..20 in slots 0..4, zeros after
+    assert np.array_equal(kc[:, :, :5, :], rec["k4"][16:21].transpose(1, 2, 0, 3))
+    assert np.all(kc[:, :, 5:, :] == 0) and np.all(kp[:, 5:] == 0)
+    # nibble order: dim 2i in the low nibble of byte i
+    c, s, m = O.quantize_int4(k[16])
+    assert np.array_equal(kc[1, 2, 0, 5] & 0xF, c[1, 64 + 10])
+    assert np.array_equal(kc[1, 2, 0, 5] >> 4, c[1, 64 + 11])
+    assert kp[1, 0, 2, 0] == s[1, 2].view(np.uint16) and kp[1, 0, 2, 1] == m[1, 2].view(np.uint16)
