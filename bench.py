@@ -1,0 +1,375 @@
+"""Benchmark: batched decode steps of paged INT4 + INT8-protected attention on B200.
+
+One step = the whole hot path for one batch: kv4_quantize_append of one new token per
+sequence (INT4 page write, INT8 copy, demotion out of the recent window) followed by
+kv4_decode_attention (INT8 protected partials, split-K INT4 partials, exact regional
+merge). The workload defaults to the 1024-sequence async-rollout batch (128 groups x 8
+responses sharing a 256-token prompt, lognormal response lengths with mean 1450).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kv4|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own full batch (data-parallel
+rollout replicas, no collective in the data path: weak scaling); the timed region is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention tokens*KV-heads/s"
+UNIT = "tokens*kv_heads/s"
+
+
+# ----------------------------------------------------------------------------
+# workload accounting (host arithmetic on lengths only)
+# ----------------------------------------------------------------------------
+
+def units_per_step(wl, lens) -> int:
+    """Context tokens x KV heads attended in one step."""
+    return int(np.asarray(lens, dtype=np.int64).sum()) * wl.num_kv_heads
+
+
+def attention_bytes(wl, lens):
+    """Algorithmic HBM bytes of one attention call: (unique, logical).
+
+    Per token and KV head: 160 B when read from INT4 (64 B K codes + 16 B K params +
+    the same for V), 260 B when read from INT8 (128 B codes + 2 B scale, K and V).
+    Plus the query read and the output write (bf16). `unique` counts a group's shared
+    prompt pages and shared sink set once; `logical` counts them per sequence."""
+    lens = np.asarray(lens, dtype=np.int64)
+    S, R, H = wl.num_sinks, wl.num_recent, wl.num_kv_heads
+    prot = np.minimum(lens, S + R)
+    int4 = np.maximum(0, lens - S - R)
+    logical = (int4 * 160 + prot * 260).sum() * H
+    io = lens.size * wl.num_q_heads * wl.head_dim * 2 * 2
+    unique = logical
+    if wl.shared_prefix:
+        P = wl.prompt_len
+        shared_int4 = np.maximum(0, np.minimum(P, lens - R) - S)  # prompt part of INT4 range
+        shared_sink = np.minimum(lens, S)
+        groups = (lens.size + wl.group_seqs - 1) // wl.group_seqs
+        dup = 0
+        for g in range(groups):
+            sl = slice(g * wl.group_seqs, (g + 1) * wl.group_seqs)
+            n = lens[sl].size
+            # counted n times, should be once (all sequences in a group share them)
+            dup += (shared_int4[sl].min() * 160 + shared_sink[sl].min() * 260) * (n - 1)
+        unique = logical - dup * H
+    return int(unique + io), int(logical + io)
+
+
+def append_bytes(wl) -> int:
+    """Per step: read bf16 K/V of the new token, write INT4 record (+ INT8 copy)."""
+    return wl.num_seqs * wl.num_kv_heads * (2 * 2 * wl.head_dim + 160 + 260)
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(wl, budget_s: float, start_seq: int = 0):
+    """Time the oracle's decode output (quantise -> dequantise -> softmax attention) on
+    consecutive sequences of the workload until `budget_s` of CPU time is used.
+    Returns (units processed, seconds, description, threads)."""
+    import torch
+    from oracle import kv4_oracle as O
+    from quantized_kv_cache_kv4_b200.workload import queries, seq_kv
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    q_all = queries(wl, 0, 0, "cpu").float().numpy()
+    units, spent, seqs = 0, 0.0, []
+    b = start_seq
+    while spent < budget_s and len(seqs) < wl.num_seqs:
+        bb = b % wl.num_seqs
+        L = int(wl.seq_lens[bb])
+        k, v = seq_kv(wl, bb, L, 0, "cpu")
+        k, v = k.float().numpy(), v.float().numpy()
+        t0 = time.perf_counter()
+        O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent)
+        spent += time.perf_counter() - t0
+        units += L * wl.num_kv_heads
+        seqs.append(bb)
+        b += 1
+    desc = (f"oracle decode_reference (fp64 numpy: quantise every position, dequantise, "
+            f"softmax attention) on {len(seqs)} sequence(s) of the workload "
+            f"({units // wl.num_kv_heads} context tokens)")
+    return units, spent, desc, threads
+
+
+def run_reference(args, rank, world):
+    from quantized_kv_cache_kv4_b200.workload import make_workload
+    if rank != 0:
+        return
+    wl = make_workload(args.workload)
+    total_units, total_s, descs, threads = 0, 0.0, [], 1
+    per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for s in range(args.warmup + args.steps):
+        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3)
+        if s >= args.warmup:
+            total_units += u
+            total_s += t
+            descs.append(d)
+    value = total_units / total_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, **wl.describe()},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": descs[0] if descs else ""},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_kv_cache_kv4_b200 import build
+    build.build()
+    from quantized_kv_cache_kv4_b200 import kv4
+    from quantized_kv_cache_kv4_b200.session import DecodeSession
+    from quantized_kv_cache_kv4_b200.workload import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    wl = make_workload(args.workload)
+    wl.seed = wl.seed + 7919 * rank  # each rank: its own replica batch (same shape)
+    W, K = args.warmup, args.steps
+    sess = DecodeSession(wl, steps=W + K, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    H = wl.num_kv_heads
+    L0 = wl.seq_lens.astype(np.int64)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for s in range(W):
+        sess.step(s)
+    torch.cuda.synchronize(dev)
+    sess.check_err()
+
+    # ---- timed region: K full steps (append + attention), device events ----
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        ev[0].record(stream)
+        for i, s in enumerate(range(W, W + K)):
+            sess.append_step(s)
+            att[i][0].record(stream)
+            sess.attention_step(s)
+            att[i][1].record(stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    sess.check_err()
+    ms = ev[0].elapsed_time(ev[1])
+    att_ms = [a.elapsed_time(b) for a, b in att]
+    units_local = sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
+    t = torch.tensor([ms, float(units_local)], dtype=torch.float64, device=dev)
+    if world > 1:
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        usum = t[1:].clone()
+        dist.all_reduce(usum, op=dist.ReduceOp.SUM)
+        ms_max, units_all = float(tmax.item()), float(usum.item())
+    else:
+        ms_max, units_all = ms, float(units_local)
+    value = units_all / (ms_max / 1000.0)
+
+    # ---- roofline of the attention call (plan + split-K attention + merge) ----
+    uniq = [attention_bytes(wl, L0 + s) for s in range(W, W + K)]
+    mean_att_s = statistics.mean(att_ms) / 1000.0
+    achieved = statistics.mean(u for u, _ in uniq) / mean_att_s / 1e9
+    peak, peak_kind = load_peaks()
+
+    # ---- e2e through the public API with host buffers (H2D inputs, D2H output) ----
+    B, Hq, D = wl.num_seqs, wl.num_q_heads, wl.head_dim
+    hk = sess.step_k.cpu().pin_memory()
+    hv = sess.step_v.cpu().pin_memory()
+    hq = sess.q.cpu().pin_memory()
+    hl = sess.step_lens.cpu().pin_memory()
+    hout = torch.empty((K, B, Hq, D), dtype=torch.bfloat16).pin_memory()
+    dk = torch.empty_like(sess.step_k[0])
+    dv = torch.empty_like(sess.step_v[0])
+    dq = torch.empty_like(sess.q[0])
+    dl = torch.empty_like(sess.step_lens[0])
+    dout = torch.empty_like(sess.out)
+    h2d = (dk.numel() + dv.numel() + dq.numel()) * 2 + dl.numel() * 4
+    d2h = dout.numel() * 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i, s in enumerate(range(W, W + K)):
+        dk.copy_(hk[s], non_blocking=True)
+        dv.copy_(hv[s], non_blocking=True)
+        dq.copy_(hq[s], non_blocking=True)
+        dl.copy_(hl[s], non_blocking=True)
+        b = sess.batch(dl)
+        kv4.quantize_append(sess.cache, b, dk, dv, None, sess.err)
+        kv4.decode_attention(sess.cache, b, dq, dout, sess.workspace, err=sess.err)
+        hout[i].copy_(dout, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sess.check_err()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = units_all / (float(e2e_ms.item()) / 1000.0)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget)
+        cpu = {"value": u / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        ub = statistics.mean(u for u, _ in uniq)
+        lb = statistics.mean(l for _, l in uniq)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc, int4/int8 codes",
+            "data": "synthetic",
+            "config": {"workload": wl.name, **wl.describe(),
+                       "l2": "inputs larger than L2: the cache read per step is "
+                             f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
+                       "parallelism": f"dp{world} (independent replica batches)"},
+            "attention_ms": statistics.mean(att_ms),
+            "attention_gbs_unique": ub / mean_att_s / 1e9,
+            "attention_gbs_logical": lb / mean_att_s / 1e9,
+            "roofline": {"kernel": "kv4_decode_attention (plan + attn + merge launches)",
+                         "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * K,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
+    ap.add_argument("--workload", default="rollout")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

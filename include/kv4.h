@@ -1,0 +1,216 @@
+/*
+ * kv4.h -- C ABI of a B200 (sm_100a) library for batched decode-step GQA attention
+ * over a paged INT4 KV cache with bounded INT8 protection of attention sinks and a
+ * recent window.
+ *
+ * The method is KV4-RL (arXiv 2610.14448, "KV4-RL: Unlocking Faster Asynchronous
+ * Rollouts for RLVR with INT4 KV Cache Quantization"):
+ *   - the whole context is kept in calibration-free INT4 in a paged format, and INT8
+ *     copies are kept for a fixed set of attention-sink and recent positions, at most
+ *     144 of them (ai4snews summary, "Interpretation" para. 3; aimodeling article,
+ *     "INT4 as the base, INT8 insurance for critical positions");
+ *   - attention runs over the integer codes and combines the regions with an exact
+ *     regional softmax merge (ai4snews summary, "Interpretation" para. 3);
+ *   - protected positions use higher-fidelity probability-value arithmetic
+ *     (aimodeling article, same section).
+ * The pages give no bit-level format and no API; the format and calls below are this
+ * library's own, chosen as the plainest reading of those statements.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned and allocated by the caller. The
+ *     library never allocates, frees or synchronises; every call is asynchronous on
+ *     the given stream (NULL = the legacy default stream).
+ *   - Arguments are checked on the host before anything is launched; a failed check
+ *     returns a negative kv4_status and launches nothing.
+ *   - Data-dependent checks run on the device: a kernel that meets a bad page id,
+ *     sequence length, side-store index or workspace overflow ORs a KV4_DEVERR_* bit
+ *     into *err_flag (a device int32 the caller zeroes and reads after synchronising)
+ *     and skips the offending work item. Kernels never trap and never spin without a
+ *     bound.
+ *   - fp16 and bf16 values are passed as their 16-bit patterns.
+ *
+ * Storage format (all little-endian; "slot" = token position within a page or tile):
+ *
+ *   INT4 pool, one block per (page, kv head), pages of 16 tokens:
+ *     k_codes, v_codes  uint8 [num_pages][Hkv][4 groups][16 slots][16 bytes]
+ *         byte i of (group g, slot t) = code(dim 32g+2i) | code(dim 32g+2i+1) << 4
+ *     k_params, v_params  fp16 [num_pages][Hkv][16 slots][4 groups][2] = (scale, min)
+ *     Per token and 32-dim group:  min = fp16(group min),
+ *         scale = fp16(fp32(fp32(max - min) / 15)),
+ *         code  = clamp(rne(fp32(fp32(x - min) / scale)), 0, 15)   (0 if scale == 0),
+ *     fp16 rounding is nearest-even saturating at +-65504. Value = code*scale + min.
+ *
+ *   INT8 side store, tiles of 16 slots:
+ *     codes  int8 [..][Hkv][tiles][8 strips][16 slots][16 bytes]
+ *         byte i of (strip c, slot t) = code(dim 16c + i)
+ *     scales fp16 [..][Hkv][tiles*16]
+ *     Per token: scale = fp16(fp32(max|x| / 127)),
+ *         code = clamp(rne(fp32(x / scale)), -127, 127)  (0 if scale == 0).
+ *     Value = code*scale.
+ *     Sink sets: tiles = ceil(S/16); slot p holds position p < S.
+ *     Recent rings: tiles = ceil(R/16); slot (p mod R) holds position p >= S.
+ *
+ *   Regions of a context of length L (S sinks, R recent, S + R <= 144):
+ *     sink [0, min(S,L)) and recent [max(S, L-R), L) are read from INT8,
+ *     [S, L-R) (when L-R > S) is read from the INT4 pages. Every position is also
+ *     stored in INT4 ("whole context in INT4"); the INT8 copy of a position is
+ *     overwritten (demoted) when position p+R is appended.
+ */
+#ifndef KV4_H
+#define KV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *kv4_stream_t;
+
+typedef enum {
+  KV4_OK = 0,
+  KV4_ERR_INVALID_ARG = -1,         /* NULL pointer, negative size, inconsistent struct */
+  KV4_ERR_UNSUPPORTED_SHAPE = -2,   /* head_dim != 128, page_size != 16, group_size != 32,
+                                       Hq not a multiple of Hkv, or Hq/Hkv > 8 */
+  KV4_ERR_PROTECTED_TOO_LARGE = -3, /* num_sinks + num_recent > 144 */
+  KV4_ERR_WORKSPACE_TOO_SMALL = -4, /* ws_bytes < kv4_workspace_size(...) */
+  KV4_ERR_CUDA = -5                 /* a CUDA runtime call failed (launch error) */
+} kv4_status;
+
+/* Bits OR-ed into *err_flag by the kernels. */
+#define KV4_DEVERR_PAGE_ID 1u    /* page-table entry outside [0, num_pages) */
+#define KV4_DEVERR_SEQ_LEN 2u    /* seq_len < 0, > max_pages*16, or fewer tokens than appended */
+#define KV4_DEVERR_SIDE_IDX 4u   /* sink_idx / ring_idx outside the side store */
+#define KV4_DEVERR_Q_RANGE 8u    /* a query element overflows fp16 (|q| > 65504) */
+#define KV4_DEVERR_WORKSPACE 16u /* the batch needs more work items than the workspace holds */
+#define KV4_DEVERR_TIMEOUT 32u   /* a bounded wait for an async copy gave up */
+
+#define KV4_MAX_PROTECTED 144
+
+typedef struct {
+  int32_t num_q_heads;  /* Hq */
+  int32_t num_kv_heads; /* Hkv; query head j reads kv head j / (Hq/Hkv) */
+  int32_t head_dim;     /* must be 128 */
+  int32_t page_size;    /* must be 16 */
+  int32_t group_size;   /* must be 32 */
+  int32_t num_sinks;    /* S >= 0 */
+  int32_t num_recent;   /* R >= 0, S + R <= 144 */
+  int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region; 0 = default (32) */
+} kv4_config;
+
+typedef struct {
+  uint8_t *k_codes;   /* see "INT4 pool" above */
+  uint8_t *v_codes;
+  uint16_t *k_params;
+  uint16_t *v_params;
+  int32_t num_pages;
+} kv4_int4_pool;
+
+typedef struct {
+  int8_t *sink_k;     /* [num_sink_sets][Hkv][ceil(S/16)][8][16][16]; may be NULL if S == 0 */
+  int8_t *sink_v;
+  uint16_t *sink_ks;  /* [num_sink_sets][Hkv][ceil(S/16)*16] */
+  uint16_t *sink_vs;
+  int32_t num_sink_sets;
+  int8_t *ring_k;     /* [num_rings][Hkv][ceil(R/16)][8][16][16]; may be NULL if R == 0 */
+  int8_t *ring_v;
+  uint16_t *ring_ks;  /* [num_rings][Hkv][ceil(R/16)*16] */
+  uint16_t *ring_vs;
+  int32_t num_rings;
+} kv4_int8_side;
+
+typedef struct {
+  const int32_t *page_table; /* [num_seqs][max_pages]: page of positions [16i, 16i+16) */
+  int32_t max_pages;
+  const int32_t *seq_lens;   /* [num_seqs]: context length AFTER this step's append */
+  const int32_t *sink_idx;   /* [num_seqs]: sink set of each sequence (sequences that share
+                                a prompt may share one); may be NULL if S == 0 */
+  const int32_t *ring_idx;   /* [num_seqs]: recent ring of each sequence; NULL = identity */
+  int32_t num_seqs;
+  int32_t max_seq_len;       /* host-side upper bound on seq_lens, sizes the workspace */
+} kv4_batch;
+
+/*
+ * Bytes of device workspace kv4_decode_attention needs for a batch of num_seqs
+ * sequences no longer than max_seq_len. Returns 0 for invalid arguments.
+ */
+size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len);
+
+/*
+ * Quantise and append new tokens' K/V: the per-step write path (with n = 1 per
+ * sequence), also usable for bulk prefill.
+ *
+ *   k_new, v_new: bf16 [total_new][Hkv][128], device.
+ *   new_indptr:   int32 [num_seqs+1], device, CSR row ranges: rows new_indptr[b] ..
+ *                 new_indptr[b+1]-1 are sequence b's new tokens, in position order,
+ *                 placed at positions seq_lens[b]-n_b .. seq_lens[b]-1. NULL means
+ *                 exactly one new token per sequence (row b, position seq_lens[b]-1).
+ *   total_new:    number of rows (== num_seqs when new_indptr is NULL).
+ *
+ * Every token is written to its INT4 page slot. A token at position p < S is also
+ * written to sink set sink_idx[b]; a token at p >= S whose position lies in the final
+ * recent window [seq_lens[b]-R, seq_lens[b]) is written to ring slot p mod R of ring
+ * ring_idx[b], overwriting -- demoting -- the INT8 copy of position p-R. (Tokens that
+ * would be demoted again within the same call are not written to the ring, so a bulk
+ * append leaves the same state as appending one token at a time.)
+ * Sequences that share pages must not append into the same page in one call.
+ */
+kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
+                               const kv4_int8_side *side, const kv4_batch *batch,
+                               const void *k_new, const void *v_new,
+                               const int32_t *new_indptr, int32_t total_new,
+                               int32_t *err_flag, kv4_stream_t stream);
+
+/*
+ * Decode-step attention: for every sequence b and query head j,
+ *   O[b, j] = softmax(K_eff q / sqrt(128)) V_eff over positions [0, seq_lens[b]),
+ * where K_eff/V_eff are the INT8 dequantised copies on protected positions and the
+ * INT4 dequantised values elsewhere. Each region (the protected set, and each chunk of
+ * `chunk_pages` INT4 pages) yields a partial softmax state (max, denominator, weighted
+ * value sum) that an exact log-sum-exp merge combines in a fixed order, so results
+ * are deterministic.
+ *
+ *   q:       bf16 [num_seqs][Hq][128]; |q| must be <= 65504 (fp16 range).
+ *   out:     bf16 [num_seqs][Hq][128].
+ *   out_f32: optional fp32 [num_seqs][Hq][128] (NULL to skip).
+ *   lse:     optional fp32 [num_seqs][Hq], natural log of the softmax denominator
+ *            (including the max); -inf for empty sequences (NULL to skip).
+ *   workspace, ws_bytes: device scratch of at least kv4_workspace_size(cfg, num_seqs,
+ *            max_seq_len) bytes, 256-byte aligned; contents need no initialisation.
+ * A sequence of length 0 yields O = 0.
+ */
+kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool,
+                                const kv4_int8_side *side, const kv4_batch *batch,
+                                const void *q, void *out, float *out_f32, float *lse,
+                                void *workspace, size_t ws_bytes, int32_t *err_flag,
+                                kv4_stream_t stream);
+
+/*
+ * Exact regional softmax merge (ai4snews summary, "Interpretation" para. 3) of partial
+ * states. A partial record is head_dim+4 floats: acc[head_dim] (sum of e^(s-m) v),
+ * m (max logit, natural-log units), l (sum of e^(s-m)), 2 unused. Record (r, j) of
+ * region r and query j sits at partials + (r*group + j)*(head_dim+4).
+ * Unit u merges regions region_offsets[u] .. region_offsets[u+1]-1 in that order:
+ *   M = max m_r, Lambda = sum l_r e^(m_r-M), O = sum acc_r e^(m_r-M) / Lambda,
+ * skipping regions with l = 0. Output (u, j): out/out_f32 at (u*group + j)*head_dim,
+ * lse at u*group + j. A unit without live regions yields O = 0 and lse = -inf.
+ *   partials, region_offsets: device; head_dim must be 128; group in [1, 8].
+ */
+kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offsets,
+                              int32_t n_units, int32_t group, int32_t head_dim,
+                              void *out, float *out_f32, float *lse,
+                              kv4_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *kv4_status_string(kv4_status status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int32_t kv4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KV4_H */

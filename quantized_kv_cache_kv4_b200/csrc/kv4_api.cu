@@ -1,0 +1,180 @@
+// C-ABI entry points declared in include/kv4.h: host-side argument checks, workspace
+// carve-up, and kernel launches on the caller's stream. No allocation, no sync.
+#include <cuda_runtime.h>
+
+#include "../../include/kv4.h"
+#include "kv4_device.cuh"
+#include "kv4_internal.h"
+
+namespace {
+
+constexpr int kDefaultChunkPages = 32;
+
+kv4_status check_config(const kv4_config *cfg) {
+  if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
+  if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_sinks < 0 ||
+      cfg->num_recent < 0 || cfg->chunk_pages < 0)
+    return KV4_ERR_INVALID_ARG;
+  if (cfg->head_dim != kv4::kHeadDim || cfg->page_size != kv4::kPage ||
+      cfg->group_size != kv4::kGroup)
+    return KV4_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->num_q_heads % cfg->num_kv_heads != 0 ||
+      cfg->num_q_heads / cfg->num_kv_heads > kv4::kMaxGqa)
+    return KV4_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->chunk_pages > 32) return KV4_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->num_sinks + cfg->num_recent > KV4_MAX_PROTECTED) return KV4_ERR_PROTECTED_TOO_LARGE;
+  return KV4_OK;
+}
+
+int chunk_of(const kv4_config *cfg) {
+  return cfg->chunk_pages > 0 ? cfg->chunk_pages : kDefaultChunkPages;
+}
+
+bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+kv4_status make_view(const kv4_config *cfg, const kv4_int4_pool *pool, const kv4_int8_side *side,
+                     const kv4_batch *batch, kv4::CacheView *v) {
+  kv4_status st = check_config(cfg);
+  if (st != KV4_OK) return st;
+  if (pool == nullptr || side == nullptr || batch == nullptr) return KV4_ERR_INVALID_ARG;
+  if (batch->num_seqs < 0 || batch->max_pages <= 0 || batch->max_seq_len < 0 ||
+      pool->num_pages < 0)
+    return KV4_ERR_INVALID_ARG;
+  if (batch->num_seqs > 0 && (batch->page_table == nullptr || batch->seq_lens == nullptr))
+    return KV4_ERR_INVALID_ARG;
+  if (!pool->k_codes || !pool->v_codes || !pool->k_params || !pool->v_params)
+    return KV4_ERR_INVALID_ARG;
+  if (misaligned16(pool->k_codes) || misaligned16(pool->v_codes) ||
+      misaligned16(pool->k_params) || misaligned16(pool->v_params))
+    return KV4_ERR_INVALID_ARG;
+  const int S = cfg->num_sinks, R = cfg->num_recent;
+  if (S > 0) {
+    if (!side->sink_k || !side->sink_v || !side->sink_ks || !side->sink_vs ||
+        side->num_sink_sets <= 0 || batch->sink_idx == nullptr)
+      return KV4_ERR_INVALID_ARG;
+    if (misaligned16(side->sink_k) || misaligned16(side->sink_v) ||
+        misaligned16(side->sink_ks) || misaligned16(side->sink_vs))
+      return KV4_ERR_INVALID_ARG;
+  }
+  if (R > 0) {
+    if (!side->ring_k || !side->ring_v || !side->ring_ks || !side->ring_vs || side->num_rings <= 0)
+      return KV4_ERR_INVALID_ARG;
+    if (misaligned16(side->ring_k) || misaligned16(side->ring_v) ||
+        misaligned16(side->ring_ks) || misaligned16(side->ring_vs))
+      return KV4_ERR_INVALID_ARG;
+  }
+  v->k_codes = pool->k_codes;
+  v->v_codes = pool->v_codes;
+  v->k_params = pool->k_params;
+  v->v_params = pool->v_params;
+  v->num_pages = pool->num_pages;
+  v->sink_k = side->sink_k;
+  v->sink_v = side->sink_v;
+  v->sink_ks = side->sink_ks;
+  v->sink_vs = side->sink_vs;
+  v->num_sink_sets = S > 0 ? side->num_sink_sets : 0;
+  v->sink_tiles = (S + kv4::kPage - 1) / kv4::kPage;
+  v->ring_k = side->ring_k;
+  v->ring_v = side->ring_v;
+  v->ring_ks = side->ring_ks;
+  v->ring_vs = side->ring_vs;
+  v->num_rings = R > 0 ? side->num_rings : 0;
+  v->ring_tiles = (R + kv4::kPage - 1) / kv4::kPage;
+  v->page_table = batch->page_table;
+  v->max_pages = batch->max_pages;
+  v->seq_lens = batch->seq_lens;
+  v->sink_idx = batch->sink_idx;
+  v->ring_idx = batch->ring_idx;
+  v->num_seqs = batch->num_seqs;
+  v->num_kv_heads = cfg->num_kv_heads;
+  v->gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  v->num_sinks = S;
+  v->num_recent = R;
+  return KV4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
+  if (check_config(cfg) != KV4_OK || num_seqs < 0 || max_seq_len < 0) return 0;
+  return kv4::workspace_bytes(num_seqs, max_seq_len, cfg->num_kv_heads,
+                              cfg->num_q_heads / cfg->num_kv_heads, chunk_of(cfg), nullptr,
+                              nullptr);
+}
+
+kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
+                               const kv4_int8_side *side, const kv4_batch *batch,
+                               const void *k_new, const void *v_new, const int32_t *new_indptr,
+                               int32_t total_new, int32_t *err_flag, kv4_stream_t stream) {
+  kv4::CacheView v;
+  kv4_status st = make_view(cfg, pool, side, batch, &v);
+  if (st != KV4_OK) return st;
+  if (total_new < 0) return KV4_ERR_INVALID_ARG;
+  if (new_indptr == nullptr && total_new != batch->num_seqs) return KV4_ERR_INVALID_ARG;
+  if (total_new > 0 && (k_new == nullptr || v_new == nullptr)) return KV4_ERR_INVALID_ARG;
+  if (misaligned16(k_new) || misaligned16(v_new)) return KV4_ERR_INVALID_ARG;
+  if (total_new == 0 || batch->num_seqs == 0) return KV4_OK;
+  cudaError_t e = kv4::launch_append(v, static_cast<const uint16_t *>(k_new),
+                                     static_cast<const uint16_t *>(v_new), new_indptr, total_new,
+                                     err_flag, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool,
+                                const kv4_int8_side *side, const kv4_batch *batch, const void *q,
+                                void *out, float *out_f32, float *lse, void *workspace,
+                                size_t ws_bytes, int32_t *err_flag, kv4_stream_t stream) {
+  kv4::CacheView v;
+  kv4_status st = make_view(cfg, pool, side, batch, &v);
+  if (st != KV4_OK) return st;
+  if (batch->num_seqs == 0) return KV4_OK;
+  if (q == nullptr || out == nullptr || workspace == nullptr) return KV4_ERR_INVALID_ARG;
+  if (misaligned16(q) || misaligned16(out) || misaligned16(out_f32) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return KV4_ERR_INVALID_ARG;
+  kv4::Workspace w;
+  const size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads,
+                                           v.gqa, chunk_of(cfg), &w, workspace);
+  if (ws_bytes < need) return KV4_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  if (e == cudaSuccess) e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
+                          static_cast<uint16_t *>(out), out_f32, lse, s);
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offsets,
+                              int32_t n_units, int32_t group, int32_t head_dim, void *out,
+                              float *out_f32, float *lse, kv4_stream_t stream) {
+  if (n_units < 0 || group < 1 || group > kv4::kMaxGqa) return KV4_ERR_INVALID_ARG;
+  if (head_dim != kv4::kHeadDim) return KV4_ERR_UNSUPPORTED_SHAPE;
+  if (n_units == 0) return KV4_OK;
+  if (partials == nullptr || region_offsets == nullptr || out == nullptr)
+    return KV4_ERR_INVALID_ARG;
+  if (misaligned16(partials) || misaligned16(out) || misaligned16(out_f32))
+    return KV4_ERR_INVALID_ARG;
+  cudaError_t e = kv4::launch_merge(partials, region_offsets, n_units, group,
+                                    static_cast<uint16_t *>(out), out_f32, lse,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+const char *kv4_status_string(kv4_status status) {
+  switch (status) {
+    case KV4_OK: return "ok";
+    case KV4_ERR_INVALID_ARG: return "invalid argument";
+    case KV4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case KV4_ERR_PROTECTED_TOO_LARGE: return "protected set larger than 144 positions";
+    case KV4_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case KV4_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int32_t kv4_version(void) { return 100; }
+
+}  // extern "C"

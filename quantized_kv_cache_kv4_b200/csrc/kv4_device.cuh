@@ -1,0 +1,169 @@
+// Device-side building blocks shared by the kv4 kernels: shared-memory async bulk
+// copies with mbarrier completion, warp-level tensor-core MMA and ldmatrix, and the
+// nibble/byte -> fp16 unpack used on integer KV codes.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/kv4.h"
+
+namespace kv4 {
+
+constexpr int kHeadDim = 128;
+constexpr int kPage = 16;       // tokens per INT4 page and per INT8 tile
+constexpr int kGroup = 32;      // INT4 group length along head_dim
+constexpr int kMaxGqa = 8;      // query heads per kv head handled by one warp (MMA N = 8)
+constexpr int kRecordFloats = kHeadDim + 4;  // partial record: acc[128], m, l, pad, pad
+
+// Bytes of one (page, kv head) INT4 block and one (tile, kv head) INT8 block.
+constexpr int kInt4CodeBytes = kPage * kHeadDim / 2;  // 1024
+constexpr int kInt4ParamBytes = kPage * 4 * 2 * 2;    // 256: 16 slots x 4 groups x (scale,min)
+constexpr int kInt8CodeBytes = kPage * kHeadDim;      // 2048
+constexpr int kInt8ScaleBytes = kPage * 2;            // 32
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk async copy (global -> shared), completion counted in bytes
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One attempt; returns true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after `limit` attempts (each attempt itself blocks for a
+// hardware-chosen interval). Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint32_t limit = (1u << 22)) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global to
+// this CTA's shared memory; completes `bytes` transactions on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// warp-level tensor cores: D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col)
+// Fragment ownership, lane = 4*gid + tig:
+//   A: a01 = (row gid, k 2tig..+1), a23 = (row gid+8, k 2tig..+1),
+//      a45 = (row gid, k 2tig+8..+9), a67 = (row gid+8, k 2tig+8..+9)
+//   B: b01 = (k 2tig..+1, col gid), b23 = (k 2tig+8..+9, col gid)
+//   C: c0,c1 = (row gid, col 2tig..+1), c2,c3 = (row gid+8, col 2tig..+1)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a01, uint32_t a23, uint32_t a45,
+                                        uint32_t a67, uint32_t b01, uint32_t b23) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a01), "r"(a23), "r"(a45), "r"(a67), "r"(b01), "r"(b23));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// ---------------------------------------------------------------------------
+// integer code -> fp16 without conversion instructions.
+// binary16 with exponent field 25 (bits 0x6400) is 1024 + mantissa, so OR-ing a small
+// unsigned integer u <= 1023 into the mantissa gives exactly 1024 + u; subtracting
+// 1024 (or 1024 + 128 for offset-binary int8) is exact.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t h2_sub(uint32_t x, uint32_t y) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&y));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+
+constexpr uint32_t kMagic1024x2 = 0x64006400u;  // (1024.0, 1024.0)
+constexpr uint32_t kMagic1152x2 = 0x64806480u;  // (1152.0, 1152.0)
+
+// Nibbles i and i+4 of a 32-bit word (i in 0..3) as an fp16 pair (low = nibble i).
+template <int I>
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
+  uint32_t x = ((w >> (4 * I)) & 0x000F000Fu) | kMagic1024x2;
+  return h2_sub(x, kMagic1024x2);
+}
+
+// Two int8 codes (bytes SEL0 and SEL1 of w) as an fp16 pair.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+// sel picks [byte, 0x64, byte, 0x64] from (w ^ 0x80808080, 0x64646464)
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t s8_pair(uint32_t w_offset_binary) {
+  return h2_sub(prmt(w_offset_binary, 0x64646464u, SEL), kMagic1152x2);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t x) {
+  return __half22float2(*reinterpret_cast<__half2 *>(&x));
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// fp16 round-to-nearest-even with saturation to +-65504.
+__device__ __forceinline__ __half f16_sat(float x) {
+  return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
+}
+
+__device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {
+  if (flag) atomicOr(reinterpret_cast<unsigned int *>(flag), bit);
+}
+
+}  // namespace kv4

@@ -1,0 +1,62 @@
+// Internal launch interfaces between the C-ABI layer (kv4_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kv4.h"
+
+namespace kv4 {
+
+// Everything a kernel needs about the cache and the batch, by value.
+struct CacheView {
+  uint8_t *k_codes, *v_codes;
+  uint16_t *k_params, *v_params;
+  int32_t num_pages;
+  int8_t *sink_k, *sink_v;
+  uint16_t *sink_ks, *sink_vs;
+  int32_t num_sink_sets, sink_tiles;
+  int8_t *ring_k, *ring_v;
+  uint16_t *ring_ks, *ring_vs;
+  int32_t num_rings, ring_tiles;
+  const int32_t *page_table;
+  int32_t max_pages;
+  const int32_t *seq_lens;
+  const int32_t *sink_idx;
+  const int32_t *ring_idx;
+  int32_t num_seqs;
+  int32_t num_kv_heads;
+  int32_t gqa;  // query heads per kv head
+  int32_t num_sinks, num_recent;
+};
+
+// Workspace carve-up for one decode-attention call.
+struct Workspace {
+  int32_t *counter;       // [1] dynamic work counter (reset by the plan kernel)
+  int32_t *n_items;       // [1] work items = pairs * Hkv
+  int2 *pairs;            // [cap_pairs] (sequence, region index within the sequence)
+  int32_t *unit_offsets;  // [num_seqs*Hkv + 1] first partial record row of each (b, h)
+  float *partials;        // [cap_pairs*Hkv][gqa][kRecordFloats]
+  int32_t cap_pairs;
+  int32_t chunk_pages;
+};
+
+size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads,
+                       int32_t gqa, int32_t chunk_pages, Workspace *carve, void *base);
+
+cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
+                          const int32_t *new_indptr, int32_t total_new, int32_t *err_flag,
+                          cudaStream_t s);
+
+cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag,
+                        cudaStream_t s);
+
+cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
+                             int32_t *err_flag, cudaStream_t s);
+
+cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
+                         int32_t group, uint16_t *out, float *out_f32, float *lse,
+                         cudaStream_t s);
+
+}  // namespace kv4

@@ -1,0 +1,141 @@
+"""The C-ABI library loads, exports every symbol include/kv4.h declares, and validates
+arguments on the host (these calls return before touching CUDA, so they run without a
+GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kv4.h")
+
+
+@pytest.fixture(scope="module")
+def kv4():
+    from quantized_kv_cache_kv4_b200 import build
+    build.build()
+    from quantized_kv_cache_kv4_b200 import kv4 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kv4_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for want in ("kv4_quantize_append", "kv4_decode_attention", "kv4_regional_merge",
+                 "kv4_workspace_size", "kv4_status_string", "kv4_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(kv4):
+    lib = ctypes.CDLL(kv4.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", kv4.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (kv4_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings_and_version(kv4):
+    lib = kv4._lib
+    assert lib.kv4_version() == 100
+    assert lib.kv4_status_string(0) == b"ok"
+    assert b"144" in lib.kv4_status_string(-3)
+    assert lib.kv4_status_string(-99) == b"unknown status"
+
+
+def _cfg(kv4, **kw):
+    d = dict(num_q_heads=32, num_kv_heads=8, num_sinks=16, num_recent=128, chunk_pages=0)
+    d.update(kw)
+    return kv4.make_config(**d)
+
+
+def test_workspace_size_host_only(kv4):
+    c = _cfg(kv4)
+    n1 = kv4.workspace_size(c, 64, 2048)
+    n2 = kv4.workspace_size(c, 128, 2048)
+    assert 0 < n1 < n2
+    assert n1 % 256 == 0
+    # partial records dominate: >= 64 seqs * 8 heads * 4 q heads * 132 floats * (1 + chunks)
+    assert n1 >= 64 * 8 * 4 * 132 * 4 * (1 + 5)
+    bad = _cfg(kv4, num_sinks=100, num_recent=45)
+    assert kv4._lib.kv4_workspace_size(ctypes.byref(bad), 4, 100) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_sinks=16, num_recent=129), -3),
+    (dict(num_sinks=145, num_recent=0), -3),
+    (dict(num_q_heads=30), -2),
+    (dict(num_q_heads=128, num_kv_heads=8), -2),
+    (dict(chunk_pages=33), -2),
+    (dict(num_sinks=-1), -1),
+])
+def test_config_rejected_before_launch(kv4, kw, status):
+    c = _cfg(kv4, **kw)
+    pool, side, batch = kv4.Int4Pool(), kv4.Int8Side(), kv4.Batch()
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                       ctypes.byref(batch), None, None, None, None, None, 0,
+                                       None, None)
+    assert st == status
+    st = kv4._lib.kv4_quantize_append(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                      ctypes.byref(batch), None, None, None, 0, None, None)
+    assert st == status
+
+
+def test_bad_shapes_and_pointers_rejected(kv4):
+    c = _cfg(kv4)
+    c.head_dim = 64
+    pool, side, batch = kv4.Int4Pool(), kv4.Int8Side(), kv4.Batch()
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                       ctypes.byref(batch), None, None, None, None, None, 0,
+                                       None, None)
+    assert st == -2
+    c = _cfg(kv4)
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), None, None, None, None, None, None, None,
+                                       None, 0, None, None)
+    assert st == -1
+    # null pool pointers
+    batch = kv4.Batch(0, 4, 0, 0, 0, 2, 100)
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                       ctypes.byref(batch), None, None, None, None, None, 0,
+                                       None, None)
+    assert st == -1
+    # misaligned codes pointer
+    pool = kv4.Int4Pool(1 << 20 | 8, 1 << 20, 1 << 20, 1 << 20, 10)
+    batch = kv4.Batch(1 << 20, 4, 1 << 20, 1 << 20, 0, 2, 100)
+    side = kv4.Int8Side(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1 << 20, 1 << 20, 1 << 20,
+                        1 << 20, 1)
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                       ctypes.byref(batch), None, None, None, None, None, 0,
+                                       None, None)
+    assert st == -1
+
+
+def test_merge_argument_checks(kv4):
+    lib = kv4._lib
+    assert lib.kv4_regional_merge(None, None, 4, 4, 64, None, None, None, None) == -2
+    assert lib.kv4_regional_merge(None, None, 4, 0, 128, None, None, None, None) == -1
+    assert lib.kv4_regional_merge(None, None, 4, 9, 128, None, None, None, None) == -1
+    assert lib.kv4_regional_merge(None, None, 0, 4, 128, None, None, None, None) == 0
+    assert lib.kv4_regional_merge(None, None, 2, 4, 128, None, None, None, None) == -1
+
+
+def test_workspace_too_small_is_reported(kv4):
+    c = _cfg(kv4)
+    need = kv4.workspace_size(c, 2, 1000)
+    pool = kv4.Int4Pool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
+    side = kv4.Int8Side(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1 << 20, 1 << 20, 1 << 20,
+                        1 << 20, 2)
+    batch = kv4.Batch(1 << 20, 64, 1 << 20, 1 << 20, 0, 2, 1000)
+    st = kv4._lib.kv4_decode_attention(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                       ctypes.byref(batch), ctypes.c_void_p(1 << 20),
+                                       ctypes.c_void_p(1 << 20), None, None,
+                                       ctypes.c_void_p(1 << 20), need - 256, None, None)
+    assert st == -4

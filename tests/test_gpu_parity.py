@@ -1,0 +1,288 @@
+"""GPU parity: the CUDA library (called through its C ABI) against the CPU oracle.
+
+* INT4 pages, INT8 sink sets and rings: bit-exact, byte for byte.
+* Attention: fp32 output within 2e-3 x max|O_ref| (the tolerance stated for this path),
+  bf16 output within that plus half a bf16 ulp of the reference (bf16 rounding alone
+  can reach 2^-9 relative), LSE within 2e-3 x max(1, |lse_ref|).
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kv4_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from quantized_kv_cache_kv4_b200 import build
+    build.build()
+
+
+def _mods():
+    from quantized_kv_cache_kv4_b200 import kv4, session, workload
+    return kv4, session, workload
+
+
+def bf16_half_ulp(x):
+    a = np.abs(x)
+    e = np.floor(np.log2(np.maximum(a, 1e-38)))
+    return np.where(a > 0, 2.0 ** (e - 8), 2.0 ** -133)
+
+
+def oracle_out(sess, b, step=0):
+    k, v = sess.streams[b]
+    L = int(sess.L0[b]) + step
+    q = sess.q[step, b].float().cpu().numpy()
+    return O.decode_reference(q, k[:L], v[:L], sess.wl.num_sinks, sess.wl.num_recent)
+
+
+def run_attention(sess, step=0):
+    B, Hq = sess.wl.num_seqs, sess.wl.num_q_heads
+    out32 = torch.empty((B, Hq, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    sess.attention_step(step, out_f32=out32, lse=lse)
+    torch.cuda.synchronize()
+    return sess.out.float().cpu().numpy(), out32.cpu().numpy(), lse.cpu().numpy()
+
+
+def check_attention(sess, seqs, step=0, got=None):
+    o16, o32, lse = got if got is not None else run_attention(sess, step)
+    refs = {b: oracle_out(sess, b, step) for b in seqs}
+    scale = max(np.abs(r[0]).max() for r in refs.values())
+    worst = 0.0
+    for b, (oref, lref) in refs.items():
+        e32 = np.abs(o32[b] - oref).max()
+        worst = max(worst, e32 / scale)
+        assert e32 <= TOL * scale, (b, e32, scale)
+        e16 = np.abs(o16[b] - oref)
+        assert np.all(e16 <= TOL * scale + bf16_half_ulp(oref)), (b, e16.max())
+        assert np.all(np.abs(lse[b] - lref) <= TOL * np.maximum(1, np.abs(lref))), b
+    return worst
+
+
+def check_cache(sess, seqs):
+    """Bit-exact INT4 pages and INT8 side store of the given sequences (after step 0)."""
+    kv4, _, _ = _mods()
+    c = sess.cache
+    S, R = sess.wl.num_sinks, sess.wl.num_recent
+    kc, vc = c.k_codes.cpu().numpy(), c.v_codes.cpu().numpy()
+    kp, vp = c.k_params.cpu().numpy().view(np.uint16), c.v_params.cpu().numpy().view(np.uint16)
+    side = [t.cpu().numpy() for t in (c.sink_k, c.sink_ks, c.sink_v, c.sink_vs,
+                                      c.ring_k, c.ring_ks, c.ring_v, c.ring_vs)]
+    for b in seqs:
+        k, v = sess.streams[b]
+        L = int(sess.L0[b])
+        rec = O.token_records(k[:L], v[:L])
+        pages = O.expected_pages(rec, L, sess.paging.page_table[b])
+        for pid, (ekc, ekp, evc, evp) in pages.items():
+            assert np.array_equal(kc[pid], ekc), (b, pid)
+            assert np.array_equal(vc[pid], evc), (b, pid)
+            assert np.array_equal(kp[pid], ekp), (b, pid)
+            assert np.array_equal(vp[pid], evp), (b, pid)
+        exp = O.expected_side(rec, L, S, R)
+        if S > 0:
+            st = sess.paging.sink_idx[b]
+            assert np.array_equal(side[0][st], exp[0]), b
+            assert np.array_equal(side[1][st].view(np.uint16), exp[1]), b
+            assert np.array_equal(side[2][st], exp[2]), b
+            assert np.array_equal(side[3][st].view(np.uint16), exp[3]), b
+        if R > 0:
+            r = sess.paging.ring_idx[b]
+            assert np.array_equal(side[4][r], exp[4]), b
+            assert np.array_equal(side[5][r].view(np.uint16), exp[5]), b
+            assert np.array_equal(side[6][r], exp[6]), b
+            assert np.array_equal(side[7][r].view(np.uint16), exp[7]), b
+
+
+def make_session(wl, keep=None, **kw):
+    _, session, _ = _mods()
+    keep = range(wl.num_seqs) if keep is None else keep
+    s = session.DecodeSession(wl, keep_streams=keep, **kw)
+    s.append_step(0)
+    torch.cuda.synchronize()
+    return s
+
+
+# ----------------------------------------------------------------------------
+# small cases: everything compared
+# ----------------------------------------------------------------------------
+
+def test_tiny_workload_bit_exact_and_attention():
+    _, _, W = _mods()
+    sess = make_session(W.make_workload("tiny"))
+    check_cache(sess, range(4))
+    check_attention(sess, range(4))
+    sess.check_err()
+
+
+EDGE = [
+    # (name, lens, Hq, Hkv, S, R, chunk_pages)
+    ("short-boundaries", [1, 2, 4, 5, 16, 17, 36, 37, 38, 48, 49, 100], 8, 2, 4, 32, 0),
+    ("pure-int4", [1, 15, 16, 17, 200], 8, 2, 0, 0, 0),
+    ("pure-int8", [1, 16, 17, 143, 144], 8, 2, 16, 128, 0),
+    ("sinks-only", [100, 150, 300], 8, 2, 144, 0, 0),
+    ("recent-only", [100, 150, 300], 8, 2, 0, 144, 0),
+    ("gqa1", [40, 333], 4, 4, 4, 32, 0),
+    ("gqa2", [40, 333], 8, 4, 4, 32, 0),
+    ("gqa8", [40, 333], 16, 2, 4, 32, 0),
+    ("one-kv-head", [300, 77], 4, 1, 16, 128, 0),
+    ("chunk1", [700, 40, 260], 8, 2, 16, 128, 1),
+    ("chunk3", [700, 40, 260], 8, 2, 16, 128, 3),
+    ("odd-S-R", [23, 64, 511], 8, 2, 7, 13, 2),
+]
+
+
+@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,C", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_cases(name, lens, Hq, Hkv, S, R, C):
+    _, _, W = _mods()
+    wl = W.custom_workload(lens, num_q_heads=Hq, num_kv_heads=Hkv, num_sinks=S, num_recent=R,
+                           seed=zlib.crc32(name.encode()) & 0xFFFF, outlier_channels=2, outlier_scale=8.0)
+    sess = make_session(wl, chunk_pages=C)
+    check_cache(sess, range(len(lens)))
+    check_attention(sess, range(len(lens)))
+    sess.check_err()
+
+
+def test_shared_prefix_groups():
+    _, _, W = _mods()
+    wl = W.custom_workload([40, 70, 33, 100, 35, 64], num_sinks=4, num_recent=16, prompt_len=32,
+                           group_seqs=3, seed=99, outlier_channels=1, outlier_scale=10.0)
+    sess = make_session(wl)
+    assert sess.paging.page_table[0, 0] == sess.paging.page_table[1, 0]
+    check_cache(sess, range(6))
+    check_attention(sess, range(6))
+    sess.check_err()
+
+
+def test_heavy_tailed_values():
+    _, _, W = _mods()
+    wl = W.custom_workload([300, 901], num_q_heads=32, num_kv_heads=8, num_sinks=16,
+                           num_recent=128, seed=5, kv_dist="student_t3")
+    sess = make_session(wl)
+    check_cache(sess, range(2))
+    check_attention(sess, range(2))
+
+
+def test_several_decode_steps_demote_and_stay_exact():
+    """Steps 0..3 each append one token (demoting position L-R) and attend."""
+    _, session, W = _mods()
+    wl = W.custom_workload([37, 150, 161], num_sinks=4, num_recent=32, seed=3)
+    sess = session.DecodeSession(wl, steps=4, keep_streams=range(3))
+    for s in range(4):
+        sess.append_step(s)
+        torch.cuda.synchronize()
+        check_attention(sess, range(3), step=s)
+    sess.check_err()
+    # after the last step the cache equals appending positions [0, L0+3) one by one
+    sess.L0 = sess.L0 + 3
+    check_cache(sess, range(3))
+
+
+def test_empty_sequence_and_determinism():
+    kv4, _, W = _mods()
+    wl = W.custom_workload([50, 300], seed=11)
+    sess = make_session(wl)
+    lens = torch.tensor([0, 300], dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 8, 128), dtype=torch.bfloat16, device="cuda")
+    o32 = torch.empty((2, 8, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((2, 8), dtype=torch.float32, device="cuda")
+    kv4.decode_attention(sess.cache, sess.batch(lens), sess.q[0], out, sess.workspace, o32, lse,
+                         sess.err)
+    torch.cuda.synchronize()
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    first = o32.clone()
+    kv4.decode_attention(sess.cache, sess.batch(lens), sess.q[0], out, sess.workspace, o32, lse,
+                         sess.err)
+    torch.cuda.synchronize()
+    assert torch.equal(first, o32)  # bitwise deterministic
+    sess.check_err()
+
+
+def test_device_error_flags_without_faulting():
+    kv4, _, W = _mods()
+    wl = W.custom_workload([600, 600], seed=12)
+    sess = make_session(wl)
+    bad_table = sess.page_table.clone()
+    bad_table[1, 1] = sess.cache.num_pages + 7  # out of range page id in the INT4 region
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b = kv4.BatchTensors(bad_table, sess.step_lens[0], sess.sink_idx, sess.ring_idx, sess.max_len)
+    kv4.decode_attention(sess.cache, b, sess.q[0], sess.out, sess.workspace, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 1
+    err.zero_()
+    q = sess.q[0].clone()
+    q[0, 0, 0] = 1e5  # beyond fp16 range
+    kv4.decode_attention(sess.cache, sess.batch(sess.step_lens[0]), q, sess.out, sess.workspace,
+                         err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 8
+    # a workspace planned for shorter sequences overflows (3 regions per sequence needed,
+    # room for 2) -> flag, no fault
+    err.zero_()
+    small = kv4.BatchTensors(sess.page_table, sess.step_lens[0], sess.sink_idx, sess.ring_idx, 16)
+    ws = torch.empty(kv4.workspace_size(sess.cfg, 2, 16), dtype=torch.uint8, device="cuda")
+    kv4.decode_attention(sess.cache, small, sess.q[0], sess.out, ws, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 16
+
+
+def test_regional_merge_matches_oracle():
+    kv4, _, _ = _mods()
+    rng = np.random.default_rng(21)
+    G = 4
+    counts = [1, 3, 0, 7, 2, 20]
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    nreg = int(offs[-1])
+    part = np.zeros((nreg, G, 132), np.float32)
+    part[:, :, :128] = rng.normal(0, 3, (nreg, G, 128))
+    part[:, :, 128] = rng.normal(0, 4, (nreg, G))
+    part[:, :, 129] = rng.uniform(0.5, 30, (nreg, G))
+    part[4, 1, 128] = -np.inf  # an empty region
+    part[4, 1, 129] = 0
+    part[4, 1, :128] = 0
+    dev = lambda a: torch.as_tensor(a, device="cuda")
+    out = torch.empty((len(counts), G, 128), dtype=torch.bfloat16, device="cuda")
+    o32 = torch.empty((len(counts), G, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((len(counts), G), dtype=torch.float32, device="cuda")
+    kv4.regional_merge(dev(part), dev(offs), G, out, o32, lse)
+    torch.cuda.synchronize()
+    o32 = o32.cpu().numpy()
+    lse = lse.cpu().numpy()
+    for u in range(len(counts)):
+        for j in range(G):
+            parts = [(float(part[r, j, 128]), float(part[r, j, 129]), part[r, j, :128].astype(np.float64))
+                     for r in range(offs[u], offs[u + 1])]
+            if not parts:
+                assert np.all(o32[u, j] == 0) and np.isneginf(lse[u, j])
+                continue
+            want, wl = O.merge_partials(parts)
+            assert np.abs(o32[u, j] - want).max() <= 1e-5 * max(1, np.abs(want).max())
+            assert abs(lse[u, j] - wl) <= 1e-5 * max(1, abs(wl))
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads, sampled sequences (launch configuration of the benchmark)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,nsample", [("qwen3-8b-layer", 6), ("rollout", 10), ("longtail", 4)])
+def test_full_size_sampled(name, nsample):
+    _, _, W = _mods()
+    wl = W.make_workload(name)
+    rng = np.random.default_rng(7)
+    lens = wl.seq_lens
+    # the longest, the shortest and random others
+    pick = {int(np.argmax(lens)), int(np.argmin(lens))}
+    pick |= set(rng.choice(wl.num_seqs, nsample, replace=False).tolist())
+    sess = make_session(wl, keep=sorted(pick))
+    check_cache(sess, sorted(pick))
+    w1 = check_attention(sess, sorted(pick))
+    sess.check_err()
+    print(f"{name}: worst error / scale = {w1:.2e}")
