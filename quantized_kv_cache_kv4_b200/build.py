@@ -28,7 +28,8 @@ def flags(verbose: bool = False):
          "-Xcompiler", "-fvisibility=default", "--expt-relaxed-constexpr"]
     if verbose:
         f += ["-Xptxas", "-v"]
-    return f
+    extra = os.environ.get("KV4_NVCC_FLAGS", "").split()
+    return f + extra
 
 
 def _stale() -> bool:

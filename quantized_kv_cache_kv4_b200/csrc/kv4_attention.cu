@@ -214,6 +214,12 @@ __device__ __forceinline__ float q_to_f16_pair(uint32_t bf2, uint32_t &out, bool
 }
 
 // ---------------------------- INT4 chunk --------------------------------
+// Token order of the QK^T M-tile rows: rows 0-7 are tokens 0-7, rows 8-11 tokens 12-15,
+// rows 12-15 tokens 8-11. With it a thread's two rows (gid, gid+8) are the tokens whose
+// P' values it packs into one 32-bit word, the transposed V loads read those pairs, and
+// neither the K nor the V ldmatrix phases hit a shared-memory bank twice.
+__device__ __forceinline__ int row_token_hi(int r) { return 8 + ((r + 4) & 7); }
+
 __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
                              const uint16_t *__restrict__ q, int b, int h, int chunk,
                              const Regions &rg, float *rec, int32_t *err) {
@@ -251,7 +257,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   const int npre = min(np, kStages);
   for (int k = 0; k < npre; ++k) issue(k);
 
-  // ---- query fragments (B operand of QK^T), head gid, k-slot order matching nib_pair ----
+  // ---- query fragments (B operand of QK^T), head gid, k-slot order matching nib_pairs4 ----
   // group g, k-tile kt: b01 = (q[32g+8tig+2kt], q[..+4]), b23 = (q[..+2kt+1], q[..+2kt+5])
   uint32_t qb[4][2][2];
   float qsum_own[4];
@@ -262,7 +268,6 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
-      // pairs (d, d+4): (0,4) (1,5) (2,6) (3,7)
       const uint32_t p04 = (v.x & 0xFFFFu) | (v.z << 16);
       const uint32_t p15 = (v.x >> 16) | (v.z & 0xFFFF0000u);
       const uint32_t p26 = (v.y & 0xFFFFu) | (v.w << 16);
@@ -278,34 +283,42 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     }
   }
   if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
-  float qsum[4][2];  // for this thread's C-fragment heads 2tig, 2tig+1
+  float2 qs[4];  // (head 2tig, head 2tig+1) sums, matching the C-fragment columns
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    qsum[g][0] = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig));
-    qsum[g][1] = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig + 1));
+    qs[g].x = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig));
+    qs[g].y = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig + 1));
   }
 
   float m[2] = {kNegBig, kNegBig}, l[2] = {0.f, 0.f};
-  float o[4][2][4];
-  float mt[4][2];
+  // o[g][mt][e] = (dim 32g+4gid+2mt, dim +1) of head 2tig+e
+  float2 o[4][2][2];
+  float2 mtp[4][2];  // sum p * vmin per group and head, split over the thread's two tokens
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    mt[g][0] = mt[g][1] = 0.f;
+  for (int g = 0; g < 4; ++g)
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[g][t][i] = 0.f;
-  }
+    for (int e = 0; e < 2; ++e) {
+      mtp[g][e] = make_float2(0.f, 0.f);
+      o[g][0][e] = make_float2(0.f, 0.f);
+      o[g][1][e] = make_float2(0.f, 0.f);
+    }
 
-  // ldmatrix lane address inside a 512-byte pair of strips: matrix m = lane/8 is
-  // (strip m/2, tokens 8*(m%2) .. +7), row r = lane%8
-  const int ld_off = ((lane >> 4) * 256) + ((lane >> 3) & 1) * 128 + (lane & 7) * 16;
+  // ldmatrix lane addresses: matrix m = lane/8 covers strip m/2 (256 B each), row r = lane%8
+  const int r8 = lane & 7;
+  const int mhalf = (lane >> 3) & 1;
+  const int strip_off = (lane >> 4) * 256;
+  const int ld_k = strip_off + (mhalf ? row_token_hi(r8) : r8) * 16;
+  // transposed V: matrix "lo" rows (2i, 2i+1) = tokens (i, 12+i), "hi" = (4+i, 8+i)
+  const int ld_v = strip_off + (mhalf ? ((r8 & 1) ? 8 + (r8 >> 1) : 4 + (r8 >> 1))
+                                      : ((r8 & 1) ? 12 + (r8 >> 1) : (r8 >> 1))) * 16;
+  const int t0 = gid, t1 = row_token_hi(gid);  // tokens of this thread's C rows gid, gid+8
   const int tok_lo = rg.int4_lo, tok_hi = rg.int4_hi;
+  uint32_t *ptw = reinterpret_cast<uint32_t *>(x.ptile);  // [4 g][8 heads][8 token pairs]
+  const float2 kappa = make_float2(kLog2e * 0.08838834764831845f, kLog2e * 0.08838834764831845f);
 
   for (int k = 0; k < np; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      // give the copies already issued a bounded chance to land, then abandon the item
       for (int kk = k + 1; kk < min(np, k + kStages); ++kk) wait_stage(x, kk % kStages, err);
       write_empty(rec, G, lane);
       return;
@@ -315,103 +328,130 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 
     // ---- S^T = K Q^T, one fp32 accumulator per 32-dim group ----
     uint32_t kw[2][4];
-    ldsm_x4(kw[0], sa + ld_off);
-    ldsm_x4(kw[1], sa + 512 + ld_off);
+    ldsm_x4(kw[0], sa + ld_k);
+    ldsm_x4(kw[1], sa + 512 + ld_k);
     float acc[4][4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const uint32_t wlo = kw[g >> 1][(g & 1) * 2], whi = kw[g >> 1][(g & 1) * 2 + 1];
+      uint32_t pl[4], ph[4];
+      nib_pairs4(kw[g >> 1][(g & 1) * 2], pl);
+      nib_pairs4(kw[g >> 1][(g & 1) * 2 + 1], ph);
       acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-      mma_f16(acc[g], nib_pair<0>(wlo), nib_pair<0>(whi), nib_pair<1>(wlo), nib_pair<1>(whi),
-              qb[g][0][0], qb[g][0][1]);
-      mma_f16(acc[g], nib_pair<2>(wlo), nib_pair<2>(whi), nib_pair<3>(wlo), nib_pair<3>(whi),
-              qb[g][1][0], qb[g][1][1]);
+      mma_f16(acc[g], pl[0], ph[0], pl[1], ph[1], qb[g][0][0], qb[g][0][1]);
+      mma_f16(acc[g], pl[2], ph[2], pl[3], ph[3], qb[g][1][0], qb[g][1][1]);
     }
-    // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), in log2 units ----
-    const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffKp4 + gid * 16),
-                         *reinterpret_cast<const uint4 *>(sp + kOffKp4 + (gid + 8) * 16)};
-    float s[2][2];
-    const int tok0 = (p0 + k) * kPage;
+    // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
+    const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffKp4 + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + kOffKp4 + t1 * 16)};
+    float2 sl[2];  // sl[hf] = logits of token (t0 | t1) for heads (2tig, 2tig+1)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const uint32_t pw[4] = {kp[hf].x, kp[hf].y, kp[hf].z, kp[hf].w};
-      const int t = tok0 + gid + 8 * hf;
-      const bool valid = t >= tok_lo && t < tok_hi;
+      float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float v = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float2 sm = h2_to_f2(pw[g]);
-          v = fmaf(sm.x, acc[g][2 * hf + e], v);
-          v = fmaf(sm.y, qsum[g][e], v);
-        }
-        s[hf][e] = valid ? v * (kLog2e * 0.08838834764831845f) : -CUDART_INF_F;
+      for (int g = 0; g < 4; ++g) {
+        const float2 sm = h2_to_f2(pw[g]);
+        v = ffma2(make_float2(sm.x, sm.x), make_float2(acc[g][2 * hf], acc[g][2 * hf + 1]), v);
+        v = ffma2(make_float2(sm.y, sm.y), qs[g], v);
       }
+      sl[hf] = fmul2(v, kappa);
     }
-    float alpha[2];
-    softmax_step(s, m, l, alpha);
+    const int tok0 = (p0 + k) * kPage;
+    if (tok0 < tok_lo || tok0 + kPage > tok_hi) {  // ragged first/last page of the range
+      const bool v0 = tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi;
+      const bool v1 = tok0 + t1 >= tok_lo && tok0 + t1 < tok_hi;
+      if (!v0) sl[0] = make_float2(-CUDART_INF_F, -CUDART_INF_F);
+      if (!v1) sl[1] = make_float2(-CUDART_INF_F, -CUDART_INF_F);
+    }
+    // ---- online softmax; the rescale is skipped while no running max moves ----
+    float p[2][2];
+    float2 alpha2[2];
+    bool moved = false;
 #pragma unroll
-    for (int g = 0; g < 4; ++g)
+    for (int e = 0; e < 2; ++e) {
+      const float s0 = e ? sl[0].y : sl[0].x, s1 = e ? sl[1].y : sl[1].x;
+      float t = fmaxf(s0, s1);
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+      const float mn = fmaxf(m[e], t);
+      const float a = mn != m[e] ? fast_exp2(m[e] - mn) : 1.0f;
+      moved |= mn != m[e];
+      m[e] = mn;
+      p[0][e] = fast_exp2(s0 - mn);
+      p[1][e] = fast_exp2(s1 - mn);
+      l[e] = fmaf(l[e], a, p[0][e] + p[1][e]);
+      alpha2[e] = make_float2(a, a);
+    }
+    if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        mt[g][e] *= alpha[e];
+      for (int g = 0; g < 4; ++g)
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          o[g][t][e] *= alpha[e];
-          o[g][t][2 + e] *= alpha[e];
+        for (int e = 0; e < 2; ++e) {
+          mtp[g][e] = fmul2(mtp[g][e], alpha2[e]);
+          o[g][0][e] = fmul2(o[g][0][e], alpha2[e]);
+          o[g][1][e] = fmul2(o[g][1][e], alpha2[e]);
         }
-      }
-    // ---- P'_g = p * vscale_g (fp16) to the P' tile; sum p * vmin_g on the side ----
-    const uint4 vp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffVp4 + gid * 16),
-                         *reinterpret_cast<const uint4 *>(sp + kOffVp4 + (gid + 8) * 16)};
+    }
+    // ---- P'_g = p * vscale_g as fp16 token pairs; sum p * vmin_g on the side ----
+    const uint4 vp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffVp4 + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + kOffVp4 + t1 * 16)};
+    const float2 pe[2] = {make_float2(p[0][0], p[1][0]), make_float2(p[0][1], p[1][1])};
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const uint32_t w0 = g == 0 ? vp[0].x : g == 1 ? vp[0].y : g == 2 ? vp[0].z : vp[0].w;
       const uint32_t w1 = g == 0 ? vp[1].x : g == 1 ? vp[1].y : g == 2 ? vp[1].z : vp[1].w;
-      const float2 sv0 = h2_to_f2(w0), sv1 = h2_to_f2(w1);
+      const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
+      const float2 sv = make_float2(f0.x, f1.x), mv = make_float2(f0.y, f1.y);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int j = 2 * tig + e;
-        if (j < G) {
-          x.ptile[(g * 8 + j) * 16 + gid] = __half_as_ushort(__float2half_rn(s[0][e] * sv0.x));
-          x.ptile[(g * 8 + j) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(s[1][e] * sv1.x));
-        }
-        mt[g][e] = fmaf(s[0][e], sv0.y, fmaf(s[1][e], sv1.y, mt[g][e]));
+        const float2 pv = fmul2(pe[e], sv);
+        if (j < G) ptw[(g * 8 + j) * 8 + gid] = pack_h2(pv.x, pv.y);
+        mtp[g][e] = ffma2(pe[e], mv, mtp[g][e]);
       }
     }
     __syncwarp();
-    // ---- O^T += V^T P' per group: A = V codes (via transposed ldmatrix), B = P'_g ----
+    // ---- O^T += V^T P' per group: A = V codes (transposed ldmatrix), B = P'_g ----
     uint32_t vw[2][4];
-    ldsm_x4_t(vw[0], sa + kOffVc4 + ld_off);
-    ldsm_x4_t(vw[1], sa + kOffVc4 + 512 + ld_off);
+    ldsm_x4_t(vw[0], sa + kOffVc4 + ld_v);
+    ldsm_x4_t(vw[1], sa + kOffVc4 + 512 + ld_v);
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const uint32_t xlo = vw[g >> 1][(g & 1) * 2], xhi = vw[g >> 1][(g & 1) * 2 + 1];
+      uint32_t vl[4], vh[4];
+      nib_pairs4(vw[g >> 1][(g & 1) * 2], vl);
+      nib_pairs4(vw[g >> 1][(g & 1) * 2 + 1], vh);
       uint32_t b01 = 0, b23 = 0;
       if (gid < G) {
-        b01 = *reinterpret_cast<const uint32_t *>(&x.ptile[(g * 8 + gid) * 16 + 2 * tig]);
-        b23 = *reinterpret_cast<const uint32_t *>(&x.ptile[(g * 8 + gid) * 16 + 2 * tig + 8]);
+        b01 = ptw[(g * 8 + gid) * 8 + tig];
+        b23 = ptw[(g * 8 + gid) * 8 + tig + 4];
       }
-      mma_f16(o[g][0], nib_pair<0>(xlo), nib_pair<1>(xlo), nib_pair<0>(xhi), nib_pair<1>(xhi), b01,
-              b23);
-      mma_f16(o[g][1], nib_pair<2>(xlo), nib_pair<3>(xlo), nib_pair<2>(xhi), nib_pair<3>(xhi), b01,
-              b23);
+      float c0[4] = {o[g][0][0].x, o[g][0][1].x, o[g][0][0].y, o[g][0][1].y};
+      mma_f16(c0, vl[0], vl[1], vh[0], vh[1], b01, b23);
+      o[g][0][0] = make_float2(c0[0], c0[2]);
+      o[g][0][1] = make_float2(c0[1], c0[3]);
+      float c1[4] = {o[g][1][0].x, o[g][1][1].x, o[g][1][0].y, o[g][1][1].y};
+      mma_f16(c1, vl[2], vl[3], vh[2], vh[3], b01, b23);
+      o[g][1][0] = make_float2(c1[0], c1[2]);
+      o[g][1][1] = make_float2(c1[1], c1[3]);
     }
     __syncwarp();
     if (k + kStages < np) issue(k + kStages);
   }
 
   // ---- finish: reduce per-thread sums over the 8 token lanes, write the partial ----
+  float mt[4][2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], off);
 #pragma unroll
-    for (int g = 0; g < 4; ++g)
+    for (int g = 0; g < 4; ++g) {
+      mt[g][e] = mtp[g][e].x + mtp[g][e].y;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1)
         mt[g][e] += __shfl_xor_sync(0xffffffffu, mt[g][e], off);
+    }
   }
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -420,9 +460,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
       float *r = rec + j * kRecordFloats;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        // rows: dim 32g+4gid+2t (c0/c1) and +1 (c2/c3)
-        const float4 v = make_float4(o[g][0][e] + mt[g][e], o[g][0][2 + e] + mt[g][e],
-                                     o[g][1][e] + mt[g][e], o[g][1][2 + e] + mt[g][e]);
+        const float4 v = make_float4(o[g][0][e].x + mt[g][e], o[g][0][e].y + mt[g][e],
+                                     o[g][1][e].x + mt[g][e], o[g][1][e].y + mt[g][e]);
         *reinterpret_cast<float4 *>(r + 32 * g + 4 * gid) = v;
       }
       if (gid == 0) {
@@ -607,7 +646,11 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   }
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 4) attn_kernel(CacheView c, Workspace w,
+#ifndef KV4_MIN_BLOCKS
+#define KV4_MIN_BLOCKS 4  // CTAs per SM the register budget is sized for
+#endif
+
+__global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(CacheView c, Workspace w,
                                                               const uint16_t *__restrict__ q,
                                                               int32_t *err) {
   extern __shared__ __align__(1024) uint8_t smem[];

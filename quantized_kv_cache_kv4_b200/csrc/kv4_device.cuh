@@ -132,6 +132,50 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
   return h2_sub(x, kMagic1024x2);
 }
 
+__device__ __forceinline__ uint32_t h2_fma(uint32_t x, uint32_t y, uint32_t z) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&y),
+                      *reinterpret_cast<__half2 *>(&z));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+
+constexpr uint32_t kSixteenthX2 = 0x2C002C00u;  // (1/16, 1/16)
+constexpr uint32_t kMinus64X2 = 0xD400D400u;    // (-64, -64)
+
+// All four nibble pairs of a word with one shift: pairs 0 and 2 sit in the low
+// mantissa bits (1024 + c, exact after subtracting 1024); pairs 1 and 3 are masked in
+// place as 1024 + 16c and brought back exactly by x/16 - 64 in one fma.
+// Returns p[i] = (nibble i, nibble i+4) as fp16 pairs.
+__device__ __forceinline__ void nib_pairs4(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2_sub((w & 0x000F000Fu) | kMagic1024x2, kMagic1024x2);
+  p[1] = h2_fma((w & 0x00F000F0u) | kMagic1024x2, kSixteenthX2, kMinus64X2);
+  p[2] = h2_sub((w8 & 0x000F000Fu) | kMagic1024x2, kMagic1024x2);
+  p[3] = h2_fma((w8 & 0x00F000F0u) | kMagic1024x2, kSixteenthX2, kMinus64X2);
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32 pairs (sm_100 f32x2 FMA pipe operations)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
 // Two int8 codes (bytes SEL0 and SEL1 of w) as an fp16 pair.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
