@@ -4,17 +4,21 @@
 // merge", ai4snews summary, "Interpretation" para. 3).
 //
 // Kernels:
-//   plan_kernel  one CTA: turns seq_lens into a work list of (sequence, region) pairs
-//                -- region 0 is the INT8 protected set, regions 1.. are chunks of
-//                `chunk_pages` INT4 pages -- and the partial-record offsets per (b, h).
-//   attn_kernel  persistent; every warp repeatedly takes one (pair, kv head) item from
-//                an atomic counter and computes that region's partial state for the G
-//                query heads of the kv head. Page tiles stream through a per-warp ring
-//                of shared-memory stages filled by bulk async copies (TMA engine,
-//                mbarrier completion). QK^T and PV run on the tensor cores
-//                (mma m16n8k16, fp16 in, fp32 accumulate) directly on the integer codes:
-//                codes are exact in fp16, and the per-group scale/min are applied
-//                outside the dot products, so no dequantised K/V is ever materialised.
+//   plan_kernel  one CTA: turns seq_lens into a work list. Region 0 of a sequence is its
+//                INT8 protected set (one entry per kv head); regions 1.. are chunks of
+//                `chunk_pages` INT4 pages (one entry per one or two kv heads).
+//   attn_kernel  persistent; every warp repeatedly takes one entry from an atomic counter
+//                and computes the partial softmax state of that region for the query
+//                heads of its kv head(s). Page tiles stream through a per-warp ring of
+//                shared-memory stages filled by bulk async copies (TMA engine, mbarrier
+//                completion). QK^T and PV run on the tensor cores (mma m16n8k16, fp16 in,
+//                fp32 accumulate) directly on the integer codes: codes are exact in fp16,
+//                and the per-group scale/min are applied outside the dot products, so no
+//                dequantised K/V is ever materialised.
+//                With G <= 4 query heads per kv head one warp serves two kv heads: the MMA
+//                N dimension (8) holds head A's queries in columns 0-3 and head B's in
+//                columns 4-7 (zeros in the other half of each B operand), so every lane's
+//                softmax and scaling work is useful.
 //   merge_kernel one warp per (b, h, query head): fixed-order exact merge -> bf16 out.
 #include <math_constants.h>
 
@@ -25,16 +29,17 @@ namespace kv4 {
 
 constexpr int kWarps = 4;                 // warps per CTA (independent work streams)
 constexpr int kStages = 3;                // shared-memory stages per warp
-constexpr int kStageBytes = 4224;         // >= one INT8 tile (4160 B), multiple of 128
-constexpr int kPtileBytes = 4 * 8 * 16 * 2;  // P' tile: [4 groups][8 heads][16 tokens] fp16
-constexpr int kWarpSmem = kStages * kStageBytes + kPtileBytes + 64;
+constexpr int kStageBytes = 5120;         // two kv heads' INT4 page blocks; >= one INT8 tile
+constexpr int kPWordsPerCol = 12;         // P' tile column stride in words (bank-conflict free)
+constexpr int kPtileBytes = 2 * 4 * 8 * kPWordsPerCol * 4;  // [2 slots][4 groups][8 cols][12 w]
+constexpr int kPtile8Bytes = 8 * 16 * 2;  // INT8 P': [8 heads][16 tokens] fp16
+constexpr int kWarpSmem = kStages * kStageBytes + kPtileBytes + kPtile8Bytes + 64;
 constexpr int kCtaSmem = kWarps * kWarpSmem;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegBig = -1.0e30f;  // running-max start: finite, so e^(m_old-m_new) is 0 not NaN
+constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
-// INT4 stage: K codes | V codes | K params | V params
-constexpr int kOffVc4 = 1024, kOffKp4 = 2048, kOffVp4 = 2304, kInt4Bytes = 2560;
 // INT8 stage: K codes | V codes | K scales | V scales
 constexpr int kOffVc8 = 2048, kOffKs8 = 4096, kOffVs8 = 4128, kInt8Bytes = 4160;
 
@@ -48,8 +53,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // region bookkeeping shared by plan and attention
 // ---------------------------------------------------------------------------
 struct Regions {
-  int has_prot;     // 1 if the INT8 protected set is non-empty
-  int first_page;   // first page of the INT4 range
+  int has_prot;          // 1 if the INT8 protected set is non-empty
+  int first_page;        // first page of the INT4 range
   int int4_lo, int4_hi;  // INT4 token range [lo, hi)
   int n_chunks;
 };
@@ -98,47 +103,59 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
   __shared__ int sh[kPlanThreads];
   const int B = c.num_seqs, H = c.num_kv_heads, C = w.chunk_pages;
   const int S = c.num_sinks, R = c.num_recent;
-  // pass 1: total number of pairs
-  int carry = 0;
+  const int hpw = w.heads_per_warp;
+  const int nslots = (H + hpw - 1) / hpw;
+  auto counts = [&](int b, int &pairs, int &ents, bool flag) {
+    pairs = ents = 0;
+    if (b >= B) return;
+    int L = c.seq_lens[b];
+    if (L < 0 || L > c.max_pages * kPage) {
+      if (flag) set_err(err, KV4_DEVERR_SEQ_LEN);
+      L = 0;
+    }
+    const Regions g = regions_of(L, S, R, C);
+    pairs = g.has_prot + g.n_chunks;
+    ents = g.has_prot * H + g.n_chunks * nslots;
+  };
+  // pass 1: totals
+  int tp = 0, te = 0;
+  for (int base = 0; base < B; base += kPlanThreads) {
+    int p, e, t;
+    counts(base + threadIdx.x, p, e, false);
+    block_exclusive_scan(p, sh, &t);
+    tp += t;
+    block_exclusive_scan(e, sh, &t);
+    te += t;
+  }
+  const bool fits = tp <= w.cap_pairs && te <= w.cap_entries;
+  // pass 2: entries and partial offsets (all units empty if the workspace is too small)
+  int run_p = 0, run_e = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    int items = 0;
+    int p, e, t;
+    counts(b, p, e, true);
+    if (!fits) p = e = 0;
+    const int po = run_p + block_exclusive_scan(p, sh, &t);
+    run_p += t;
+    int eo = run_e + block_exclusive_scan(e, sh, &t);
+    run_e += t;
     if (b < B) {
       int L = c.seq_lens[b];
       if (L < 0 || L > c.max_pages * kPage) L = 0;
-      Regions g = regions_of(L, S, R, C);
-      items = g.has_prot + g.n_chunks;
-    }
-    int tot;
-    block_exclusive_scan(items, sh, &tot);
-    carry += tot;
-  }
-  const bool fits = carry <= w.cap_pairs;
-  // pass 2: write pairs and offsets (all-empty units if the workspace is too small)
-  int run = 0;
-  for (int base = 0; base < B; base += kPlanThreads) {
-    const int b = base + threadIdx.x;
-    int items = 0;
-    if (b < B) {
-      int L = c.seq_lens[b];
-      if (L < 0 || L > c.max_pages * kPage) {
-        set_err(err, KV4_DEVERR_SEQ_LEN);
-        L = 0;
+      const Regions g = regions_of(L, S, R, C);
+      if (p > 0) {
+        if (g.has_prot)
+          for (int h = 0; h < H; ++h) w.entries[eo++] = make_int4(b, 0, h, 1);
+        for (int ch = 0; ch < g.n_chunks; ++ch)
+          for (int s = 0; s < nslots; ++s)
+            w.entries[eo++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
       }
-      Regions g = regions_of(L, S, R, C);
-      items = fits ? g.has_prot + g.n_chunks : 0;
+      for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * p;
     }
-    int tot;
-    const int off = run + block_exclusive_scan(items, sh, &tot);
-    if (b < B) {
-      for (int r = 0; r < items; ++r) w.pairs[off + r] = make_int2(b, r);
-      for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * off + h * items;
-    }
-    run += tot;
   }
   if (threadIdx.x == 0) {
-    w.unit_offsets[B * H] = H * run;
-    *w.n_items = run * H;
+    w.unit_offsets[B * H] = H * run_p;
+    *w.n_items = run_e;
     *w.counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
   }
@@ -149,7 +166,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
 // ---------------------------------------------------------------------------
 struct WarpCtx {
   uint8_t *stage0;     // first stage (generic pointer)
-  uint16_t *ptile;     // P' tile
+  uint32_t *ptile;     // INT4 P' tile [2 slots][4 groups][8 cols][12 words], zero padded
+  uint16_t *ptile8;    // INT8 P' tile [8 heads][16 tokens]
   uint64_t *bars;      // kStages mbarriers
   uint32_t parity;     // bit s = parity of the next completion of stage s
   int lane, gid, tig;
@@ -185,7 +203,7 @@ __device__ __forceinline__ bool wait_stage(WarpCtx &x, int stage, int32_t *err) 
   return ok;
 }
 
-// Write the empty partial state (-inf, 0, 0) for the G heads of an item.
+// Write the empty partial state (-inf, 0, 0) for the G heads of a record group.
 __device__ void write_empty(float *rec, int G, int lane) {
   for (int j = 0; j < G; ++j) {
     float *r = rec + j * kRecordFloats;
@@ -197,13 +215,17 @@ __device__ void write_empty(float *rec, int G, int lane) {
   }
 }
 
-// Load this lane's query values: head gid (zero if gid >= G), dims off..off+7 for the
-// given offsets, converted to fp16 (exact for |q| in fp16's normal range).
+__device__ __forceinline__ float *record_of(const Workspace &w, int H, int G, int b, int h, int r) {
+  return w.partials + static_cast<size_t>(w.unit_offsets[b * H + h] + r) * G * kRecordFloats;
+}
+
 __device__ __forceinline__ uint4 load_q8(const uint16_t *qrow, int dim0, bool live) {
   if (!live) return make_uint4(0, 0, 0, 0);
   return *reinterpret_cast<const uint4 *>(qrow + dim0);
 }
 
+// bf16 pair -> fp16 pair (exact for |q| in fp16's normal range); returns the sum of the
+// two fp16 values and flags magnitudes beyond fp16.
 __device__ __forceinline__ float q_to_f16_pair(uint32_t bf2, uint32_t &out, bool &bad) {
   const float lo = __uint_as_float(bf2 << 16);
   const float hi = __uint_as_float(bf2 & 0xFFFF0000u);
@@ -213,266 +235,8 @@ __device__ __forceinline__ float q_to_f16_pair(uint32_t bf2, uint32_t &out, bool
   return back.x + back.y;
 }
 
-// ---------------------------- INT4 chunk --------------------------------
-// Token order of the QK^T M-tile rows: rows 0-7 are tokens 0-7, rows 8-11 tokens 12-15,
-// rows 12-15 tokens 8-11. With it a thread's two rows (gid, gid+8) are the tokens whose
-// P' values it packs into one 32-bit word, the transposed V loads read those pairs, and
-// neither the K nor the V ldmatrix phases hit a shared-memory bank twice.
-__device__ __forceinline__ int row_token_hi(int r) { return 8 + ((r + 4) & 7); }
-
-__device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
-                             const uint16_t *__restrict__ q, int b, int h, int chunk,
-                             const Regions &rg, float *rec, int32_t *err) {
-  const int G = c.gqa, H = c.num_kv_heads;
-  const int lane = x.lane, gid = x.gid, tig = x.tig;
-  const int p0 = rg.first_page + chunk * w.chunk_pages;
-  const int last = (rg.int4_hi - 1) / kPage;
-  const int np = min(w.chunk_pages, last - p0 + 1);
-
-  int pid = 0;
-  if (lane < np) pid = c.page_table[static_cast<size_t>(b) * c.max_pages + p0 + lane];
-  const bool bad = lane < np && (pid < 0 || pid >= c.num_pages);
-  if (__any_sync(0xffffffffu, bad)) {
-    if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
-    write_empty(rec, G, lane);
-    return;
-  }
-
-  auto issue = [&](int k) {
-    const int pk = __shfl_sync(0xffffffffu, pid, k);
-    if (lane == 0) {
-      const int st = k % kStages;
-      uint8_t *dst = x.stage0 + st * kStageBytes;
-      const size_t blk = static_cast<size_t>(pk) * H + h;
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&x.bars[st], kInt4Bytes);
-      bulk_g2s(dst, c.k_codes + blk * kInt4CodeBytes, kInt4CodeBytes, &x.bars[st]);
-      bulk_g2s(dst + kOffVc4, c.v_codes + blk * kInt4CodeBytes, kInt4CodeBytes, &x.bars[st]);
-      bulk_g2s(dst + kOffKp4, reinterpret_cast<const uint8_t *>(c.k_params) + blk * kInt4ParamBytes,
-               kInt4ParamBytes, &x.bars[st]);
-      bulk_g2s(dst + kOffVp4, reinterpret_cast<const uint8_t *>(c.v_params) + blk * kInt4ParamBytes,
-               kInt4ParamBytes, &x.bars[st]);
-    }
-  };
-  const int npre = min(np, kStages);
-  for (int k = 0; k < npre; ++k) issue(k);
-
-  // ---- query fragments (B operand of QK^T), head gid, k-slot order matching nib_pairs4 ----
-  // group g, k-tile kt: b01 = (q[32g+8tig+2kt], q[..+4]), b23 = (q[..+2kt+1], q[..+2kt+5])
-  uint32_t qb[4][2][2];
-  float qsum_own[4];
-  bool qbad = false;
-  {
-    const bool live = gid < G;
-    const uint16_t *qrow = q + (static_cast<size_t>(b) * c.num_kv_heads * G + h * G + gid) * kHeadDim;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
-      const uint32_t p04 = (v.x & 0xFFFFu) | (v.z << 16);
-      const uint32_t p15 = (v.x >> 16) | (v.z & 0xFFFF0000u);
-      const uint32_t p26 = (v.y & 0xFFFFu) | (v.w << 16);
-      const uint32_t p37 = (v.y >> 16) | (v.w & 0xFFFF0000u);
-      float sum = 0.f;
-      sum += q_to_f16_pair(p04, qb[g][0][0], qbad);
-      sum += q_to_f16_pair(p15, qb[g][0][1], qbad);
-      sum += q_to_f16_pair(p26, qb[g][1][0], qbad);
-      sum += q_to_f16_pair(p37, qb[g][1][1], qbad);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      qsum_own[g] = sum;  // sum over the group's 32 dims for head gid
-    }
-  }
-  if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
-  float2 qs[4];  // (head 2tig, head 2tig+1) sums, matching the C-fragment columns
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    qs[g].x = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig));
-    qs[g].y = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig + 1));
-  }
-
-  float m[2] = {kNegBig, kNegBig}, l[2] = {0.f, 0.f};
-  // o[g][mt][e] = (dim 32g+4gid+2mt, dim +1) of head 2tig+e
-  float2 o[4][2][2];
-  float2 mtp[4][2];  // sum p * vmin per group and head, split over the thread's two tokens
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      mtp[g][e] = make_float2(0.f, 0.f);
-      o[g][0][e] = make_float2(0.f, 0.f);
-      o[g][1][e] = make_float2(0.f, 0.f);
-    }
-
-  // ldmatrix lane addresses: matrix m = lane/8 covers strip m/2 (256 B each), row r = lane%8
-  const int r8 = lane & 7;
-  const int mhalf = (lane >> 3) & 1;
-  const int strip_off = (lane >> 4) * 256;
-  const int ld_k = strip_off + (mhalf ? row_token_hi(r8) : r8) * 16;
-  // transposed V: matrix "lo" rows (2i, 2i+1) = tokens (i, 12+i), "hi" = (4+i, 8+i)
-  const int ld_v = strip_off + (mhalf ? ((r8 & 1) ? 8 + (r8 >> 1) : 4 + (r8 >> 1))
-                                      : ((r8 & 1) ? 12 + (r8 >> 1) : (r8 >> 1))) * 16;
-  const int t0 = gid, t1 = row_token_hi(gid);  // tokens of this thread's C rows gid, gid+8
-  const int tok_lo = rg.int4_lo, tok_hi = rg.int4_hi;
-  uint32_t *ptw = reinterpret_cast<uint32_t *>(x.ptile);  // [4 g][8 heads][8 token pairs]
-  const float2 kappa = make_float2(kLog2e * 0.08838834764831845f, kLog2e * 0.08838834764831845f);
-
-  for (int k = 0; k < np; ++k) {
-    const int st = k % kStages;
-    if (!wait_stage(x, st, err)) {
-      for (int kk = k + 1; kk < min(np, k + kStages); ++kk) wait_stage(x, kk % kStages, err);
-      write_empty(rec, G, lane);
-      return;
-    }
-    uint8_t *sp = x.stage0 + st * kStageBytes;
-    const uint32_t sa = smem_u32(sp);
-
-    // ---- S^T = K Q^T, one fp32 accumulator per 32-dim group ----
-    uint32_t kw[2][4];
-    ldsm_x4(kw[0], sa + ld_k);
-    ldsm_x4(kw[1], sa + 512 + ld_k);
-    float acc[4][4];
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      uint32_t pl[4], ph[4];
-      nib_pairs4(kw[g >> 1][(g & 1) * 2], pl);
-      nib_pairs4(kw[g >> 1][(g & 1) * 2 + 1], ph);
-      acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-      mma_f16(acc[g], pl[0], ph[0], pl[1], ph[1], qb[g][0][0], qb[g][0][1]);
-      mma_f16(acc[g], pl[2], ph[2], pl[3], ph[3], qb[g][1][0], qb[g][1][1]);
-    }
-    // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
-    const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffKp4 + t0 * 16),
-                         *reinterpret_cast<const uint4 *>(sp + kOffKp4 + t1 * 16)};
-    float2 sl[2];  // sl[hf] = logits of token (t0 | t1) for heads (2tig, 2tig+1)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const uint32_t pw[4] = {kp[hf].x, kp[hf].y, kp[hf].z, kp[hf].w};
-      float2 v = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float2 sm = h2_to_f2(pw[g]);
-        v = ffma2(make_float2(sm.x, sm.x), make_float2(acc[g][2 * hf], acc[g][2 * hf + 1]), v);
-        v = ffma2(make_float2(sm.y, sm.y), qs[g], v);
-      }
-      sl[hf] = fmul2(v, kappa);
-    }
-    const int tok0 = (p0 + k) * kPage;
-    if (tok0 < tok_lo || tok0 + kPage > tok_hi) {  // ragged first/last page of the range
-      const bool v0 = tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi;
-      const bool v1 = tok0 + t1 >= tok_lo && tok0 + t1 < tok_hi;
-      if (!v0) sl[0] = make_float2(-CUDART_INF_F, -CUDART_INF_F);
-      if (!v1) sl[1] = make_float2(-CUDART_INF_F, -CUDART_INF_F);
-    }
-    // ---- online softmax; the rescale is skipped while no running max moves ----
-    float p[2][2];
-    float2 alpha2[2];
-    bool moved = false;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float s0 = e ? sl[0].y : sl[0].x, s1 = e ? sl[1].y : sl[1].x;
-      float t = fmaxf(s0, s1);
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-      const float mn = fmaxf(m[e], t);
-      const float a = mn != m[e] ? fast_exp2(m[e] - mn) : 1.0f;
-      moved |= mn != m[e];
-      m[e] = mn;
-      p[0][e] = fast_exp2(s0 - mn);
-      p[1][e] = fast_exp2(s1 - mn);
-      l[e] = fmaf(l[e], a, p[0][e] + p[1][e]);
-      alpha2[e] = make_float2(a, a);
-    }
-    if (__any_sync(0xffffffffu, moved)) {
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          mtp[g][e] = fmul2(mtp[g][e], alpha2[e]);
-          o[g][0][e] = fmul2(o[g][0][e], alpha2[e]);
-          o[g][1][e] = fmul2(o[g][1][e], alpha2[e]);
-        }
-    }
-    // ---- P'_g = p * vscale_g as fp16 token pairs; sum p * vmin_g on the side ----
-    const uint4 vp[2] = {*reinterpret_cast<const uint4 *>(sp + kOffVp4 + t0 * 16),
-                         *reinterpret_cast<const uint4 *>(sp + kOffVp4 + t1 * 16)};
-    const float2 pe[2] = {make_float2(p[0][0], p[1][0]), make_float2(p[0][1], p[1][1])};
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const uint32_t w0 = g == 0 ? vp[0].x : g == 1 ? vp[0].y : g == 2 ? vp[0].z : vp[0].w;
-      const uint32_t w1 = g == 0 ? vp[1].x : g == 1 ? vp[1].y : g == 2 ? vp[1].z : vp[1].w;
-      const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
-      const float2 sv = make_float2(f0.x, f1.x), mv = make_float2(f0.y, f1.y);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = 2 * tig + e;
-        const float2 pv = fmul2(pe[e], sv);
-        if (j < G) ptw[(g * 8 + j) * 8 + gid] = pack_h2(pv.x, pv.y);
-        mtp[g][e] = ffma2(pe[e], mv, mtp[g][e]);
-      }
-    }
-    __syncwarp();
-    // ---- O^T += V^T P' per group: A = V codes (transposed ldmatrix), B = P'_g ----
-    uint32_t vw[2][4];
-    ldsm_x4_t(vw[0], sa + kOffVc4 + ld_v);
-    ldsm_x4_t(vw[1], sa + kOffVc4 + 512 + ld_v);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      uint32_t vl[4], vh[4];
-      nib_pairs4(vw[g >> 1][(g & 1) * 2], vl);
-      nib_pairs4(vw[g >> 1][(g & 1) * 2 + 1], vh);
-      uint32_t b01 = 0, b23 = 0;
-      if (gid < G) {
-        b01 = ptw[(g * 8 + gid) * 8 + tig];
-        b23 = ptw[(g * 8 + gid) * 8 + tig + 4];
-      }
-      float c0[4] = {o[g][0][0].x, o[g][0][1].x, o[g][0][0].y, o[g][0][1].y};
-      mma_f16(c0, vl[0], vl[1], vh[0], vh[1], b01, b23);
-      o[g][0][0] = make_float2(c0[0], c0[2]);
-      o[g][0][1] = make_float2(c0[1], c0[3]);
-      float c1[4] = {o[g][1][0].x, o[g][1][1].x, o[g][1][0].y, o[g][1][1].y};
-      mma_f16(c1, vl[2], vl[3], vh[2], vh[3], b01, b23);
-      o[g][1][0] = make_float2(c1[0], c1[2]);
-      o[g][1][1] = make_float2(c1[1], c1[3]);
-    }
-    __syncwarp();
-    if (k + kStages < np) issue(k + kStages);
-  }
-
-  // ---- finish: reduce per-thread sums over the 8 token lanes, write the partial ----
-  float mt[4][2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], off);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      mt[g][e] = mtp[g][e].x + mtp[g][e].y;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1)
-        mt[g][e] += __shfl_xor_sync(0xffffffffu, mt[g][e], off);
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int j = 2 * tig + e;
-    if (j < G) {
-      float *r = rec + j * kRecordFloats;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 v = make_float4(o[g][0][e].x + mt[g][e], o[g][0][e].y + mt[g][e],
-                                     o[g][1][e].x + mt[g][e], o[g][1][e].y + mt[g][e]);
-        *reinterpret_cast<float4 *>(r + 32 * g + 4 * gid) = v;
-      }
-      if (gid == 0) {
-        r[kHeadDim] = m[e] * kLn2;
-        r[kHeadDim + 1] = l[e];
-      }
-    }
-  }
-}
-
 // ------------------------- INT8 protected set ----------------------------
+// One kv head's protected set: sink tiles then recent-ring tiles, INT8 codes.
 __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t *__restrict__ q,
                                   int b, int h, int L, float *rec, int32_t *err) {
   const int G = c.gqa, H = c.num_kv_heads;
@@ -600,15 +364,15 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
     for (int e = 0; e < 2; ++e) {
       const int j = 2 * tig + e;
       if (j < G) {
-        x.ptile[j * 16 + gid] = __half_as_ushort(__float2half_rn(s[0][e] * sv0));
-        x.ptile[j * 16 + gid + 8] = __half_as_ushort(__float2half_rn(s[1][e] * sv1));
+        x.ptile8[j * 16 + gid] = __half_as_ushort(__float2half_rn(s[0][e] * sv0));
+        x.ptile8[j * 16 + gid + 8] = __half_as_ushort(__float2half_rn(s[1][e] * sv1));
       }
     }
     __syncwarp();
     uint32_t b01 = 0, b23 = 0;
     if (gid < G) {
-      b01 = *reinterpret_cast<const uint32_t *>(&x.ptile[gid * 16 + 2 * tig]);
-      b23 = *reinterpret_cast<const uint32_t *>(&x.ptile[gid * 16 + 2 * tig + 8]);
+      b01 = *reinterpret_cast<const uint32_t *>(&x.ptile8[gid * 16 + 2 * tig]);
+      b23 = *reinterpret_cast<const uint32_t *>(&x.ptile8[gid * 16 + 2 * tig + 8]);
     }
 #pragma unroll
     for (int pr = 0; pr < 4; ++pr) {
@@ -646,13 +410,310 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   }
 }
 
+
+// ---------------------------- INT4 chunk --------------------------------
+// Token order of the QK^T M-tile rows: rows 0-7 are tokens 0-7, rows 8-11 tokens 12-15,
+// rows 12-15 tokens 8-11. With it a thread's two rows (gid, gid+8) are the tokens whose
+// P' values it packs into one 32-bit word, the transposed V loads read those pairs, and
+// neither the K nor the V ldmatrix phases hit a shared-memory bank twice.
+__device__ __forceinline__ int row_token_hi(int r) { return 8 + ((r + 4) & 7); }
+
+// One chunk of INT4 pages for HPW kv heads (h0 .. h0+nh-1, nh <= HPW). MMA column
+// col (0..7) belongs to head slot col / CPH and query j = col % CPH of that head.
+template <int HPW>
+__device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
+                             const uint16_t *__restrict__ q, int b, int h0, int nh, int r,
+                             int chunk, const Regions &rg, int32_t *err) {
+  constexpr int CPH = 8 / HPW;  // MMA columns per kv head slot
+  const int G = c.gqa, H = c.num_kv_heads;
+  const int lane = x.lane, gid = x.gid, tig = x.tig;
+  const int p0 = rg.first_page + chunk * w.chunk_pages;
+  const int last = (rg.int4_hi - 1) / kPage;
+  const int np = min(w.chunk_pages, last - p0 + 1);
+  // this lane's C-fragment columns 2tig, 2tig+1: head slot and query index
+  const int hs_c = (2 * tig) / CPH;
+  const int jc0 = (2 * tig) % CPH;
+  const bool head_c_live = hs_c < nh;
+
+  int pid = 0;
+  if (lane < np) pid = c.page_table[static_cast<size_t>(b) * c.max_pages + p0 + lane];
+  const bool bad = lane < np && (pid < 0 || pid >= c.num_pages);
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
+    for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+    return;
+  }
+
+  // stage layout: K codes [HPW][1024] | V codes [HPW][1024] | K params [HPW][256] | V params
+  constexpr int kOffVc = HPW * kInt4CodeBytes;
+  constexpr int kOffKp = 2 * HPW * kInt4CodeBytes;
+  constexpr int kOffVp = kOffKp + HPW * kInt4ParamBytes;
+  auto issue = [&](int k) {
+    const int pk = __shfl_sync(0xffffffffu, pid, k);
+    if (lane == 0) {
+      const int st = k % kStages;
+      uint8_t *dst = x.stage0 + st * kStageBytes;
+      const size_t blk = static_cast<size_t>(pk) * H + h0;
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&x.bars[st], HPW * (2 * kInt4CodeBytes + 2 * kInt4ParamBytes));
+      if (nh == HPW) {  // the kv heads of one page are adjacent: one copy per array
+        bulk_g2s(dst, c.k_codes + blk * kInt4CodeBytes, HPW * kInt4CodeBytes, &x.bars[st]);
+        bulk_g2s(dst + kOffVc, c.v_codes + blk * kInt4CodeBytes, HPW * kInt4CodeBytes, &x.bars[st]);
+        bulk_g2s(dst + kOffKp, reinterpret_cast<const uint8_t *>(c.k_params) + blk * kInt4ParamBytes,
+                 HPW * kInt4ParamBytes, &x.bars[st]);
+        bulk_g2s(dst + kOffVp, reinterpret_cast<const uint8_t *>(c.v_params) + blk * kInt4ParamBytes,
+                 HPW * kInt4ParamBytes, &x.bars[st]);
+      } else {  // fewer heads than slots: fill the spare slots with a copy of head h0
+        for (int hs = 0; hs < HPW; ++hs) {
+          bulk_g2s(dst + hs * kInt4CodeBytes, c.k_codes + blk * kInt4CodeBytes, kInt4CodeBytes,
+                   &x.bars[st]);
+          bulk_g2s(dst + kOffVc + hs * kInt4CodeBytes, c.v_codes + blk * kInt4CodeBytes,
+                   kInt4CodeBytes, &x.bars[st]);
+          bulk_g2s(dst + kOffKp + hs * kInt4ParamBytes,
+                   reinterpret_cast<const uint8_t *>(c.k_params) + blk * kInt4ParamBytes,
+                   kInt4ParamBytes, &x.bars[st]);
+          bulk_g2s(dst + kOffVp + hs * kInt4ParamBytes,
+                   reinterpret_cast<const uint8_t *>(c.v_params) + blk * kInt4ParamBytes,
+                   kInt4ParamBytes, &x.bars[st]);
+        }
+      }
+    }
+  };
+  const int npre = min(np, kStages);
+  for (int k = 0; k < npre; ++k) issue(k);
+
+  // ---- query fragments (B operand of QK^T). Lane column gid = (slot gid/CPH, query
+  // gid%CPH); slot hs's fragments are zero unless the column is in slot hs.
+  // group g, k-tile kt: b01 = (q[32g+8tig+2kt], q[..+4]), b23 = (q[..+2kt+1], q[..+2kt+5])
+  uint32_t qb[HPW][4][2][2];
+  float qsum_own[4];
+  bool qbad = false;
+  {
+    const int hs_b = gid / CPH, jb = gid % CPH;
+    const bool live = jb < G && hs_b < nh;
+    const uint16_t *qrow =
+        q + (static_cast<size_t>(b) * H * G + (h0 + hs_b) * G + jb) * kHeadDim;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
+      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.z << 16), (v.x >> 16) | (v.z & 0xFFFF0000u),
+                              (v.y & 0xFFFFu) | (v.w << 16), (v.y >> 16) | (v.w & 0xFFFF0000u)};
+      float sum = 0.f;
+      uint32_t f16[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sum += q_to_f16_pair(pr[i], f16[i], qbad);
+#pragma unroll
+      for (int hs = 0; hs < HPW; ++hs) {
+        const bool mine = hs == hs_b;
+        qb[hs][g][0][0] = mine ? f16[0] : 0u;
+        qb[hs][g][0][1] = mine ? f16[1] : 0u;
+        qb[hs][g][1][0] = mine ? f16[2] : 0u;
+        qb[hs][g][1][1] = mine ? f16[3] : 0u;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      qsum_own[g] = sum;  // sum over the group's 32 dims for column gid
+    }
+  }
+  if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
+  float2 qs[4];  // column (2tig, 2tig+1) sums, matching the C-fragment columns
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    qs[g].x = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig));
+    qs[g].y = __shfl_sync(0xffffffffu, qsum_own[g], 4 * (2 * tig + 1));
+  }
+
+  float m[2] = {kNegBig, kNegBig}, l[2] = {0.f, 0.f};
+  float o[4][2][4];  // [group][m-tile]: rows dim 32g+4gid+2mt (c0,c1) and +1 (c2,c3)
+  float mt[4][2];    // sum p * vmin per group and column
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    mt[g][0] = mt[g][1] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) o[g][t][0] = o[g][t][1] = o[g][t][2] = o[g][t][3] = 0.f;
+  }
+
+  // ldmatrix lane addresses: matrix m = lane/8 covers strip m/2 (256 B each), row r = lane%8
+  const int r8 = lane & 7;
+  const int mhalf = (lane >> 3) & 1;
+  const int strip_off = (lane >> 4) * 256;
+  const int ld_k = strip_off + (mhalf ? row_token_hi(r8) : r8) * 16;
+  // transposed V: matrix "lo" rows (2i, 2i+1) = tokens (i, 12+i), "hi" = (4+i, 8+i)
+  const int ld_v = strip_off + (mhalf ? ((r8 & 1) ? 8 + (r8 >> 1) : 4 + (r8 >> 1))
+                                      : ((r8 & 1) ? 12 + (r8 >> 1) : (r8 >> 1))) * 16;
+  const int t0 = gid, t1 = row_token_hi(gid);  // tokens of this thread's C rows gid, gid+8
+  const int tok_lo = rg.int4_lo, tok_hi = rg.int4_hi;
+  const int kp_off = kOffKp + hs_c * kInt4ParamBytes;
+  const int vp_off = kOffVp + hs_c * kInt4ParamBytes;
+  const bool write_p0 = head_c_live && jc0 < G, write_p1 = head_c_live && jc0 + 1 < G;
+  uint32_t *pt_mine = x.ptile + (hs_c * 4 * 8 + 2 * tig) * kPWordsPerCol + gid;
+
+  for (int k = 0; k < np; ++k) {
+    const int st = k % kStages;
+    if (!wait_stage(x, st, err)) {
+      for (int kk = k + 1; kk < min(np, k + kStages); ++kk) wait_stage(x, kk % kStages, err);
+      for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+      return;
+    }
+    uint8_t *sp = x.stage0 + st * kStageBytes;
+    const uint32_t sa = smem_u32(sp);
+
+    // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
+    const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kp_off + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + kp_off + t1 * 16)};
+    float2 sl0 = make_float2(0.f, 0.f), sl1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {  // group pairs (2gp, 2gp+1): one ldmatrix.x4 per head
+      uint32_t kw[HPW][4];
+#pragma unroll
+      for (int hs = 0; hs < HPW; ++hs) ldsm_x4(kw[hs], sa + hs * kInt4CodeBytes + gp * 512 + ld_k);
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = 2 * gp + gg;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hs = 0; hs < HPW; ++hs) {
+          uint32_t pl[4], ph[4];
+          nib_pairs4(kw[hs][2 * gg], pl);
+          nib_pairs4(kw[hs][2 * gg + 1], ph);
+          mma_f16(acc, pl[0], ph[0], pl[1], ph[1], qb[hs][g][0][0], qb[hs][g][0][1]);
+          mma_f16(acc, pl[2], ph[2], pl[3], ph[3], qb[hs][g][1][0], qb[hs][g][1][1]);
+        }
+        const uint32_t w0 = g == 0 ? kp[0].x : g == 1 ? kp[0].y : g == 2 ? kp[0].z : kp[0].w;
+        const uint32_t w1 = g == 0 ? kp[1].x : g == 1 ? kp[1].y : g == 2 ? kp[1].z : kp[1].w;
+        const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
+        sl0 = ffma2(make_float2(f0.x, f0.x), make_float2(acc[0], acc[1]), sl0);
+        sl0 = ffma2(make_float2(f0.y, f0.y), qs[g], sl0);
+        sl1 = ffma2(make_float2(f1.x, f1.x), make_float2(acc[2], acc[3]), sl1);
+        sl1 = ffma2(make_float2(f1.y, f1.y), qs[g], sl1);
+      }
+    }
+    float s[2][2];
+    s[0][0] = sl0.x * kScaleLog2;
+    s[0][1] = sl0.y * kScaleLog2;
+    s[1][0] = sl1.x * kScaleLog2;
+    s[1][1] = sl1.y * kScaleLog2;
+    const int tok0 = (p0 + k) * kPage;
+    if (tok0 < tok_lo || tok0 + kPage > tok_hi) {  // ragged first/last page of the range
+      if (!(tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi)) s[0][0] = s[0][1] = -CUDART_INF_F;
+      if (!(tok0 + t1 >= tok_lo && tok0 + t1 < tok_hi)) s[1][0] = s[1][1] = -CUDART_INF_F;
+    }
+    // ---- online softmax; the rescale is skipped while no running max moves ----
+    float a[2];
+    bool moved = false;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float t = fmaxf(s[0][e], s[1][e]);
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+      const float mn = fmaxf(m[e], t);
+      const bool mv = mn != m[e];
+      a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
+      moved |= mv;
+      m[e] = mn;
+      s[0][e] = fast_exp2(s[0][e] - mn);
+      s[1][e] = fast_exp2(s[1][e] - mn);
+      l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
+    }
+    if (__any_sync(0xffffffffu, moved)) {
+      const float2 a2 = make_float2(a[0], a[1]);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        mt[g][0] *= a[0];
+        mt[g][1] *= a[1];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const float2 u = fmul2(make_float2(o[g][t][0], o[g][t][1]), a2);
+          const float2 v = fmul2(make_float2(o[g][t][2], o[g][t][3]), a2);
+          o[g][t][0] = u.x; o[g][t][1] = u.y; o[g][t][2] = v.x; o[g][t][3] = v.y;
+        }
+      }
+    }
+    // ---- P'_g = p * vscale_g as fp16 token pairs; sum p * vmin_g on the side ----
+    const uint4 vp[2] = {*reinterpret_cast<const uint4 *>(sp + vp_off + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + vp_off + t1 * 16)};
+    const float2 pe0 = make_float2(s[0][0], s[1][0]), pe1 = make_float2(s[0][1], s[1][1]);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t w0 = g == 0 ? vp[0].x : g == 1 ? vp[0].y : g == 2 ? vp[0].z : vp[0].w;
+      const uint32_t w1 = g == 0 ? vp[1].x : g == 1 ? vp[1].y : g == 2 ? vp[1].z : vp[1].w;
+      const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
+      const float2 sv = make_float2(f0.x, f1.x);
+      const float2 q0 = fmul2(pe0, sv), q1 = fmul2(pe1, sv);
+      if (write_p0) pt_mine[(g * 8) * kPWordsPerCol] = pack_h2(q0.x, q0.y);
+      if (write_p1) pt_mine[(g * 8 + 1) * kPWordsPerCol] = pack_h2(q1.x, q1.y);
+      mt[g][0] = fmaf(pe0.x, f0.y, fmaf(pe0.y, f1.y, mt[g][0]));
+      mt[g][1] = fmaf(pe1.x, f0.y, fmaf(pe1.y, f1.y, mt[g][1]));
+    }
+    __syncwarp();
+    // ---- O^T += V^T P' per group and head slot: A = V codes, B = P'_g of that slot ----
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {
+      uint32_t vw[HPW][4];
+#pragma unroll
+      for (int hs = 0; hs < HPW; ++hs)
+        ldsm_x4_t(vw[hs], sa + kOffVc + hs * kInt4CodeBytes + gp * 512 + ld_v);
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = 2 * gp + gg;
+#pragma unroll
+        for (int hs = 0; hs < HPW; ++hs) {
+          uint32_t vl[4], vh[4];
+          nib_pairs4(vw[hs][2 * gg], vl);
+          nib_pairs4(vw[hs][2 * gg + 1], vh);
+          const uint32_t *pb = x.ptile + ((hs * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
+          const uint32_t b01 = pb[0], b23 = pb[4];
+          mma_f16(o[g][0], vl[0], vl[1], vh[0], vh[1], b01, b23);
+          mma_f16(o[g][1], vl[2], vl[3], vh[2], vh[3], b01, b23);
+        }
+      }
+    }
+    __syncwarp();
+    if (k + kStages < np) issue(k + kStages);
+  }
+
+  // ---- finish: reduce per-thread sums over the 8 token lanes, write the partial ----
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], off);
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1)
+        mt[g][e] += __shfl_xor_sync(0xffffffffu, mt[g][e], off);
+  }
+  if (head_c_live) {
+    float *rec = record_of(w, H, G, b, h0 + hs_c, r);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = jc0 + e;
+      if (j < G) {
+        float *rr = rec + j * kRecordFloats;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 v = make_float4(o[g][0][e] + mt[g][e], o[g][0][2 + e] + mt[g][e],
+                                       o[g][1][e] + mt[g][e], o[g][1][2 + e] + mt[g][e]);
+          *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
+        }
+        if (gid == 0) {
+          rr[kHeadDim] = m[e] * kLn2;
+          rr[kHeadDim + 1] = l[e];
+        }
+      }
+    }
+  }
+}
+
 #ifndef KV4_MIN_BLOCKS
-#define KV4_MIN_BLOCKS 4  // CTAs per SM the register budget is sized for
+#define KV4_MIN_BLOCKS 3  // CTAs per SM the register budget is sized for
 #endif
 
+template <int HPW>
 __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(CacheView c, Workspace w,
-                                                              const uint16_t *__restrict__ q,
-                                                              int32_t *err) {
+                                                                           const uint16_t *__restrict__ q,
+                                                                           int32_t *err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   WarpCtx x;
   const int warp = threadIdx.x >> 5;
@@ -661,10 +722,13 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
   x.tig = x.lane & 3;
   uint8_t *mine = smem + warp * kWarpSmem;
   x.stage0 = mine;
-  x.ptile = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes);
-  x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes);
+  x.ptile = reinterpret_cast<uint32_t *>(mine + kStages * kStageBytes);
+  x.ptile8 = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes + kPtileBytes);
+  x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes + kPtile8Bytes);
   x.parity = 0;
   x.dead = false;
+  // the INT4 P' tile's unused columns stay zero for the whole kernel
+  for (int i = x.lane; i < kPtileBytes / 4; i += 32) x.ptile[i] = 0u;
   if (x.lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&x.bars[s], 1);
     fence_barrier_init();
@@ -678,18 +742,14 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
     if (x.lane == 0) item = atomicAdd(w.counter, 1);
     item = __shfl_sync(0xffffffffu, item, 0);
     if (item >= n_items) break;
-    const int pair = item / H;
-    const int h = item - pair * H;
-    const int2 pr = w.pairs[pair];
-    const int b = pr.x, r = pr.y;
+    const int4 en = w.entries[item];
+    const int b = en.x, r = en.y, h0 = en.z, nh = en.w;
     const int L = c.seq_lens[b];
     const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages);
-    float *rec = w.partials +
-                 static_cast<size_t>(w.unit_offsets[b * H + h] + r) * G * kRecordFloats;
     if (r < rg.has_prot)
-      process_protected(x, c, q, b, h, L, rec, err);
+      process_protected(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
     else
-      process_int4(x, c, w, q, b, h, r - rg.has_prot, rg, rec, err);
+      process_int4<HPW>(x, c, w, q, b, h0, nh, r, r - rg.has_prot, rg, err);
     if (x.dead) break;
   }
 }
@@ -747,26 +807,37 @@ cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_fla
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
-                             int32_t *err_flag, cudaStream_t s) {
+template <int HPW>
+static cudaError_t launch_attn_t(const CacheView &c, const Workspace &w, const uint16_t *q,
+                                 int32_t *err_flag, cudaStream_t s) {
   static int configured_device = -1;
   static int grid = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev != configured_device) {
-    e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCtaSmem);
+    e = cudaFuncSetAttribute(attn_kernel<HPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kCtaSmem);
     if (e != cudaSuccess) return e;
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel, kWarps * 32, kCtaSmem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<HPW>, kWarps * 32,
+                                                      kCtaSmem);
     if (e != cudaSuccess) return e;
     grid = sms * (per_sm > 0 ? per_sm : 1);
     configured_device = dev;
   }
-  attn_kernel<<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
+  attn_kernel<HPW><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
   return cudaGetLastError();
+}
+
+int heads_per_warp_for(int gqa) { return gqa <= 4 ? 2 : 1; }
+
+cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
+                             int32_t *err_flag, cudaStream_t s) {
+  return w.heads_per_warp == 2 ? launch_attn_t<2>(c, w, q, err_flag, s)
+                               : launch_attn_t<1>(c, w, q, err_flag, s);
 }
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
@@ -784,10 +855,11 @@ size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_hea
   const long long pages = (static_cast<long long>(max_seq_len) + kPage - 1) / kPage + 1;
   const long long per_seq = 1 + (pages + chunk_pages - 1) / chunk_pages;
   const long long cap = static_cast<long long>(num_seqs) * per_seq;
+  const long long cap_e = cap * num_kv_heads;
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
   size_t off = 256;  // counter, n_items
-  const size_t pairs_off = off;
-  off = up(off + static_cast<size_t>(cap) * sizeof(int2));
+  const size_t ent_off = off;
+  off = up(off + static_cast<size_t>(cap_e) * sizeof(int4));
   const size_t units_off = off;
   off = up(off + (static_cast<size_t>(num_seqs) * num_kv_heads + 1) * sizeof(int32_t));
   const size_t part_off = off;
@@ -796,11 +868,13 @@ size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_hea
     uint8_t *p = static_cast<uint8_t *>(base);
     carve->counter = reinterpret_cast<int32_t *>(p);
     carve->n_items = reinterpret_cast<int32_t *>(p) + 1;
-    carve->pairs = reinterpret_cast<int2 *>(p + pairs_off);
+    carve->entries = reinterpret_cast<int4 *>(p + ent_off);
     carve->unit_offsets = reinterpret_cast<int32_t *>(p + units_off);
     carve->partials = reinterpret_cast<float *>(p + part_off);
     carve->cap_pairs = static_cast<int32_t>(cap);
+    carve->cap_entries = static_cast<int32_t>(cap_e);
     carve->chunk_pages = chunk_pages;
+    carve->heads_per_warp = heads_per_warp_for(gqa);
   }
   return off;
 }

@@ -34,12 +34,14 @@ struct CacheView {
 // Workspace carve-up for one decode-attention call.
 struct Workspace {
   int32_t *counter;       // [1] dynamic work counter (reset by the plan kernel)
-  int32_t *n_items;       // [1] work items = pairs * Hkv
-  int2 *pairs;            // [cap_pairs] (sequence, region index within the sequence)
+  int32_t *n_items;       // [1] number of work entries
+  int4 *entries;          // [cap_entries] (sequence, region, first kv head, kv heads)
   int32_t *unit_offsets;  // [num_seqs*Hkv + 1] first partial record row of each (b, h)
   float *partials;        // [cap_pairs*Hkv][gqa][kRecordFloats]
-  int32_t cap_pairs;
+  int32_t cap_pairs;      // (sequence, region) pairs the partial area holds
+  int32_t cap_entries;    // work entries the entry list holds
   int32_t chunk_pages;
+  int32_t heads_per_warp;  // kv heads one warp serves in an INT4 region entry (1 or 2)
 };
 
 size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads,
