@@ -335,7 +335,7 @@ def run_gpu(args, rank, world, local_rank):
             "attention_ms": statistics.mean(att_ms),
             "attention_gbs_unique": ub / mean_att_s / 1e9,
             "attention_gbs_logical": lb / mean_att_s / 1e9,
-            "roofline": {"kernel": "kv4_decode_attention (plan + attn + merge launches)",
+            "roofline": {"kernel": "kv4_decode_attention (plan + attention + merge launches)",
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": None},

@@ -140,7 +140,8 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   if (ws_bytes < need) return KV4_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
-  if (e == cudaSuccess) e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
                           static_cast<uint16_t *>(out), out_f32, lse, s);

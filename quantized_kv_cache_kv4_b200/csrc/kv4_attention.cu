@@ -19,7 +19,8 @@
 //                N dimension (8) holds head A's queries in columns 0-3 and head B's in
 //                columns 4-7 (zeros in the other half of each B operand), so every lane's
 //                softmax and scaling work is useful.
-//   merge_kernel one warp per (b, h, query head): fixed-order exact merge -> bf16 out.
+//   merge_kernel one warp per (unit, query): fixed-order exact merge -> bf16 out; also
+//                the kernel behind kv4_regional_merge.
 #include <math_constants.h>
 
 #include "kv4_device.cuh"
@@ -82,75 +83,100 @@ __device__ __forceinline__ Regions regions_of(int L, int S, int R, int C) {
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 
-__device__ int block_exclusive_scan(int v, int *sh, int *total) {
-  const int tid = threadIdx.x;
-  sh[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < kPlanThreads; off <<= 1) {
-    int t = tid >= off ? sh[tid - off] : 0;
-    __syncthreads();
-    sh[tid] += t;
-    __syncthreads();
+// Exclusive block-wide scan (warp shuffles + one warp over the 32 warp totals).
+__device__ int block_scan(int v, int *warp_sums, int *total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
   }
-  int incl = sh[tid];
-  *total = sh[kPlanThreads - 1];
+  if (lane == 31) warp_sums[wid] = x;
   __syncthreads();
-  return incl - v;
+  if (wid == 0) {
+    int s = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += y;
+    }
+    warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int base = wid ? warp_sums[wid - 1] : 0;
+  *total = warp_sums[31];
+  __syncthreads();
+  return base + x - v;
 }
 
+// Per-sequence counts for the work list.
+struct SeqPlan {
+  Regions g;
+  int pairs;    // regions (protected set + INT4 chunks)
+  int entries;  // work entries: one per kv head for the protected set, one per kv-head
+                // slot for every INT4 chunk
+};
+
+// Work list for one call, in (sequence, region, kv head) order: the kv heads of one page
+// and the sequences that share a prompt are processed next to each other, so shared
+// pages are read while they are still in L2.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspace w,
                                                             int32_t *err) {
-  __shared__ int sh[kPlanThreads];
+  __shared__ int warp_sums[32];
   const int B = c.num_seqs, H = c.num_kv_heads, C = w.chunk_pages;
   const int S = c.num_sinks, R = c.num_recent;
   const int hpw = w.heads_per_warp;
   const int nslots = (H + hpw - 1) / hpw;
-  auto counts = [&](int b, int &pairs, int &ents, bool flag) {
-    pairs = ents = 0;
-    if (b >= B) return;
+
+  auto plan_of = [&](int b, bool flag) {
+    SeqPlan sp;
     int L = c.seq_lens[b];
     if (L < 0 || L > c.max_pages * kPage) {
       if (flag) set_err(err, KV4_DEVERR_SEQ_LEN);
       L = 0;
     }
-    const Regions g = regions_of(L, S, R, C);
-    pairs = g.has_prot + g.n_chunks;
-    ents = g.has_prot * H + g.n_chunks * nslots;
+    sp.g = regions_of(L, S, R, C);
+    sp.pairs = sp.g.has_prot + sp.g.n_chunks;
+    sp.entries = sp.g.has_prot * H + sp.g.n_chunks * nslots;
+    return sp;
   };
+
   // pass 1: totals
   int tp = 0, te = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
-    int p, e, t;
-    counts(base + threadIdx.x, p, e, false);
-    block_exclusive_scan(p, sh, &t);
+    const int b = base + threadIdx.x;
+    SeqPlan sp{};
+    if (b < B) sp = plan_of(b, false);
+    int t;
+    block_scan(sp.pairs, warp_sums, &t);
     tp += t;
-    block_exclusive_scan(e, sh, &t);
+    block_scan(sp.entries, warp_sums, &t);
     te += t;
   }
   const bool fits = tp <= w.cap_pairs && te <= w.cap_entries;
-  // pass 2: entries and partial offsets (all units empty if the workspace is too small)
+
+  // pass 2: partial offsets and entries (every unit empty if the workspace is too small)
   int run_p = 0, run_e = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    int p, e, t;
-    counts(b, p, e, true);
-    if (!fits) p = e = 0;
-    const int po = run_p + block_exclusive_scan(p, sh, &t);
+    SeqPlan sp{};
+    if (b < B) sp = plan_of(b, true);
+    if (!fits) sp.pairs = sp.entries = 0;
+    int t;
+    const int po = run_p + block_scan(sp.pairs, warp_sums, &t);
     run_p += t;
-    int eo = run_e + block_exclusive_scan(e, sh, &t);
+    int eo = run_e + block_scan(sp.entries, warp_sums, &t);
     run_e += t;
-    if (b < B) {
-      int L = c.seq_lens[b];
-      if (L < 0 || L > c.max_pages * kPage) L = 0;
-      const Regions g = regions_of(L, S, R, C);
-      if (p > 0) {
-        if (g.has_prot)
-          for (int h = 0; h < H; ++h) w.entries[eo++] = make_int4(b, 0, h, 1);
-        for (int ch = 0; ch < g.n_chunks; ++ch)
-          for (int s = 0; s < nslots; ++s)
-            w.entries[eo++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
-      }
-      for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * p;
+    if (b >= B) continue;
+    for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * sp.pairs;
+    if (sp.entries) {
+      const Regions &g = sp.g;
+      if (g.has_prot)
+        for (int h = 0; h < H; ++h) w.entries[eo++] = make_int4(b, 0, h, 1);
+      for (int ch = 0; ch < g.n_chunks; ++ch)
+        for (int s = 0; s < nslots; ++s)
+          w.entries[eo++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
     }
   }
   if (threadIdx.x == 0) {
@@ -706,6 +732,77 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   }
 }
 
+// ---------------------------------------------------------------------------
+// exact regional merge
+// ---------------------------------------------------------------------------
+// One warp merges query j of unit u over its regions r0 .. r0+n-1:
+//   M = max m_r, Lambda = sum l_r e^(m_r - M), O = sum acc_r e^(m_r - M) / Lambda,
+//   lse = M + ln Lambda, over live regions (l_r > 0); no live region gives O = 0,
+//   lse = -inf.
+// The region weights e^(m_r - M) are computed with the regions spread over the lanes
+// (fixed assignment and reduction tree); the weighted sum then walks the regions in
+// order with lane i owning dims 4i..4i+3, its loads independent of each other. The
+// arithmetic order is fixed, so the result is deterministic.
+__global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
+                                                    const int32_t *__restrict__ offs, int n_units,
+                                                    int G, Outputs o) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_units * G) return;
+  const int u = warp / G, j = warp - u * G;
+  const int r0 = offs[u], n = offs[u + 1] - r0;
+  auto rec_of = [&](int r) {
+    return partials + (static_cast<size_t>(r0 + r) * G + j) * kRecordFloats;
+  };
+  float M = -CUDART_INF_F;
+  for (int r = lane; r < n; r += 32) {
+    const float *rec = rec_of(r);
+    if (rec[kHeadDim + 1] > 0.f) M = fmaxf(M, rec[kHeadDim]);
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float lam = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -CUDART_INF_F) {
+    for (int base = 0; base < n; base += 32) {
+      // weights of regions base .. base+31, one per lane
+      float wl = 0.f;
+      if (base + lane < n) {
+        const float *rec = rec_of(base + lane);
+        const float lr = rec[kHeadDim + 1];
+        if (lr > 0.f) {
+          wl = expf(rec[kHeadDim] - M);
+          lam = fmaf(lr, wl, lam);
+        }
+      }
+      const int cnt = min(32, n - base);
+#pragma unroll 4
+      for (int i = 0; i < cnt; ++i) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, i);
+        const float4 a = reinterpret_cast<const float4 *>(rec_of(base + i))[lane];
+        if (wgt > 0.f) {
+          acc.x = fmaf(a.x, wgt, acc.x);
+          acc.y = fmaf(a.y, wgt, acc.y);
+          acc.z = fmaf(a.z, wgt, acc.z);
+          acc.w = fmaf(a.w, wgt, acc.w);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) lam += __shfl_xor_sync(0xffffffffu, lam, off);
+  }
+  const float inv = lam > 0.f ? 1.0f / lam : 0.f;
+  const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  const size_t row = static_cast<size_t>(u) * G + j;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t *>(&lo);
+  packed.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(o.out + row * kHeadDim + 4 * lane) = packed;
+  if (o.out_f32) *reinterpret_cast<float4 *>(o.out_f32 + row * kHeadDim + 4 * lane) = v;
+  if (o.lse && lane == 0) o.lse[row] = lam > 0.f ? M + logf(lam) : -CUDART_INF_F;
+}
+
 #ifndef KV4_MIN_BLOCKS
 #define KV4_MIN_BLOCKS 3  // CTAs per SM the register budget is sized for
 #endif
@@ -755,54 +852,10 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
 }
 
 // ---------------------------------------------------------------------------
-// exact regional merge
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
-                                                    const int32_t *__restrict__ offs, int n_units,
-                                                    int G, uint16_t *__restrict__ out,
-                                                    float *__restrict__ out_f32,
-                                                    float *__restrict__ lse) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= n_units * G) return;
-  const int u = warp / G, j = warp - u * G;
-  const int r0 = offs[u], r1 = offs[u + 1];
-  float M = -CUDART_INF_F, lam = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int r = r0; r < r1; ++r) {
-    const float *rec = partials + (static_cast<size_t>(r) * G + j) * kRecordFloats;
-    const float mr = rec[kHeadDim], lr = rec[kHeadDim + 1];
-    if (!(lr > 0.f)) continue;
-    const float4 a = reinterpret_cast<const float4 *>(rec)[lane];
-    if (mr > M) {
-      const float sc = expf(M - mr);
-      acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
-      lam *= sc;
-      M = mr;
-    }
-    const float wgt = expf(mr - M);
-    acc.x = fmaf(a.x, wgt, acc.x);
-    acc.y = fmaf(a.y, wgt, acc.y);
-    acc.z = fmaf(a.z, wgt, acc.z);
-    acc.w = fmaf(a.w, wgt, acc.w);
-    lam = fmaf(lr, wgt, lam);
-  }
-  const float inv = lam > 0.f ? 1.0f / lam : 0.f;
-  const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  const size_t o = (static_cast<size_t>(u) * G + j) * kHeadDim + 4 * lane;
-  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-  uint2 packed;
-  packed.x = *reinterpret_cast<uint32_t *>(&lo);
-  packed.y = *reinterpret_cast<uint32_t *>(&hi);
-  *reinterpret_cast<uint2 *>(out + o) = packed;
-  if (out_f32) *reinterpret_cast<float4 *>(out_f32 + o) = v;
-  if (lse && lane == 0) lse[static_cast<size_t>(u) * G + j] = lam > 0.f ? M + logf(lam) : -CUDART_INF_F;
-}
-
-// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag, cudaStream_t s) {
+cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag,
+                        cudaStream_t s) {
   plan_kernel<<<1, kPlanThreads, 0, s>>>(c, w, err_flag);
   return cudaGetLastError();
 }
@@ -846,7 +899,7 @@ cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps * 32 + 255) / 256;
   merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(partials, unit_offsets, n_units, group,
-                                                             out, out_f32, lse);
+                                                             Outputs{out, out_f32, lse});
   return cudaGetLastError();
 }
 

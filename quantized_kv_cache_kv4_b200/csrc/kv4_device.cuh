@@ -206,6 +206,14 @@ __device__ __forceinline__ __half f16_sat(float x) {
   return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
 }
 
+// atom.add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {
   if (flag) atomicOr(reinterpret_cast<unsigned int *>(flag), bit);
 }

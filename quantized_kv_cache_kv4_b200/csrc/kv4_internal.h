@@ -44,6 +44,13 @@ struct Workspace {
   int32_t heads_per_warp;  // kv heads one warp serves in an INT4 region entry (1 or 2)
 };
 
+// Where the merged attention output goes.
+struct Outputs {
+  uint16_t *out;   // bf16 [B][Hq][128]
+  float *out_f32;  // optional fp32 [B][Hq][128]
+  float *lse;      // optional fp32 [B][Hq]
+};
+
 size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads,
                        int32_t gqa, int32_t chunk_pages, Workspace *carve, void *base);
 
