@@ -110,17 +110,36 @@ __device__ int block_scan(int v, int *warp_sums, int *total) {
   return base + x - v;
 }
 
-// Per-sequence counts for the work list.
+// Work classes, processed in this order: full-length INT4 chunks, INT4 chunks of at
+// least half the length, protected sets, short INT4 chunks. Inside a class the order is
+// (sequence, region, kv head). Long work first keeps the end of the kernel short; the
+// natural order inside a class keeps the kv heads of one page and the sequences that
+// share a prompt next to each other, so shared pages are read while they are in L2.
+#ifndef KV4_PLAN_ORDER
+#define KV4_PLAN_ORDER 2  // 0: one class (natural order), 1: full chunks first, 2: four classes
+#endif
+constexpr int kClasses = 4;
+__device__ __forceinline__ int class_slot(int k) {
+#if KV4_PLAN_ORDER == 0
+  return 0 * k;
+#elif KV4_PLAN_ORDER == 1
+  return k == 0 ? 0 : 1;
+#else
+  return k;
+#endif
+}
+__device__ __forceinline__ int chunk_class(int pages, int C) {
+  return pages >= C ? 0 : (2 * pages >= C ? 1 : 3);
+}
+
+// Per-sequence entry counts per class.
 struct SeqPlan {
   Regions g;
-  int pairs;    // regions (protected set + INT4 chunks)
-  int entries;  // work entries: one per kv head for the protected set, one per kv-head
-                // slot for every INT4 chunk
+  int pages;          // INT4 pages of the sequence's INT4 range
+  int pairs;          // regions (protected set + INT4 chunks)
+  int e[kClasses];    // entries per class slot
 };
 
-// Work list for one call, in (sequence, region, kv head) order: the kv heads of one page
-// and the sequences that share a prompt are processed next to each other, so shared
-// pages are read while they are still in L2.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspace w,
                                                             int32_t *err) {
   __shared__ int warp_sums[32];
@@ -138,12 +157,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     }
     sp.g = regions_of(L, S, R, C);
     sp.pairs = sp.g.has_prot + sp.g.n_chunks;
-    sp.entries = sp.g.has_prot * H + sp.g.n_chunks * nslots;
+    sp.pages = sp.g.n_chunks ? (sp.g.int4_hi - 1) / kPage - sp.g.first_page + 1 : 0;
+#pragma unroll
+    for (int k = 0; k < kClasses; ++k) sp.e[k] = 0;
+    sp.e[class_slot(2)] += sp.g.has_prot * H;
+    const int nfull = sp.pages / C;
+    sp.e[class_slot(0)] += nfull * nslots;
+    if (sp.g.n_chunks > nfull) sp.e[class_slot(chunk_class(sp.pages - nfull * C, C))] += nslots;
     return sp;
   };
 
   // pass 1: totals
-  int tp = 0, te = 0;
+  int tp = 0, te[kClasses] = {0, 0, 0, 0};
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
     SeqPlan sp{};
@@ -151,37 +176,53 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     int t;
     block_scan(sp.pairs, warp_sums, &t);
     tp += t;
-    block_scan(sp.entries, warp_sums, &t);
-    te += t;
+#pragma unroll
+    for (int k = 0; k < kClasses; ++k) {
+      block_scan(sp.e[k], warp_sums, &t);
+      te[k] += t;
+    }
   }
-  const bool fits = tp <= w.cap_pairs && te <= w.cap_entries;
+  const int te_all = te[0] + te[1] + te[2] + te[3];
+  const bool fits = tp <= w.cap_pairs && te_all <= w.cap_entries;
 
   // pass 2: partial offsets and entries (every unit empty if the workspace is too small)
-  int run_p = 0, run_e = 0;
+  int run_p = 0, run_e[kClasses] = {0, te[0], te[0] + te[1], te[0] + te[1] + te[2]};
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
     SeqPlan sp{};
     if (b < B) sp = plan_of(b, true);
-    if (!fits) sp.pairs = sp.entries = 0;
+    if (!fits) {
+      sp.pairs = 0;
+#pragma unroll
+      for (int k = 0; k < kClasses; ++k) sp.e[k] = 0;
+    }
     int t;
     const int po = run_p + block_scan(sp.pairs, warp_sums, &t);
     run_p += t;
-    int eo = run_e + block_scan(sp.entries, warp_sums, &t);
-    run_e += t;
+    int eo[kClasses];
+#pragma unroll
+    for (int k = 0; k < kClasses; ++k) {
+      eo[k] = run_e[k] + block_scan(sp.e[k], warp_sums, &t);
+      run_e[k] += t;
+    }
     if (b >= B) continue;
     for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * sp.pairs;
-    if (sp.entries) {
+    if (sp.pairs) {
       const Regions &g = sp.g;
-      if (g.has_prot)
-        for (int h = 0; h < H; ++h) w.entries[eo++] = make_int4(b, 0, h, 1);
-      for (int ch = 0; ch < g.n_chunks; ++ch)
+      if (g.has_prot) {
+        const int k = class_slot(2);
+        for (int h = 0; h < H; ++h) w.entries[eo[k]++] = make_int4(b, 0, h, 1);
+      }
+      for (int ch = 0; ch < g.n_chunks; ++ch) {
+        const int k = class_slot(chunk_class(min(C, sp.pages - ch * C), C));
         for (int s = 0; s < nslots; ++s)
-          w.entries[eo++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
+          w.entries[eo[k]++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
+      }
     }
   }
   if (threadIdx.x == 0) {
     w.unit_offsets[B * H] = H * run_p;
-    *w.n_items = run_e;
+    *w.n_items = fits ? te_all : 0;
     *w.counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
   }
