@@ -551,7 +551,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 
   // ---- query fragments (B operand of QK^T). Lane column gid = (slot gid/CPH, query
   // gid%CPH); slot hs's fragments are zero unless the column is in slot hs.
-  // group g, k-tile kt: b01 = (q[32g+8tig+2kt], q[..+4]), b23 = (q[..+2kt+1], q[..+2kt+5])
+  // group g: k-tile 0 b01 = (q[32g+8tig], q[..+2]), b23 = (q[..+4], q[..+6]);
+  //          k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7])
   uint32_t qb[HPW][4][2][2];
   float qsum_own[4];
   bool qbad = false;
@@ -563,8 +564,9 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
-      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.z << 16), (v.x >> 16) | (v.z & 0xFFFF0000u),
-                              (v.y & 0xFFFFu) | (v.w << 16), (v.y >> 16) | (v.w & 0xFFFF0000u)};
+      // pairs matching nib_pairs_k: (0,2) (4,6) (1,3) (5,7)
+      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.y << 16), (v.z & 0xFFFFu) | (v.w << 16),
+                              (v.x >> 16) | (v.y & 0xFFFF0000u), (v.z >> 16) | (v.w & 0xFFFF0000u)};
       float sum = 0.f;
       uint32_t f16[4];
 #pragma unroll
@@ -628,7 +630,10 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
     const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kp_off + t0 * 16),
                          *reinterpret_cast<const uint4 *>(sp + kp_off + t1 * 16)};
-    float2 sl0 = make_float2(0.f, 0.f), sl1 = make_float2(0.f, 0.f);
+    // sc*: sum_g scale_g * (q . c)_g / 512 (codes enter the MMA scaled by 2^-9);
+    // mn*: sum_g min_g * sum_g(q)
+    float2 sc0 = make_float2(0.f, 0.f), sc1 = make_float2(0.f, 0.f);
+    float2 mn0 = make_float2(0.f, 0.f), mn1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int gp = 0; gp < 2; ++gp) {  // group pairs (2gp, 2gp+1): one ldmatrix.x4 per head
       uint32_t kw[HPW][4];
@@ -641,25 +646,29 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t pl[4], ph[4];
-          nib_pairs4(kw[hs][2 * gg], pl);
-          nib_pairs4(kw[hs][2 * gg + 1], ph);
+          nib_pairs_k(kw[hs][2 * gg], pl);
+          nib_pairs_k(kw[hs][2 * gg + 1], ph);
           mma_f16(acc, pl[0], ph[0], pl[1], ph[1], qb[hs][g][0][0], qb[hs][g][0][1]);
           mma_f16(acc, pl[2], ph[2], pl[3], ph[3], qb[hs][g][1][0], qb[hs][g][1][1]);
         }
         const uint32_t w0 = g == 0 ? kp[0].x : g == 1 ? kp[0].y : g == 2 ? kp[0].z : kp[0].w;
         const uint32_t w1 = g == 0 ? kp[1].x : g == 1 ? kp[1].y : g == 2 ? kp[1].z : kp[1].w;
         const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
-        sl0 = ffma2(make_float2(f0.x, f0.x), make_float2(acc[0], acc[1]), sl0);
-        sl0 = ffma2(make_float2(f0.y, f0.y), qs[g], sl0);
-        sl1 = ffma2(make_float2(f1.x, f1.x), make_float2(acc[2], acc[3]), sl1);
-        sl1 = ffma2(make_float2(f1.y, f1.y), qs[g], sl1);
+        sc0 = ffma2(make_float2(f0.x, f0.x), make_float2(acc[0], acc[1]), sc0);
+        mn0 = ffma2(make_float2(f0.y, f0.y), qs[g], mn0);
+        sc1 = ffma2(make_float2(f1.x, f1.x), make_float2(acc[2], acc[3]), sc1);
+        mn1 = ffma2(make_float2(f1.y, f1.y), qs[g], mn1);
       }
     }
+    const float2 k512 = make_float2(kCvtUnscale * kScaleLog2, kCvtUnscale * kScaleLog2);
+    const float2 k1 = make_float2(kScaleLog2, kScaleLog2);
+    const float2 sl0 = ffma2(sc0, k512, fmul2(mn0, k1));
+    const float2 sl1 = ffma2(sc1, k512, fmul2(mn1, k1));
     float s[2][2];
-    s[0][0] = sl0.x * kScaleLog2;
-    s[0][1] = sl0.y * kScaleLog2;
-    s[1][0] = sl1.x * kScaleLog2;
-    s[1][1] = sl1.y * kScaleLog2;
+    s[0][0] = sl0.x;
+    s[0][1] = sl0.y;
+    s[1][0] = sl1.x;
+    s[1][1] = sl1.y;
     const int tok0 = (p0 + k) * kPage;
     if (tok0 < tok_lo || tok0 + kPage > tok_hi) {  // ragged first/last page of the range
       if (!(tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi)) s[0][0] = s[0][1] = -CUDART_INF_F;
@@ -727,8 +736,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t vl[4], vh[4];
-          nib_pairs4(vw[hs][2 * gg], vl);
-          nib_pairs4(vw[hs][2 * gg + 1], vh);
+          nib_pairs_v(vw[hs][2 * gg], vl);
+          nib_pairs_v(vw[hs][2 * gg + 1], vh);
           const uint32_t *pb = x.ptile + ((hs * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
           const uint32_t b01 = pb[0], b23 = pb[4];
           mma_f16(o[g][0], vl[0], vl[1], vh[0], vh[1], b01, b23);
@@ -760,8 +769,11 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         float *rr = rec + j * kRecordFloats;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          const float4 v = make_float4(o[g][0][e] + mt[g][e], o[g][0][2 + e] + mt[g][e],
-                                       o[g][1][e] + mt[g][e], o[g][1][2 + e] + mt[g][e]);
+          // V codes entered the MMA scaled by 2^-9
+          const float4 v = make_float4(fmaf(o[g][0][e], kCvtUnscale, mt[g][e]),
+                                       fmaf(o[g][0][2 + e], kCvtUnscale, mt[g][e]),
+                                       fmaf(o[g][1][e], kCvtUnscale, mt[g][e]),
+                                       fmaf(o[g][1][2 + e], kCvtUnscale, mt[g][e]));
           *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
         }
         if (gid == 0) {

@@ -154,6 +154,44 @@ __device__ __forceinline__ void nib_pairs4(uint32_t w, uint32_t (&p)[4]) {
 }
 
 // ---------------------------------------------------------------------------
+// nibble -> fp16 through the fp8 conversion: a byte b in 0..15 read as e4m3 is exactly
+// b * 2^-9 (subnormals 0..7 and the first normal binade 8..15 are evenly spaced), so
+// masking the nibbles into bytes and converting two bytes at a time gives the codes
+// exactly, scaled by 2^-9; the scale is applied once after the dot products.
+// ---------------------------------------------------------------------------
+constexpr float kCvtUnscale = 512.0f;  // 2^9
+
+__device__ __forceinline__ uint32_t cvt_e4m3x2(uint32_t two_bytes) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+      : "=r"(d)
+      : "r"(two_bytes));
+  return d;
+}
+
+// K word (8 nibbles n0..n7 of one token, n_i = dim i): fp16 pairs
+// p0 = (n0, n2), p1 = (n4, n6), p2 = (n1, n3), p3 = (n5, n7), each scaled by 2^-9.
+__device__ __forceinline__ void nib_pairs_k(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  p[0] = cvt_e4m3x2(lo);
+  p[1] = cvt_e4m3x2(lo >> 16);
+  p[2] = cvt_e4m3x2(hi);
+  p[3] = cvt_e4m3x2(hi >> 16);
+}
+
+// V word from a transposed ldmatrix (token t0's nibbles d0..d3 in bits 0-15, token t1's
+// in bits 16-31): p[k] = (t0 dim k, t1 dim k), scaled by 2^-9.
+__device__ __forceinline__ void nib_pairs_v(uint32_t x, uint32_t (&p)[4]) {
+  uint32_t y;
+  asm("prmt.b32 %0, %1, %1, 0x3120;" : "=r"(y) : "r"(x));  // bytes t0(d0d1) t1(d0d1) t0(d2d3) t1(d2d3)
+  const uint32_t lo = y & 0x0F0F0F0Fu, hi = (y >> 4) & 0x0F0F0F0Fu;
+  p[0] = cvt_e4m3x2(lo);
+  p[1] = cvt_e4m3x2(hi);
+  p[2] = cvt_e4m3x2(lo >> 16);
+  p[3] = cvt_e4m3x2(hi >> 16);
+}
+
+// ---------------------------------------------------------------------------
 // packed fp32 pairs (sm_100 f32x2 FMA pipe operations)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
