@@ -41,6 +41,31 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegBig = -1.0e30f;  // running-max start: finite, so e^(m_old-m_new) is 0 not NaN
 constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
+// Nibble unpack of the INT4 codes: 1 = through the fp8 conversion (codes scaled by 2^-9),
+// 0 = through the exponent-bias OR (exact codes). Chosen per operand by measurement.
+#ifndef KV4_UNPACK_K
+#define KV4_UNPACK_K 1
+#endif
+#ifndef KV4_UNPACK_V
+#define KV4_UNPACK_V 1
+#endif
+constexpr float kUnscaleK = KV4_UNPACK_K ? kCvtUnscale : 1.0f;
+constexpr float kUnscaleV = KV4_UNPACK_V ? kCvtUnscale : 1.0f;
+__device__ __forceinline__ void unpack_k(uint32_t w, uint32_t (&p)[4]) {
+#if KV4_UNPACK_K
+  nib_pairs_k(w, p);
+#else
+  nib_pairs_k_or(w, p);
+#endif
+}
+__device__ __forceinline__ void unpack_v(uint32_t x, uint32_t (&p)[4]) {
+#if KV4_UNPACK_V
+  nib_pairs_v(x, p);
+#else
+  nib_pairs_v_or(x, p);
+#endif
+}
+
 // INT8 stage: K codes | V codes | K scales | V scales
 constexpr int kOffVc8 = 2048, kOffKs8 = 4096, kOffVs8 = 4128, kInt8Bytes = 4160;
 
@@ -551,8 +576,9 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 
   // ---- query fragments (B operand of QK^T). Lane column gid = (slot gid/CPH, query
   // gid%CPH); slot hs's fragments are zero unless the column is in slot hs.
-  // group g: k-tile 0 b01 = (q[32g+8tig], q[..+2]), b23 = (q[..+4], q[..+6]);
-  //          k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7])
+  // group g, with the fp8-conversion unpack: k-tile 0 b01 = (q[32g+8tig], q[..+2]),
+  // b23 = (q[..+4], q[..+6]); k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7]).
+  // With the exponent-bias unpack the pairs are (0,4) (1,5) | (2,6) (3,7).
   uint32_t qb[HPW][4][2][2];
   float qsum_own[4];
   bool qbad = false;
@@ -564,9 +590,15 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
+#if KV4_UNPACK_K
       // pairs matching nib_pairs_k: (0,2) (4,6) (1,3) (5,7)
       const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.y << 16), (v.z & 0xFFFFu) | (v.w << 16),
                               (v.x >> 16) | (v.y & 0xFFFF0000u), (v.z >> 16) | (v.w & 0xFFFF0000u)};
+#else
+      // pairs matching nib_pairs_k_or: (0,4) (1,5) (2,6) (3,7)
+      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.z << 16), (v.x >> 16) | (v.z & 0xFFFF0000u),
+                              (v.y & 0xFFFFu) | (v.w << 16), (v.y >> 16) | (v.w & 0xFFFF0000u)};
+#endif
       float sum = 0.f;
       uint32_t f16[4];
 #pragma unroll
@@ -630,7 +662,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
     const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kp_off + t0 * 16),
                          *reinterpret_cast<const uint4 *>(sp + kp_off + t1 * 16)};
-    // sc*: sum_g scale_g * (q . c)_g / 512 (codes enter the MMA scaled by 2^-9);
+    // sc*: sum_g scale_g * (q . c)_g / kUnscaleK (codes may enter the MMA scaled by 2^-9);
     // mn*: sum_g min_g * sum_g(q)
     float2 sc0 = make_float2(0.f, 0.f), sc1 = make_float2(0.f, 0.f);
     float2 mn0 = make_float2(0.f, 0.f), mn1 = make_float2(0.f, 0.f);
@@ -646,8 +678,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t pl[4], ph[4];
-          nib_pairs_k(kw[hs][2 * gg], pl);
-          nib_pairs_k(kw[hs][2 * gg + 1], ph);
+          unpack_k(kw[hs][2 * gg], pl);
+          unpack_k(kw[hs][2 * gg + 1], ph);
           mma_f16(acc, pl[0], ph[0], pl[1], ph[1], qb[hs][g][0][0], qb[hs][g][0][1]);
           mma_f16(acc, pl[2], ph[2], pl[3], ph[3], qb[hs][g][1][0], qb[hs][g][1][1]);
         }
@@ -660,7 +692,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         mn1 = ffma2(make_float2(f1.y, f1.y), qs[g], mn1);
       }
     }
-    const float2 k512 = make_float2(kCvtUnscale * kScaleLog2, kCvtUnscale * kScaleLog2);
+    const float2 k512 = make_float2(kUnscaleK * kScaleLog2, kUnscaleK * kScaleLog2);
     const float2 k1 = make_float2(kScaleLog2, kScaleLog2);
     const float2 sl0 = ffma2(sc0, k512, fmul2(mn0, k1));
     const float2 sl1 = ffma2(sc1, k512, fmul2(mn1, k1));
@@ -736,8 +768,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t vl[4], vh[4];
-          nib_pairs_v(vw[hs][2 * gg], vl);
-          nib_pairs_v(vw[hs][2 * gg + 1], vh);
+          unpack_v(vw[hs][2 * gg], vl);
+          unpack_v(vw[hs][2 * gg + 1], vh);
           const uint32_t *pb = x.ptile + ((hs * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
           const uint32_t b01 = pb[0], b23 = pb[4];
           mma_f16(o[g][0], vl[0], vl[1], vh[0], vh[1], b01, b23);
@@ -769,11 +801,11 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         float *rr = rec + j * kRecordFloats;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          // V codes entered the MMA scaled by 2^-9
-          const float4 v = make_float4(fmaf(o[g][0][e], kCvtUnscale, mt[g][e]),
-                                       fmaf(o[g][0][2 + e], kCvtUnscale, mt[g][e]),
-                                       fmaf(o[g][1][e], kCvtUnscale, mt[g][e]),
-                                       fmaf(o[g][1][2 + e], kCvtUnscale, mt[g][e]));
+          // V codes may have entered the MMA scaled by 2^-9
+          const float4 v = make_float4(fmaf(o[g][0][e], kUnscaleV, mt[g][e]),
+                                       fmaf(o[g][0][2 + e], kUnscaleV, mt[g][e]),
+                                       fmaf(o[g][1][e], kUnscaleV, mt[g][e]),
+                                       fmaf(o[g][1][2 + e], kUnscaleV, mt[g][e]));
           *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
         }
         if (gid == 0) {

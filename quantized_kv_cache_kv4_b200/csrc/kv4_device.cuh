@@ -191,6 +191,18 @@ __device__ __forceinline__ void nib_pairs_v(uint32_t x, uint32_t (&p)[4]) {
   p[3] = cvt_e4m3x2(hi >> 16);
 }
 
+// V word from a transposed ldmatrix through the exponent-bias OR (exact codes, unscaled):
+// p[k] = (t0 dim k, t1 dim k); nibbles 0 and 2 of each half sit in the low mantissa
+// bits, nibbles 1 and 3 are masked in place as 1024 + 16c and brought back by x/16 - 64.
+__device__ __forceinline__ void nib_pairs_v_or(uint32_t x, uint32_t (&p)[4]) {
+  uint32_t q[4];
+  nib_pairs4(x, q);  // q[i] = (nibble i, nibble i+4) = (t0 dim i, t1 dim i)
+  p[0] = q[0]; p[1] = q[1]; p[2] = q[2]; p[3] = q[3];
+}
+
+// K word through the exponent-bias OR (exact codes, unscaled): p[i] = (n_i, n_{i+4}).
+__device__ __forceinline__ void nib_pairs_k_or(uint32_t w, uint32_t (&p)[4]) { nib_pairs4(w, p); }
+
 // ---------------------------------------------------------------------------
 // packed fp32 pairs (sm_100 f32x2 FMA pipe operations)
 // ---------------------------------------------------------------------------
