@@ -169,14 +169,19 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(uint32_t two_bytes) {
   return d;
 }
 
+// Both byte pairs of a word: lo = bytes (0, 1), hi = bytes (2, 3).
+__device__ __forceinline__ void cvt_e4m3x2x2(uint32_t four_bytes, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four_bytes));
+}
+
 // K word (8 nibbles n0..n7 of one token, n_i = dim i): fp16 pairs
 // p0 = (n0, n2), p1 = (n4, n6), p2 = (n1, n3), p3 = (n5, n7), each scaled by 2^-9.
 __device__ __forceinline__ void nib_pairs_k(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  p[0] = cvt_e4m3x2(lo);
-  p[1] = cvt_e4m3x2(lo >> 16);
-  p[2] = cvt_e4m3x2(hi);
-  p[3] = cvt_e4m3x2(hi >> 16);
+  cvt_e4m3x2x2(w & 0x0F0F0F0Fu, p[0], p[1]);
+  cvt_e4m3x2x2((w >> 4) & 0x0F0F0F0Fu, p[2], p[3]);
 }
 
 // V word from a transposed ldmatrix (token t0's nibbles d0..d3 in bits 0-15, token t1's
@@ -184,11 +189,8 @@ __device__ __forceinline__ void nib_pairs_k(uint32_t w, uint32_t (&p)[4]) {
 __device__ __forceinline__ void nib_pairs_v(uint32_t x, uint32_t (&p)[4]) {
   uint32_t y;
   asm("prmt.b32 %0, %1, %1, 0x3120;" : "=r"(y) : "r"(x));  // bytes t0(d0d1) t1(d0d1) t0(d2d3) t1(d2d3)
-  const uint32_t lo = y & 0x0F0F0F0Fu, hi = (y >> 4) & 0x0F0F0F0Fu;
-  p[0] = cvt_e4m3x2(lo);
-  p[1] = cvt_e4m3x2(hi);
-  p[2] = cvt_e4m3x2(lo >> 16);
-  p[3] = cvt_e4m3x2(hi >> 16);
+  cvt_e4m3x2x2(y & 0x0F0F0F0Fu, p[0], p[2]);
+  cvt_e4m3x2x2((y >> 4) & 0x0F0F0F0Fu, p[1], p[3]);
 }
 
 // V word from a transposed ldmatrix through the exponent-bias OR (exact codes, unscaled):
