@@ -49,6 +49,11 @@ constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(1
 #ifndef KV4_UNPACK_V
 #define KV4_UNPACK_V 1
 #endif
+// QK^T on the integer tensor-core path: K codes as bytes, the query as a 15-bit fixed
+// point split into two byte slices, exact int32 sums (1); or fp16 codes x fp16 query (0).
+#ifndef KV4_QK_INT8
+#define KV4_QK_INT8 1
+#endif
 constexpr float kUnscaleK = KV4_UNPACK_K ? kCvtUnscale : 1.0f;
 constexpr float kUnscaleV = KV4_UNPACK_V ? kCvtUnscale : 1.0f;
 __device__ __forceinline__ void unpack_k(uint32_t w, uint32_t (&p)[4]) {
@@ -579,6 +584,69 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   // group g, with the fp8-conversion unpack: k-tile 0 b01 = (q[32g+8tig], q[..+2]),
   // b23 = (q[..+4], q[..+6]); k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7]).
   // With the exponent-bias unpack the pairs are (0,4) (1,5) | (2,6) (3,7).
+#if KV4_QK_INT8
+  // Integer path: q = qstep * (256*hi + lo) with qstep = 2^e chosen per query so that
+  // |256*hi + lo| < 2^14; b0 holds dims 8tig+{0,2,4,6} and b1 dims 8tig+{1,3,5,7} of a
+  // group (the low and high nibbles of the lane's K word), as bytes.
+  uint32_t qh[HPW][4][2], ql[HPW][4][2];
+  float qsum_own[4];
+  float qstep_own;
+  {
+    const int hs_b = gid / CPH, jb = gid % CPH;
+    const bool live = jb < G && hs_b < nh;
+    const uint16_t *qrow =
+        q + (static_cast<size_t>(b) * H * G + (h0 + hs_b) * G + jb) * kHeadDim;
+    float qv[4][8];
+    float amax = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        qv[g][2 * i] = __uint_as_float(w4[i] << 16);
+        qv[g][2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+        sum += qv[g][2 * i] + qv[g][2 * i + 1];
+        amax = fmaxf(amax, fmaxf(fabsf(qv[g][2 * i]), fabsf(qv[g][2 * i + 1])));
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      qsum_own[g] = sum;  // sum over the group's 32 dims for column gid
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int ex = 0;
+    if (amax > 0.f) {
+      frexpf(amax, &ex);  // amax < 2^ex
+      ex -= 14;
+    }
+    const float inv = ldexpf(1.0f, -ex);
+    qstep_own = ldexpf(1.0f, ex);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int qi = __float2int_rn(qv[g][i] * inv);  // exact scaling by 2^-ex
+        const int sel = i & 1, byte = i >> 1;           // dim 8tig+i -> b[i&1], byte i>>1
+        lb[sel] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * byte);
+        hb[sel] |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * byte);
+      }
+#pragma unroll
+      for (int hs = 0; hs < HPW; ++hs) {
+        const bool mine = hs == hs_b;
+        qh[hs][g][0] = mine ? hb[0] : 0u;
+        qh[hs][g][1] = mine ? hb[1] : 0u;
+        ql[hs][g][0] = mine ? lb[0] : 0u;
+        ql[hs][g][1] = mine ? lb[1] : 0u;
+      }
+    }
+  }
+  float2 kq;  // qstep * log2(e)/sqrt(d) of the C-fragment columns (2tig, 2tig+1)
+  kq.x = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig)) * kScaleLog2;
+  kq.y = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig + 1)) * kScaleLog2;
+#else
   uint32_t qb[HPW][4][2][2];
   float qsum_own[4];
   bool qbad = false;
@@ -617,6 +685,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     }
   }
   if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
+#endif
   float2 qs[4];  // column (2tig, 2tig+1) sums, matching the C-fragment columns
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -674,6 +743,20 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
       for (int gg = 0; gg < 2; ++gg) {
         const int g = 2 * gp + gg;
+#if KV4_QK_INT8
+        int32_t ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int hs = 0; hs < HPW; ++hs) {
+          const uint32_t wlo = kw[hs][2 * gg], whi = kw[hs][2 * gg + 1];
+          const uint32_t a0 = wlo & 0x0F0F0F0Fu, a1 = whi & 0x0F0F0F0Fu;
+          const uint32_t a2 = (wlo >> 4) & 0x0F0F0F0Fu, a3 = (whi >> 4) & 0x0F0F0F0Fu;
+          mma_u8s8(ah, a0, a1, a2, a3, qh[hs][g][0], qh[hs][g][1]);
+          mma_u8u8(al, a0, a1, a2, a3, ql[hs][g][0], ql[hs][g][1]);
+        }
+        float acc[4];  // exact integer dot products, |.| < 2^24
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ah[i] * 256 + al[i]);
+#else
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
@@ -683,6 +766,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
           mma_f16(acc, pl[0], ph[0], pl[1], ph[1], qb[hs][g][0][0], qb[hs][g][0][1]);
           mma_f16(acc, pl[2], ph[2], pl[3], ph[3], qb[hs][g][1][0], qb[hs][g][1][1]);
         }
+#endif
         const uint32_t w0 = g == 0 ? kp[0].x : g == 1 ? kp[0].y : g == 2 ? kp[0].z : kp[0].w;
         const uint32_t w1 = g == 0 ? kp[1].x : g == 1 ? kp[1].y : g == 2 ? kp[1].z : kp[1].w;
         const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
@@ -692,7 +776,11 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         mn1 = ffma2(make_float2(f1.y, f1.y), qs[g], mn1);
       }
     }
+#if KV4_QK_INT8
+    const float2 k512 = kq;  // the integer dot products are in units of qstep
+#else
     const float2 k512 = make_float2(kUnscaleK * kScaleLog2, kUnscaleK * kScaleLog2);
+#endif
     const float2 k1 = make_float2(kScaleLog2, kScaleLog2);
     const float2 sl0 = ffma2(sc0, k512, fmul2(mn0, k1));
     const float2 sl1 = ffma2(sc1, k512, fmul2(mn1, k1));

@@ -99,6 +99,28 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a01, uint32_t a2
       : "r"(a01), "r"(a23), "r"(a45), "r"(a67), "r"(b01), "r"(b23));
 }
 
+// D(16x8, s32) += A(16x32, u8, row) * B(32x8, s8 or u8, col). Fragments, lane = 4*gid+tig:
+//   A: a0 = (row gid, k 4tig..+3), a1 = (row gid+8, k 4tig..+3),
+//      a2 = (row gid, k 16+4tig..+3), a3 = (row gid+8, k 16+4tig..+3)
+//   B: b0 = (k 4tig..+3, col gid), b1 = (k 16+4tig..+3, col gid); C as for mma_f16.
+__device__ __forceinline__ void mma_u8s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_u8u8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
