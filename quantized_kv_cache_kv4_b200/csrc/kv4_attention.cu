@@ -145,29 +145,14 @@ __device__ int block_scan(int v, int *warp_sums, int *total) {
 // (sequence, region, kv head). Long work first keeps the end of the kernel short; the
 // natural order inside a class keeps the kv heads of one page and the sequences that
 // share a prompt next to each other, so shared pages are read while they are in L2.
-#ifndef KV4_PLAN_ORDER
-#define KV4_PLAN_ORDER 2  // 0: one class (natural order), 1: full chunks first, 2: four classes
-#endif
-constexpr int kClasses = 4;
-__device__ __forceinline__ int class_slot(int k) {
-#if KV4_PLAN_ORDER == 0
-  return 0 * k;
-#elif KV4_PLAN_ORDER == 1
-  return k == 0 ? 0 : 1;
-#else
-  return k;
-#endif
-}
-__device__ __forceinline__ int chunk_class(int pages, int C) {
-  return pages >= C ? 0 : (2 * pages >= C ? 1 : 3);
-}
-
-// Per-sequence entry counts per class.
+// (Class counters are plain scalars: a runtime-indexed array would live in local memory.)
 struct SeqPlan {
   Regions g;
-  int pages;          // INT4 pages of the sequence's INT4 range
-  int pairs;          // regions (protected set + INT4 chunks)
-  int e[kClasses];    // entries per class slot
+  int pages;   // INT4 pages of the sequence's INT4 range
+  int pairs;   // regions (protected set + INT4 chunks)
+  int nfull;   // INT4 chunks of exactly chunk_pages pages
+  int e_full, e_long, e_prot, e_short;  // entries per class
+  bool last_long;  // the shorter last chunk (if any) has at least half the pages
 };
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspace w,
@@ -188,66 +173,70 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     sp.g = regions_of(L, S, R, C);
     sp.pairs = sp.g.has_prot + sp.g.n_chunks;
     sp.pages = sp.g.n_chunks ? (sp.g.int4_hi - 1) / kPage - sp.g.first_page + 1 : 0;
-#pragma unroll
-    for (int k = 0; k < kClasses; ++k) sp.e[k] = 0;
-    sp.e[class_slot(2)] += sp.g.has_prot * H;
-    const int nfull = sp.pages / C;
-    sp.e[class_slot(0)] += nfull * nslots;
-    if (sp.g.n_chunks > nfull) sp.e[class_slot(chunk_class(sp.pages - nfull * C, C))] += nslots;
+    sp.nfull = sp.pages / C;
+    const bool has_last = sp.g.n_chunks > sp.nfull;
+    sp.last_long = 2 * (sp.pages - sp.nfull * C) >= C;
+    sp.e_full = sp.nfull * nslots;
+    sp.e_prot = sp.g.has_prot * H;
+    sp.e_long = has_last && sp.last_long ? nslots : 0;
+    sp.e_short = has_last && !sp.last_long ? nslots : 0;
+    return sp;
+  };
+  auto empty_plan = [] {
+    SeqPlan sp{};
     return sp;
   };
 
   // pass 1: totals
-  int tp = 0, te[kClasses] = {0, 0, 0, 0};
+  int tp = 0, tf = 0, tl = 0, tpr = 0, ts = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    SeqPlan sp{};
-    if (b < B) sp = plan_of(b, false);
+    const SeqPlan sp = b < B ? plan_of(b, false) : empty_plan();
     int t;
     block_scan(sp.pairs, warp_sums, &t);
     tp += t;
-#pragma unroll
-    for (int k = 0; k < kClasses; ++k) {
-      block_scan(sp.e[k], warp_sums, &t);
-      te[k] += t;
-    }
+    block_scan(sp.e_full, warp_sums, &t);
+    tf += t;
+    block_scan(sp.e_long, warp_sums, &t);
+    tl += t;
+    block_scan(sp.e_prot, warp_sums, &t);
+    tpr += t;
+    block_scan(sp.e_short, warp_sums, &t);
+    ts += t;
   }
-  const int te_all = te[0] + te[1] + te[2] + te[3];
+  const int te_all = tf + tl + tpr + ts;
   const bool fits = tp <= w.cap_pairs && te_all <= w.cap_entries;
 
   // pass 2: partial offsets and entries (every unit empty if the workspace is too small)
-  int run_p = 0, run_e[kClasses] = {0, te[0], te[0] + te[1], te[0] + te[1] + te[2]};
+  int run_p = 0, run_f = 0, run_l = tf, run_pr = tf + tl, run_s = tf + tl + tpr;
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    SeqPlan sp{};
-    if (b < B) sp = plan_of(b, true);
-    if (!fits) {
-      sp.pairs = 0;
-#pragma unroll
-      for (int k = 0; k < kClasses; ++k) sp.e[k] = 0;
-    }
+    SeqPlan sp = b < B ? plan_of(b, true) : empty_plan();
+    if (!fits) sp = empty_plan();
     int t;
     const int po = run_p + block_scan(sp.pairs, warp_sums, &t);
     run_p += t;
-    int eo[kClasses];
-#pragma unroll
-    for (int k = 0; k < kClasses; ++k) {
-      eo[k] = run_e[k] + block_scan(sp.e[k], warp_sums, &t);
-      run_e[k] += t;
-    }
+    int ef = run_f + block_scan(sp.e_full, warp_sums, &t);
+    run_f += t;
+    const int el = run_l + block_scan(sp.e_long, warp_sums, &t);
+    run_l += t;
+    int epr = run_pr + block_scan(sp.e_prot, warp_sums, &t);
+    run_pr += t;
+    const int es = run_s + block_scan(sp.e_short, warp_sums, &t);
+    run_s += t;
     if (b >= B) continue;
     for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * sp.pairs;
-    if (sp.pairs) {
-      const Regions &g = sp.g;
-      if (g.has_prot) {
-        const int k = class_slot(2);
-        for (int h = 0; h < H; ++h) w.entries[eo[k]++] = make_int4(b, 0, h, 1);
-      }
-      for (int ch = 0; ch < g.n_chunks; ++ch) {
-        const int k = class_slot(chunk_class(min(C, sp.pages - ch * C), C));
-        for (int s = 0; s < nslots; ++s)
-          w.entries[eo[k]++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
-      }
+    if (sp.pairs == 0) continue;
+    const Regions &g = sp.g;
+    if (g.has_prot)
+      for (int h = 0; h < H; ++h) w.entries[epr++] = make_int4(b, 0, h, 1);
+    for (int ch = 0; ch < sp.nfull; ++ch)
+      for (int s = 0; s < nslots; ++s)
+        w.entries[ef++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
+    if (g.n_chunks > sp.nfull) {
+      int e = sp.last_long ? el : es;
+      for (int s = 0; s < nslots; ++s)
+        w.entries[e++] = make_int4(b, g.has_prot + sp.nfull, s * hpw, min(hpw, H - s * hpw));
     }
   }
   if (threadIdx.x == 0) {
@@ -912,13 +901,15 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 //   M = max m_r, Lambda = sum l_r e^(m_r - M), O = sum acc_r e^(m_r - M) / Lambda,
 //   lse = M + ln Lambda, over live regions (l_r > 0); no live region gives O = 0,
 //   lse = -inf.
-// The region weights e^(m_r - M) are computed with the regions spread over the lanes
-// (fixed assignment and reduction tree); the weighted sum then walks the regions in
-// order with lane i owning dims 4i..4i+3, its loads independent of each other. The
-// arithmetic order is fixed, so the result is deterministic.
+// Regions are taken in batches of 8: the lanes first issue every load of the batch (the
+// region maxima and sums spread over the lanes, each lane's 4 dims of every record),
+// then the batch's weights are formed and added in region order. The arithmetic order
+// is fixed, so the result is deterministic; M is the running maximum over the batches
+// (with a rescale between batches, as in the online softmax).
 __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
                                                     const int32_t *__restrict__ offs, int n_units,
                                                     int G, Outputs o) {
+  constexpr int kBatch = 8;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= n_units * G) return;
@@ -927,42 +918,47 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
   auto rec_of = [&](int r) {
     return partials + (static_cast<size_t>(r0 + r) * G + j) * kRecordFloats;
   };
-  float M = -CUDART_INF_F;
-  for (int r = lane; r < n; r += 32) {
-    const float *rec = rec_of(r);
-    if (rec[kHeadDim + 1] > 0.f) M = fmaxf(M, rec[kHeadDim]);
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float lam = 0.f;
+  float M = -CUDART_INF_F, lam = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -CUDART_INF_F) {
-    for (int base = 0; base < n; base += 32) {
-      // weights of regions base .. base+31, one per lane
-      float wl = 0.f;
-      if (base + lane < n) {
-        const float *rec = rec_of(base + lane);
-        const float lr = rec[kHeadDim + 1];
-        if (lr > 0.f) {
-          wl = expf(rec[kHeadDim] - M);
-          lam = fmaf(lr, wl, lam);
-        }
-      }
-      const int cnt = min(32, n - base);
-#pragma unroll 4
-      for (int i = 0; i < cnt; ++i) {
-        const float wgt = __shfl_sync(0xffffffffu, wl, i);
-        const float4 a = reinterpret_cast<const float4 *>(rec_of(base + i))[lane];
-        if (wgt > 0.f) {
-          acc.x = fmaf(a.x, wgt, acc.x);
-          acc.y = fmaf(a.y, wgt, acc.y);
-          acc.z = fmaf(a.z, wgt, acc.z);
-          acc.w = fmaf(a.w, wgt, acc.w);
-        }
+  for (int base = 0; base < n; base += kBatch) {
+    const int cnt = min(kBatch, n - base);
+    float4 a[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (i < cnt) a[i] = __ldcg(reinterpret_cast<const float4 *>(rec_of(base + i)) + lane);
+    float mr = -CUDART_INF_F, lr = 0.f;
+    if (lane < cnt) {
+      const float *rec = rec_of(base + lane);
+      lr = __ldcg(rec + kHeadDim + 1);
+      mr = lr > 0.f ? __ldcg(rec + kHeadDim) : -CUDART_INF_F;
+    }
+    float bm = mr;
+#pragma unroll
+    for (int off = 4; off; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+    bm = __shfl_sync(0xffffffffu, bm, 0);  // max over the batch (lanes 0..7)
+    if (bm == -CUDART_INF_F) continue;     // no live region in this batch
+    const float Mn = fmaxf(M, bm);
+    if (Mn != M) {  // rescale what was accumulated under the old maximum
+      const float sc = expf(M - Mn);
+      acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
+      lam *= sc;
+      M = Mn;
+    }
+    const float wl = lr > 0.f ? expf(mr - M) : 0.f;  // this lane's region weight
+    float ls = lr * wl;
+#pragma unroll
+    for (int off = 4; off; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+    lam += __shfl_sync(0xffffffffu, ls, 0);
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const float wgt = __shfl_sync(0xffffffffu, wl, i);
+      if (i < cnt && wgt > 0.f) {
+        acc.x = fmaf(a[i].x, wgt, acc.x);
+        acc.y = fmaf(a[i].y, wgt, acc.y);
+        acc.z = fmaf(a[i].z, wgt, acc.z);
+        acc.w = fmaf(a[i].w, wgt, acc.w);
       }
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) lam += __shfl_xor_sync(0xffffffffu, lam, off);
   }
   const float inv = lam > 0.f ? 1.0f / lam : 0.f;
   const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
