@@ -203,6 +203,33 @@ kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offse
                               void *out, float *out_f32, float *lse,
                               kv4_stream_t stream);
 
+/*
+ * Decode attention for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call; it exists for callers of this library
+ * that cannot call cudaMalloc (code that must not touch the allocator, e.g. inside a
+ * fixed memory pool or a runtime that owns all device memory) and so cannot supply the
+ * workspace kv4_decode_attention needs. Same arguments, semantics and results as
+ * kv4_decode_attention, minus the workspace: the scratch space is a fixed array of
+ * KV4_NOALLOC_SCRATCH_BYTES bytes in the library's device image, which every GPU that
+ * loads the library holds until the process exits. Nothing is allocated or freed.
+ *   - A batch whose kv4_workspace_size(cfg, num_seqs, max_seq_len) exceeds
+ *     KV4_NOALLOC_SCRATCH_BYTES is rejected with KV4_ERR_WORKSPACE_TOO_SMALL.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before capturing a stream into a CUDA graph.
+ *   - All calls share the one array per device: calls whose kernels overlap on the GPU
+ *     (different streams without ordering between them) race and give wrong results.
+ *     Calls ordered on one stream are safe; each call re-initialises what it reads.
+ */
+#define KV4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+kv4_status kv4_decode_attention_noalloc(const kv4_config *cfg, const kv4_int4_pool *pool,
+                                        const kv4_int8_side *side, const kv4_batch *batch,
+                                        const void *q, void *out, float *out_f32, float *lse,
+                                        int32_t *err_flag, kv4_stream_t stream);
+
+/* Size of the fixed scratch array kv4_decode_attention_noalloc uses, in bytes. */
+size_t kv4_noalloc_scratch_bytes(void);
+
 /* Human-readable name of a status code (static string). */
 const char *kv4_status_string(kv4_status status);
 

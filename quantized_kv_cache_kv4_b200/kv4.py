@@ -29,7 +29,8 @@ PAGE = 16
 GROUP = 32
 
 EXPORTS = ("kv4_workspace_size", "kv4_quantize_append", "kv4_decode_attention",
-           "kv4_regional_merge", "kv4_status_string", "kv4_version")
+           "kv4_regional_merge", "kv4_status_string", "kv4_version",
+           "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes")
 
 
 class Config(ctypes.Structure):
@@ -80,6 +81,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kv4_regional_merge.restype = ctypes.c_int
     lib.kv4_regional_merge.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        P, P, P, P]
+    lib.kv4_decode_attention_noalloc.restype = ctypes.c_int
+    lib.kv4_decode_attention_noalloc.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Int4Pool),
+                                                 ctypes.POINTER(Int8Side), ctypes.POINTER(Batch),
+                                                 P, P, P, P, P, P]
+    lib.kv4_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kv4_noalloc_scratch_bytes.argtypes = []
     lib.kv4_status_string.restype = ctypes.c_char_p
     lib.kv4_status_string.argtypes = [ctypes.c_int]
     lib.kv4_version.restype = ctypes.c_int32
@@ -214,6 +221,25 @@ def decode_attention(cache: Cache, batch: BatchTensors, q: torch.Tensor, out: to
                                    _ptr(out_f32), _ptr(lse), _ptr(workspace),
                                    workspace.numel(), _ptr(err), _stream(stream))
     _check(st, "kv4_decode_attention")
+
+
+def decode_attention_noalloc(cache: Cache, batch: BatchTensors, q: torch.Tensor,
+                             out: torch.Tensor, out_f32: torch.Tensor | None = None,
+                             lse: torch.Tensor | None = None, err: torch.Tensor | None = None,
+                             stream=None):
+    """decode_attention without a workspace argument, for callers that cannot allocate
+    device memory: the library's fixed scratch array (kv4_noalloc_scratch_bytes()) is
+    used instead. Calls that overlap on the GPU race on that array."""
+    pool, side, bs = cache.pool_struct(), cache.side_struct(), batch.struct()
+    st = _lib.kv4_decode_attention_noalloc(ctypes.byref(cache.cfg), ctypes.byref(pool),
+                                           ctypes.byref(side), ctypes.byref(bs), _ptr(q),
+                                           _ptr(out), _ptr(out_f32), _ptr(lse), _ptr(err),
+                                           _stream(stream))
+    _check(st, "kv4_decode_attention_noalloc")
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_lib.kv4_noalloc_scratch_bytes())
 
 
 def regional_merge(partials: torch.Tensor, region_offsets: torch.Tensor, group: int,
