@@ -4,17 +4,23 @@
 // merge", ai4snews summary, "Interpretation" para. 3).
 //
 // Kernels:
-//   plan_kernel  one CTA: turns seq_lens into a work list. Region 0 of a sequence is its
-//                INT8 protected set (one entry per kv head); regions 1.. are chunks of
-//                `chunk_pages` INT4 pages (one entry per one or two kv heads).
+//   plan_kernel  turns seq_lens into a work list. Region 0 of a sequence is its INT8
+//                protected set (one entry per kv head); regions 1.. are chunks of
+//                `chunk_pages` INT4 pages (one entry per one or two kv heads). Entries
+//                come in four classes (full chunks, long partial chunks, protected sets,
+//                short chunks) so that the longest work starts first.
 //   attn_kernel  persistent; every warp repeatedly takes one entry from an atomic counter
 //                and computes the partial softmax state of that region for the query
 //                heads of its kv head(s). Page tiles stream through a per-warp ring of
 //                shared-memory stages filled by bulk async copies (TMA engine, mbarrier
-//                completion). QK^T and PV run on the tensor cores (mma m16n8k16, fp16 in,
-//                fp32 accumulate) directly on the integer codes: codes are exact in fp16,
-//                and the per-group scale/min are applied outside the dot products, so no
-//                dequantised K/V is ever materialised.
+//                completion). Both products run on the tensor cores directly on the
+//                integer codes, and the per-group scale/min are applied outside them, so
+//                no dequantised K/V is ever materialised:
+//                  QK^T  integer MMA (m16n8k32): K codes as bytes times the query in
+//                        15-bit fixed point split into a signed high and an unsigned low
+//                        byte, exact int32 dot products;
+//                  PV    fp16 MMA (m16n8k16, fp32 accumulate): V codes converted exactly
+//                        by the fp8 conversion, P' = p * vscale rounded once to fp16.
 //                With G <= 4 query heads per kv head one warp serves two kv heads: the MMA
 //                N dimension (8) holds head A's queries in columns 0-3 and head B's in
 //                columns 4-7 (zeros in the other half of each B operand), so every lane's
@@ -41,35 +47,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegBig = -1.0e30f;  // running-max start: finite, so e^(m_old-m_new) is 0 not NaN
 constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
-// Nibble unpack of the INT4 codes: 1 = through the fp8 conversion (codes scaled by 2^-9),
-// 0 = through the exponent-bias OR (exact codes). Chosen per operand by measurement.
-#ifndef KV4_UNPACK_K
-#define KV4_UNPACK_K 1
-#endif
-#ifndef KV4_UNPACK_V
-#define KV4_UNPACK_V 1
-#endif
-// QK^T on the integer tensor-core path: K codes as bytes, the query as a 15-bit fixed
-// point split into two byte slices, exact int32 sums (1); or fp16 codes x fp16 query (0).
-#ifndef KV4_QK_INT8
-#define KV4_QK_INT8 1
-#endif
-constexpr float kUnscaleK = KV4_UNPACK_K ? kCvtUnscale : 1.0f;
-constexpr float kUnscaleV = KV4_UNPACK_V ? kCvtUnscale : 1.0f;
-__device__ __forceinline__ void unpack_k(uint32_t w, uint32_t (&p)[4]) {
-#if KV4_UNPACK_K
-  nib_pairs_k(w, p);
-#else
-  nib_pairs_k_or(w, p);
-#endif
-}
-__device__ __forceinline__ void unpack_v(uint32_t x, uint32_t (&p)[4]) {
-#if KV4_UNPACK_V
-  nib_pairs_v(x, p);
-#else
-  nib_pairs_v_or(x, p);
-#endif
-}
+// V codes enter the PV product through the fp8 conversion: a byte b in 0..15 read as
+// e4m3 is exactly b * 2^-9, so the products are scaled by 2^-9 and the 2^9 is applied
+// once to the output.
+constexpr float kUnscaleV = kCvtUnscale;
 
 // INT8 stage: K codes | V codes | K scales | V scales
 constexpr int kOffVc8 = 2048, kOffKs8 = 4096, kOffVs8 = 4128, kInt8Bytes = 4160;
@@ -109,125 +90,126 @@ __device__ __forceinline__ Regions regions_of(int L, int S, int R, int C) {
 }
 
 // ---------------------------------------------------------------------------
-// plan: one CTA, 1024 threads
+// plan: a few CTAs of 1024 threads. Every CTA scans all sequences (a few KB of lengths)
+// to get the same offsets, then writes the entries of its own slice of sequences only,
+// so the scattered 16-byte entry stores are spread over several SMs.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
+constexpr int kPlanSeqsPerCta = 32;  // sequences per CTA, until kPlanMaxCtas is reached
+constexpr int kPlanMaxCtas = 148;
+constexpr int kScanN = 5;            // values scanned together per sequence
 
-// Exclusive block-wide scan (warp shuffles + one warp over the 32 warp totals).
-__device__ int block_scan(int v, int *warp_sums, int *total) {
+// Exclusive block-wide scan of kScanN values at once (warp shuffles + one warp over the
+// 32 warp totals per value); totals returned in tot.
+__device__ void block_scan_n(int (&v)[kScanN], int (&tot)[kScanN], int (*warp_sums)[32]) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
+  int x[kScanN];
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) warp_sums[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    int s = warp_sums[lane];
+  for (int i = 0; i < kScanN; ++i) {
+    x[i] = v[i];
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += y;
+      const int y = __shfl_up_sync(0xffffffffu, x[i], off);
+      if (lane >= off) x[i] += y;
     }
-    warp_sums[lane] = s;
+    if (lane == 31) warp_sums[i][wid] = x[i];
   }
   __syncthreads();
-  const int base = wid ? warp_sums[wid - 1] : 0;
-  *total = warp_sums[31];
+  if (wid < kScanN) {
+    int t = warp_sums[wid][lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, off);
+      if (lane >= off) t += y;
+    }
+    warp_sums[wid][lane] = t;
+  }
   __syncthreads();
-  return base + x - v;
+#pragma unroll
+  for (int i = 0; i < kScanN; ++i) {
+    const int base = wid ? warp_sums[i][wid - 1] : 0;
+    tot[i] = warp_sums[i][31];
+    v[i] = base + x[i] - v[i];
+  }
+  __syncthreads();
 }
 
-// Work classes, processed in this order: full-length INT4 chunks, INT4 chunks of at
-// least half the length, protected sets, short INT4 chunks. Inside a class the order is
-// (sequence, region, kv head). Long work first keeps the end of the kernel short; the
-// natural order inside a class keeps the kv heads of one page and the sequences that
-// share a prompt next to each other, so shared pages are read while they are in L2.
-// (Class counters are plain scalars: a runtime-indexed array would live in local memory.)
 struct SeqPlan {
   Regions g;
   int pages;   // INT4 pages of the sequence's INT4 range
-  int pairs;   // regions (protected set + INT4 chunks)
   int nfull;   // INT4 chunks of exactly chunk_pages pages
-  int e_full, e_long, e_prot, e_short;  // entries per class
   bool last_long;  // the shorter last chunk (if any) has at least half the pages
+  // scanned values: regions (protected set + INT4 chunks), then entries per class
+  // (full chunks, long partial chunks, protected sets, short chunks)
+  int n[kScanN];
 };
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspace w,
                                                             int32_t *err) {
-  __shared__ int warp_sums[32];
+  __shared__ int warp_sums[kScanN][32];
   const int B = c.num_seqs, H = c.num_kv_heads, C = w.chunk_pages;
   const int S = c.num_sinks, R = c.num_recent;
   const int hpw = w.heads_per_warp;
   const int nslots = (H + hpw - 1) / hpw;
+  const int per = (B + gridDim.x - 1) / gridDim.x;  // sequences written by this CTA
+  const int my_lo = blockIdx.x * per;
+  const int my_hi = min(B, my_lo + per);
 
-  auto plan_of = [&](int b, bool flag) {
-    SeqPlan sp;
+  auto plan_of = [&](int b) {
+    SeqPlan sp{};
+    if (b >= B) return sp;
     int L = c.seq_lens[b];
     if (L < 0 || L > c.max_pages * kPage) {
-      if (flag) set_err(err, KV4_DEVERR_SEQ_LEN);
+      if (b >= my_lo && b < my_hi) set_err(err, KV4_DEVERR_SEQ_LEN);
       L = 0;
     }
     sp.g = regions_of(L, S, R, C);
-    sp.pairs = sp.g.has_prot + sp.g.n_chunks;
     sp.pages = sp.g.n_chunks ? (sp.g.int4_hi - 1) / kPage - sp.g.first_page + 1 : 0;
     sp.nfull = sp.pages / C;
     const bool has_last = sp.g.n_chunks > sp.nfull;
     sp.last_long = 2 * (sp.pages - sp.nfull * C) >= C;
-    sp.e_full = sp.nfull * nslots;
-    sp.e_prot = sp.g.has_prot * H;
-    sp.e_long = has_last && sp.last_long ? nslots : 0;
-    sp.e_short = has_last && !sp.last_long ? nslots : 0;
-    return sp;
-  };
-  auto empty_plan = [] {
-    SeqPlan sp{};
+    sp.n[0] = sp.g.has_prot + sp.g.n_chunks;
+    sp.n[1] = sp.nfull * nslots;
+    sp.n[2] = has_last && sp.last_long ? nslots : 0;
+    sp.n[3] = sp.g.has_prot * H;
+    sp.n[4] = has_last && !sp.last_long ? nslots : 0;
     return sp;
   };
 
-  // pass 1: totals
-  int tp = 0, tf = 0, tl = 0, tpr = 0, ts = 0;
+  // pass 1: totals over every sequence
+  int tot[kScanN] = {0, 0, 0, 0, 0};
   for (int base = 0; base < B; base += kPlanThreads) {
-    const int b = base + threadIdx.x;
-    const SeqPlan sp = b < B ? plan_of(b, false) : empty_plan();
-    int t;
-    block_scan(sp.pairs, warp_sums, &t);
-    tp += t;
-    block_scan(sp.e_full, warp_sums, &t);
-    tf += t;
-    block_scan(sp.e_long, warp_sums, &t);
-    tl += t;
-    block_scan(sp.e_prot, warp_sums, &t);
-    tpr += t;
-    block_scan(sp.e_short, warp_sums, &t);
-    ts += t;
+    SeqPlan sp = plan_of(base + threadIdx.x);
+    int t[kScanN];
+    block_scan_n(sp.n, t, warp_sums);
+#pragma unroll
+    for (int i = 0; i < kScanN; ++i) tot[i] += t[i];
   }
-  const int te_all = tf + tl + tpr + ts;
-  const bool fits = tp <= w.cap_pairs && te_all <= w.cap_entries;
+  const int te_all = tot[1] + tot[2] + tot[3] + tot[4];
+  const bool fits = tot[0] <= w.cap_pairs && te_all <= w.cap_entries;
 
-  // pass 2: partial offsets and entries (every unit empty if the workspace is too small)
-  int run_p = 0, run_f = 0, run_l = tf, run_pr = tf + tl, run_s = tf + tl + tpr;
-  for (int base = 0; base < B; base += kPlanThreads) {
+  // pass 2: offsets up to this CTA's slice; entries of the slice (every unit empty if
+  // the workspace is too small)
+  // class bases: full chunks at 0, then long partial chunks, protected sets, short chunks
+  int run[kScanN] = {0, 0, tot[1], tot[1] + tot[2], tot[1] + tot[2] + tot[3]};
+  for (int base = 0; base < my_hi; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    SeqPlan sp = b < B ? plan_of(b, true) : empty_plan();
-    if (!fits) sp = empty_plan();
-    int t;
-    const int po = run_p + block_scan(sp.pairs, warp_sums, &t);
-    run_p += t;
-    int ef = run_f + block_scan(sp.e_full, warp_sums, &t);
-    run_f += t;
-    const int el = run_l + block_scan(sp.e_long, warp_sums, &t);
-    run_l += t;
-    int epr = run_pr + block_scan(sp.e_prot, warp_sums, &t);
-    run_pr += t;
-    const int es = run_s + block_scan(sp.e_short, warp_sums, &t);
-    run_s += t;
-    if (b >= B) continue;
-    for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * po + h * sp.pairs;
-    if (sp.pairs == 0) continue;
+    SeqPlan sp = fits ? plan_of(b) : SeqPlan{};
+    int off[kScanN], t[kScanN];
+#pragma unroll
+    for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
+    block_scan_n(off, t, warp_sums);
+#pragma unroll
+    for (int i = 0; i < kScanN; ++i) {
+      off[i] += run[i];
+      run[i] += t[i];
+    }
+    if (b < my_lo || b >= my_hi) continue;
+    const int pairs = sp.n[0];
+    for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * off[0] + h * pairs;
+    if (pairs == 0) continue;
     const Regions &g = sp.g;
+    int ef = off[1], el = off[2], epr = off[3], es = off[4];
     if (g.has_prot)
       for (int h = 0; h < H; ++h) w.entries[epr++] = make_int4(b, 0, h, 1);
     for (int ch = 0; ch < sp.nfull; ++ch)
@@ -239,8 +221,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
         w.entries[e++] = make_int4(b, g.has_prot + sp.nfull, s * hpw, min(hpw, H - s * hpw));
     }
   }
-  if (threadIdx.x == 0) {
-    w.unit_offsets[B * H] = H * run_p;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    w.unit_offsets[B * H] = H * tot[0];
     *w.n_items = fits ? te_all : 0;
     *w.counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
@@ -573,7 +555,6 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   // group g, with the fp8-conversion unpack: k-tile 0 b01 = (q[32g+8tig], q[..+2]),
   // b23 = (q[..+4], q[..+6]); k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7]).
   // With the exponent-bias unpack the pairs are (0,4) (1,5) | (2,6) (3,7).
-#if KV4_QK_INT8
   // Integer path: q = qstep * (256*hi + lo) with qstep = 2^e chosen per query so that
   // |256*hi + lo| < 2^14; b0 holds dims 8tig+{0,2,4,6} and b1 dims 8tig+{1,3,5,7} of a
   // group (the low and high nibbles of the lane's K word), as bytes.
@@ -635,46 +616,6 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   float2 kq;  // qstep * log2(e)/sqrt(d) of the C-fragment columns (2tig, 2tig+1)
   kq.x = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig)) * kScaleLog2;
   kq.y = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig + 1)) * kScaleLog2;
-#else
-  uint32_t qb[HPW][4][2][2];
-  float qsum_own[4];
-  bool qbad = false;
-  {
-    const int hs_b = gid / CPH, jb = gid % CPH;
-    const bool live = jb < G && hs_b < nh;
-    const uint16_t *qrow =
-        q + (static_cast<size_t>(b) * H * G + (h0 + hs_b) * G + jb) * kHeadDim;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);  // bf16 dims +0..+7
-#if KV4_UNPACK_K
-      // pairs matching nib_pairs_k: (0,2) (4,6) (1,3) (5,7)
-      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.y << 16), (v.z & 0xFFFFu) | (v.w << 16),
-                              (v.x >> 16) | (v.y & 0xFFFF0000u), (v.z >> 16) | (v.w & 0xFFFF0000u)};
-#else
-      // pairs matching nib_pairs_k_or: (0,4) (1,5) (2,6) (3,7)
-      const uint32_t pr[4] = {(v.x & 0xFFFFu) | (v.z << 16), (v.x >> 16) | (v.z & 0xFFFF0000u),
-                              (v.y & 0xFFFFu) | (v.w << 16), (v.y >> 16) | (v.w & 0xFFFF0000u)};
-#endif
-      float sum = 0.f;
-      uint32_t f16[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sum += q_to_f16_pair(pr[i], f16[i], qbad);
-#pragma unroll
-      for (int hs = 0; hs < HPW; ++hs) {
-        const bool mine = hs == hs_b;
-        qb[hs][g][0][0] = mine ? f16[0] : 0u;
-        qb[hs][g][0][1] = mine ? f16[1] : 0u;
-        qb[hs][g][1][0] = mine ? f16[2] : 0u;
-        qb[hs][g][1][1] = mine ? f16[3] : 0u;
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      qsum_own[g] = sum;  // sum over the group's 32 dims for column gid
-    }
-  }
-  if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
-#endif
   float2 qs[4];  // column (2tig, 2tig+1) sums, matching the C-fragment columns
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
@@ -720,7 +661,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     // ---- logits: s = sum_g scale_g * (q . c)_g + min_g * sum_g(q), log2 units ----
     const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kp_off + t0 * 16),
                          *reinterpret_cast<const uint4 *>(sp + kp_off + t1 * 16)};
-    // sc*: sum_g scale_g * (q . c)_g / kUnscaleK (codes may enter the MMA scaled by 2^-9);
+    // sc*: sum_g scale_g * (q . c)_g in units of the query step;
     // mn*: sum_g min_g * sum_g(q)
     float2 sc0 = make_float2(0.f, 0.f), sc1 = make_float2(0.f, 0.f);
     float2 mn0 = make_float2(0.f, 0.f), mn1 = make_float2(0.f, 0.f);
@@ -732,7 +673,6 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
       for (int gg = 0; gg < 2; ++gg) {
         const int g = 2 * gp + gg;
-#if KV4_QK_INT8
         int32_t ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
@@ -745,17 +685,6 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         float acc[4];  // exact integer dot products, |.| < 2^24
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ah[i] * 256 + al[i]);
-#else
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int hs = 0; hs < HPW; ++hs) {
-          uint32_t pl[4], ph[4];
-          unpack_k(kw[hs][2 * gg], pl);
-          unpack_k(kw[hs][2 * gg + 1], ph);
-          mma_f16(acc, pl[0], ph[0], pl[1], ph[1], qb[hs][g][0][0], qb[hs][g][0][1]);
-          mma_f16(acc, pl[2], ph[2], pl[3], ph[3], qb[hs][g][1][0], qb[hs][g][1][1]);
-        }
-#endif
         const uint32_t w0 = g == 0 ? kp[0].x : g == 1 ? kp[0].y : g == 2 ? kp[0].z : kp[0].w;
         const uint32_t w1 = g == 0 ? kp[1].x : g == 1 ? kp[1].y : g == 2 ? kp[1].z : kp[1].w;
         const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
@@ -765,11 +694,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         mn1 = ffma2(make_float2(f1.y, f1.y), qs[g], mn1);
       }
     }
-#if KV4_QK_INT8
     const float2 k512 = kq;  // the integer dot products are in units of qstep
-#else
-    const float2 k512 = make_float2(kUnscaleK * kScaleLog2, kUnscaleK * kScaleLog2);
-#endif
     const float2 k1 = make_float2(kScaleLog2, kScaleLog2);
     const float2 sl0 = ffma2(sc0, k512, fmul2(mn0, k1));
     const float2 sl1 = ffma2(sc1, k512, fmul2(mn1, k1));
@@ -845,8 +770,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t vl[4], vh[4];
-          unpack_v(vw[hs][2 * gg], vl);
-          unpack_v(vw[hs][2 * gg + 1], vh);
+          nib_pairs_v(vw[hs][2 * gg], vl);
+          nib_pairs_v(vw[hs][2 * gg + 1], vh);
           const uint32_t *pb = x.ptile + ((hs * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
           const uint32_t b01 = pb[0], b23 = pb[4];
           mma_f16(o[g][0], vl[0], vl[1], vh[0], vh[1], b01, b23);
@@ -1025,7 +950,8 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
 // ---------------------------------------------------------------------------
 cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag,
                         cudaStream_t s) {
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(c, w, err_flag);
+  const int ctas = max(1, min(kPlanMaxCtas, (c.num_seqs + kPlanSeqsPerCta - 1) / kPlanSeqsPerCta));
+  plan_kernel<<<ctas, kPlanThreads, 0, s>>>(c, w, err_flag);
   return cudaGetLastError();
 }
 

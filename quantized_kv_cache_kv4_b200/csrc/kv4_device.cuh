@@ -134,7 +134,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
 }
 
 // ---------------------------------------------------------------------------
-// integer code -> fp16 without conversion instructions.
+// int8 code -> fp16 without conversion instructions.
 // binary16 with exponent field 25 (bits 0x6400) is 1024 + mantissa, so OR-ing a small
 // unsigned integer u <= 1023 into the mantissa gives exactly 1024 + u; subtracting
 // 1024 (or 1024 + 128 for offset-binary int8) is exact.
@@ -144,36 +144,7 @@ __device__ __forceinline__ uint32_t h2_sub(uint32_t x, uint32_t y) {
   return *reinterpret_cast<uint32_t *>(&r);
 }
 
-constexpr uint32_t kMagic1024x2 = 0x64006400u;  // (1024.0, 1024.0)
 constexpr uint32_t kMagic1152x2 = 0x64806480u;  // (1152.0, 1152.0)
-
-// Nibbles i and i+4 of a 32-bit word (i in 0..3) as an fp16 pair (low = nibble i).
-template <int I>
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
-  uint32_t x = ((w >> (4 * I)) & 0x000F000Fu) | kMagic1024x2;
-  return h2_sub(x, kMagic1024x2);
-}
-
-__device__ __forceinline__ uint32_t h2_fma(uint32_t x, uint32_t y, uint32_t z) {
-  __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&y),
-                      *reinterpret_cast<__half2 *>(&z));
-  return *reinterpret_cast<uint32_t *>(&r);
-}
-
-constexpr uint32_t kSixteenthX2 = 0x2C002C00u;  // (1/16, 1/16)
-constexpr uint32_t kMinus64X2 = 0xD400D400u;    // (-64, -64)
-
-// All four nibble pairs of a word with one shift: pairs 0 and 2 sit in the low
-// mantissa bits (1024 + c, exact after subtracting 1024); pairs 1 and 3 are masked in
-// place as 1024 + 16c and brought back exactly by x/16 - 64 in one fma.
-// Returns p[i] = (nibble i, nibble i+4) as fp16 pairs.
-__device__ __forceinline__ void nib_pairs4(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t w8 = w >> 8;
-  p[0] = h2_sub((w & 0x000F000Fu) | kMagic1024x2, kMagic1024x2);
-  p[1] = h2_fma((w & 0x00F000F0u) | kMagic1024x2, kSixteenthX2, kMinus64X2);
-  p[2] = h2_sub((w8 & 0x000F000Fu) | kMagic1024x2, kMagic1024x2);
-  p[3] = h2_fma((w8 & 0x00F000F0u) | kMagic1024x2, kSixteenthX2, kMinus64X2);
-}
 
 // ---------------------------------------------------------------------------
 // nibble -> fp16 through the fp8 conversion: a byte b in 0..15 read as e4m3 is exactly
@@ -183,27 +154,12 @@ __device__ __forceinline__ void nib_pairs4(uint32_t w, uint32_t (&p)[4]) {
 // ---------------------------------------------------------------------------
 constexpr float kCvtUnscale = 512.0f;  // 2^9
 
-__device__ __forceinline__ uint32_t cvt_e4m3x2(uint32_t two_bytes) {
-  uint32_t d;
-  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
-      : "=r"(d)
-      : "r"(two_bytes));
-  return d;
-}
-
 // Both byte pairs of a word: lo = bytes (0, 1), hi = bytes (2, 3).
 __device__ __forceinline__ void cvt_e4m3x2x2(uint32_t four_bytes, uint32_t &lo, uint32_t &hi) {
   asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
       "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(four_bytes));
-}
-
-// K word (8 nibbles n0..n7 of one token, n_i = dim i): fp16 pairs
-// p0 = (n0, n2), p1 = (n4, n6), p2 = (n1, n3), p3 = (n5, n7), each scaled by 2^-9.
-__device__ __forceinline__ void nib_pairs_k(uint32_t w, uint32_t (&p)[4]) {
-  cvt_e4m3x2x2(w & 0x0F0F0F0Fu, p[0], p[1]);
-  cvt_e4m3x2x2((w >> 4) & 0x0F0F0F0Fu, p[2], p[3]);
 }
 
 // V word from a transposed ldmatrix (token t0's nibbles d0..d3 in bits 0-15, token t1's
@@ -214,18 +170,6 @@ __device__ __forceinline__ void nib_pairs_v(uint32_t x, uint32_t (&p)[4]) {
   cvt_e4m3x2x2(y & 0x0F0F0F0Fu, p[0], p[2]);
   cvt_e4m3x2x2((y >> 4) & 0x0F0F0F0Fu, p[1], p[3]);
 }
-
-// V word from a transposed ldmatrix through the exponent-bias OR (exact codes, unscaled):
-// p[k] = (t0 dim k, t1 dim k); nibbles 0 and 2 of each half sit in the low mantissa
-// bits, nibbles 1 and 3 are masked in place as 1024 + 16c and brought back by x/16 - 64.
-__device__ __forceinline__ void nib_pairs_v_or(uint32_t x, uint32_t (&p)[4]) {
-  uint32_t q[4];
-  nib_pairs4(x, q);  // q[i] = (nibble i, nibble i+4) = (t0 dim i, t1 dim i)
-  p[0] = q[0]; p[1] = q[1]; p[2] = q[2]; p[3] = q[3];
-}
-
-// K word through the exponent-bias OR (exact codes, unscaled): p[i] = (n_i, n_{i+4}).
-__device__ __forceinline__ void nib_pairs_k_or(uint32_t w, uint32_t (&p)[4]) { nib_pairs4(w, p); }
 
 // ---------------------------------------------------------------------------
 // packed fp32 pairs (sm_100 f32x2 FMA pipe operations)
@@ -278,14 +222,6 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 // fp16 round-to-nearest-even with saturation to +-65504.
 __device__ __forceinline__ __half f16_sat(float x) {
   return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
-}
-
-// atom.add with acquire-release semantics at GPU scope; returns the old value.
-__device__ __forceinline__ int atomic_add_acq_rel_gpu(int32_t *p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
-               : "memory");
-  return old;
 }
 
 __device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {
