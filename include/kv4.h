@@ -83,7 +83,8 @@ typedef enum {
 #define KV4_DEVERR_PAGE_ID 1u    /* page-table entry outside [0, num_pages) */
 #define KV4_DEVERR_SEQ_LEN 2u    /* seq_len < 0, > max_pages*16, or fewer tokens than appended */
 #define KV4_DEVERR_SIDE_IDX 4u   /* sink_idx / ring_idx outside the side store */
-#define KV4_DEVERR_Q_RANGE 8u    /* a query element overflows fp16 (|q| > 65504) */
+#define KV4_DEVERR_Q_RANGE 8u    /* reserved: no longer raised (queries enter the dot
+                                    products in per-query fixed point, any finite value) */
 #define KV4_DEVERR_WORKSPACE 16u /* the batch needs more work items than the workspace holds */
 #define KV4_DEVERR_TIMEOUT 32u   /* a bounded wait for an async copy gave up */
 
@@ -97,7 +98,10 @@ typedef struct {
   int32_t group_size;   /* must be 32 */
   int32_t num_sinks;    /* S >= 0 */
   int32_t num_recent;   /* R >= 0, S + R <= 144 */
-  int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region; 0 = default (32) */
+  int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region, 1..32; 0 = chosen
+                           per call from num_seqs and max_seq_len: 32 for large batches, down
+                           to 8 when 32-page chunks would leave the GPU's warps idle (and 32
+                           whenever the workspace passed is too small for the finer split) */
 } kv4_config;
 
 typedef struct {
@@ -172,7 +176,9 @@ kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
  * value sum) that an exact log-sum-exp merge combines in a fixed order, so results
  * are deterministic.
  *
- *   q:       bf16 [num_seqs][Hq][128]; |q| must be <= 65504 (fp16 range).
+ *   q:       bf16 [num_seqs][Hq][128], finite. Each query enters the dot products as
+ *            15-bit fixed point with a power-of-two step set by its largest element
+ *            (relative rounding at most 2^-15 of that element).
  *   out:     bf16 [num_seqs][Hq][128].
  *   out_f32: optional fp32 [num_seqs][Hq][128] (NULL to skip).
  *   lse:     optional fp32 [num_seqs][Hq], natural log of the softmax denominator

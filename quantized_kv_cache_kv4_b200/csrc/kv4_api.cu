@@ -2,13 +2,15 @@
 // carve-up, and kernel launches on the caller's stream. No allocation, no sync.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "../../include/kv4.h"
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 
 namespace {
 
-constexpr int kDefaultChunkPages = 32;
+constexpr int kDefaultChunkPages = 32;  // automatic choice when the workspace is small
 
 kv4_status check_config(const kv4_config *cfg) {
   if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
@@ -26,8 +28,27 @@ kv4_status check_config(const kv4_config *cfg) {
   return KV4_OK;
 }
 
-int chunk_of(const kv4_config *cfg) {
-  return cfg->chunk_pages > 0 ? cfg->chunk_pages : kDefaultChunkPages;
+// Automatic chunk length (chunk_pages == 0): the longest chunk in kAutoChunks that still
+// gives the persistent attention grid about one entry per resident warp (148 SMs x 3
+// CTAs x 4 warps) for num_seqs sequences of max_seq_len tokens. Long batches get 32-page
+// chunks (fewest partial states to merge); small batches are split finer so every warp
+// has work.
+constexpr int kAutoChunks[] = {32, 24, 16, 12, 8};
+constexpr long long kAutoTargetEntries = 148LL * 3 * 4;
+
+int chunk_of(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
+  if (cfg->chunk_pages > 0) return cfg->chunk_pages;
+  const int H = cfg->num_kv_heads;
+  const int hpw = kv4::heads_per_warp_for(cfg->num_q_heads / H);
+  const long long nslots = (H + hpw - 1) / hpw;
+  const int protect = cfg->num_sinks + cfg->num_recent;
+  const long long int4_pages = (std::max(0, max_seq_len - protect) + kv4::kPage - 1) / kv4::kPage + 1;
+  const long long prot_entries = protect > 0 ? nslots : 0;
+  for (int C : kAutoChunks) {
+    const long long entries = num_seqs * (nslots * ((int4_pages + C - 1) / C) + prot_entries);
+    if (entries >= kAutoTargetEntries) return C;
+  }
+  return kAutoChunks[sizeof(kAutoChunks) / sizeof(kAutoChunks[0]) - 1];
 }
 
 bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
@@ -100,8 +121,8 @@ extern "C" {
 size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
   if (check_config(cfg) != KV4_OK || num_seqs < 0 || max_seq_len < 0) return 0;
   return kv4::workspace_bytes(num_seqs, max_seq_len, cfg->num_kv_heads,
-                              cfg->num_q_heads / cfg->num_kv_heads, chunk_of(cfg), nullptr,
-                              nullptr);
+                              cfg->num_q_heads / cfg->num_kv_heads,
+                              chunk_of(cfg, num_seqs, max_seq_len), nullptr, nullptr);
 }
 
 kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
@@ -135,8 +156,15 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return KV4_ERR_INVALID_ARG;
   kv4::Workspace w;
-  const size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads,
-                                           v.gqa, chunk_of(cfg), &w, workspace);
+  size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
+                                     chunk_of(cfg, batch->num_seqs, batch->max_seq_len), &w,
+                                     workspace);
+  // A workspace sized for a larger batch or longer sequences (where the automatic choice
+  // is 32 pages) may be too small for a finer automatic split of this one: fall back to
+  // 32-page chunks, for which it is large enough.
+  if (ws_bytes < need && cfg->chunk_pages == 0)
+    need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
+                                kDefaultChunkPages, &w, workspace);
   if (ws_bytes < need) return KV4_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);

@@ -5,8 +5,8 @@
 //
 // Kernels:
 //   plan_kernel  turns seq_lens into a work list. Region 0 of a sequence is its INT8
-//                protected set (one entry per kv head); regions 1.. are chunks of
-//                `chunk_pages` INT4 pages (one entry per one or two kv heads). Entries
+//                protected set; regions 1.. are chunks of `chunk_pages` INT4 pages; one
+//                entry per region and one or two kv heads. Entries
 //                come in four classes (full chunks, long partial chunks, protected sets,
 //                short chunks) so that the longest work starts first.
 //   attn_kernel  persistent; every warp repeatedly takes one entry from an atomic counter
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     sp.n[0] = sp.g.has_prot + sp.g.n_chunks;
     sp.n[1] = sp.nfull * nslots;
     sp.n[2] = has_last && sp.last_long ? nslots : 0;
-    sp.n[3] = sp.g.has_prot * H;
+    sp.n[3] = sp.g.has_prot * nslots;
     sp.n[4] = has_last && !sp.last_long ? nslots : 0;
     return sp;
   };
@@ -211,7 +211,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     const Regions &g = sp.g;
     int ef = off[1], el = off[2], epr = off[3], es = off[4];
     if (g.has_prot)
-      for (int h = 0; h < H; ++h) w.entries[epr++] = make_int4(b, 0, h, 1);
+      for (int s = 0; s < nslots; ++s)
+        w.entries[epr++] = make_int4(b, 0, s * hpw, min(hpw, H - s * hpw));
     for (int ch = 0; ch < sp.nfull; ++ch)
       for (int s = 0; s < nslots; ++s)
         w.entries[ef++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
@@ -292,15 +293,17 @@ __device__ __forceinline__ uint4 load_q8(const uint16_t *qrow, int dim0, bool li
   return *reinterpret_cast<const uint4 *>(qrow + dim0);
 }
 
-// bf16 pair -> fp16 pair (exact for |q| in fp16's normal range); returns the sum of the
-// two fp16 values and flags magnitudes beyond fp16.
-__device__ __forceinline__ float q_to_f16_pair(uint32_t bf2, uint32_t &out, bool &bad) {
-  const float lo = __uint_as_float(bf2 << 16);
-  const float hi = __uint_as_float(bf2 & 0xFFFF0000u);
-  bad |= fabsf(lo) > 65504.0f || fabsf(hi) > 65504.0f;
-  out = pack_h2(lo, hi);
-  const float2 back = h2_to_f2(out);
-  return back.x + back.y;
+// Fixed-point step of a query: 2^e with max|q| < 2^(e+14), so every |q / 2^e| <= 2^14
+// (15 bits with the sign). amax is the lane's max|q|; the 4 lanes of a column combine.
+__device__ __forceinline__ float query_step(float amax) {
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  int ex = 0;
+  if (amax > 0.f) {
+    frexpf(amax, &ex);  // amax < 2^ex
+    ex -= 14;
+  }
+  return ldexpf(1.0f, ex);
 }
 
 // ------------------------- INT8 protected set ----------------------------
@@ -351,21 +354,48 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   const int npre = min(nt, kStages);
   for (int k = 0; k < npre; ++k) issue(k);
 
-  // query fragments for int8 strips: k-tile c: b01 = (q[16c+4tig], q[..+1]),
-  // b23 = (q[16c+4tig+2], q[..+3])
-  uint32_t qb[8][2];
-  bool qbad = false;
+  // query fragments (B operand of QK^T, m16n8k32): lane column gid = query gid; k-step
+  // ks: b0 = dims 32ks+4tig..+3, b1 = dims 32ks+16+4tig..+3, as bytes of
+  // q / qstep = 256*hi + lo
+  uint32_t qh[4][2], ql[4][2];
+  float2 kq;  // qstep * log2(e)/sqrt(d) of the C-fragment columns (2tig, 2tig+1)
   {
     const bool live = gid < G;
     const uint16_t *qrow = q + (static_cast<size_t>(b) * H * G + h * G + gid) * kHeadDim;
+    float qv[4][2][4];
+    float amax = 0.f;
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
-      uint2 v = live ? *reinterpret_cast<const uint2 *>(qrow + 16 * cc + 4 * tig) : make_uint2(0, 0);
-      q_to_f16_pair(v.x, qb[cc][0], qbad);
-      q_to_f16_pair(v.y, qb[cc][1], qbad);
-    }
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint2 v = live ? *reinterpret_cast<const uint2 *>(qrow + 32 * ks + 16 * hf + 4 * tig)
+                             : make_uint2(0u, 0u);
+        qv[ks][hf][0] = __uint_as_float(v.x << 16);
+        qv[ks][hf][1] = __uint_as_float(v.x & 0xFFFF0000u);
+        qv[ks][hf][2] = __uint_as_float(v.y << 16);
+        qv[ks][hf][3] = __uint_as_float(v.y & 0xFFFF0000u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(qv[ks][hf][i]));
+      }
+    const float qstep = query_step(amax);
+    const float inv = 1.0f / qstep;  // a power of two: exact
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t hb = 0u, lb = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int qi = __float2int_rn(qv[ks][hf][i] * inv);
+          lb |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * i);
+          hb |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * i);
+        }
+        qh[ks][hf] = hb;
+        ql[ks][hf] = lb;
+      }
+    kq.x = __shfl_sync(0xffffffffu, qstep, 4 * (2 * tig)) * kScaleLog2;
+    kq.y = __shfl_sync(0xffffffffu, qstep, 4 * (2 * tig + 1)) * kScaleLog2;
   }
-  if (qbad) set_err(err, KV4_DEVERR_Q_RANGE);
 
   float m[2] = {kNegBig, kNegBig}, l[2] = {0.f, 0.f};
   float o[8][4];
@@ -384,18 +414,13 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
     uint8_t *sp = x.stage0 + st * kStageBytes;
     const uint32_t sa = smem_u32(sp);
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int32_t ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int pr = 0; pr < 4; ++pr) {
-      uint32_t kw[4];
-      ldsm_x4(kw, sa + pr * 512 + ld_off);
-#pragma unroll
-      for (int hs = 0; hs < 2; ++hs) {
-        const int cc = 2 * pr + hs;
-        const uint32_t ulo = kw[2 * hs] ^ 0x80808080u, uhi = kw[2 * hs + 1] ^ 0x80808080u;
-        mma_f16(acc, s8_pair<0x4140>(ulo), s8_pair<0x4140>(uhi), s8_pair<0x4342>(ulo),
-                s8_pair<0x4342>(uhi), qb[cc][0], qb[cc][1]);
-      }
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t kw[4];  // rows = positions, k = dims 32ks..32ks+31
+      ldsm_x4(kw, sa + ks * 512 + ld_off);
+      mma_s8s8(ah, kw[0], kw[1], kw[2], kw[3], qh[ks][0], qh[ks][1]);
+      mma_s8u8(al, kw[0], kw[1], kw[2], kw[3], ql[ks][0], ql[ks][1]);
     }
     const uint16_t *ks = reinterpret_cast<const uint16_t *>(sp + kOffKs8);
     const uint16_t *vs = reinterpret_cast<const uint16_t *>(sp + kOffVs8);
@@ -413,9 +438,11 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
         valid = rs < R && ring_base + d >= S;
       }
       const float sk = __half2float(__ushort_as_half(ks[slot]));
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-        s[hf][e] = valid ? sk * acc[2 * hf + e] * (kLog2e * 0.08838834764831845f) : -CUDART_INF_F;
+      // exact integer dot products: |.| < 2^29
+      const float d0 = static_cast<float>(ah[2 * hf] * 256 + al[2 * hf]);
+      const float d1 = static_cast<float>(ah[2 * hf + 1] * 256 + al[2 * hf + 1]);
+      s[hf][0] = valid ? d0 * sk * kq.x : -CUDART_INF_F;
+      s[hf][1] = valid ? d1 * sk * kq.y : -CUDART_INF_F;
     }
     float alpha[2];
     softmax_step(s, m, l, alpha);
@@ -478,6 +505,282 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   }
 }
 
+
+// ------------------- INT8 protected set, two kv heads per warp -------------------
+// The protected sets of kv heads h0 and h0+1 (G <= 4) in the column layout of the INT4
+// pair path: MMA N columns 0-3 are head slot 0's queries, 4-7 slot 1's. A tile of 16
+// positions takes two ring stages: first the K codes and scales of both heads, then their
+// V codes and scales, so the K stage is refilled as soon as the logits are taken.
+// QK^T on the integer tensor cores: int8 K codes times the query in 15-bit fixed point
+// (signed high byte, unsigned low byte), exact int32 dot products; the per-token K scale
+// and the query step are applied to the sums in fp32. PV as in the one-head path.
+constexpr int kOffScale8P = 2 * kInt8CodeBytes;                       // scales of slot hs at +32 hs
+constexpr int kInt8PairBytes = 2 * kInt8CodeBytes + 2 * kInt8ScaleBytes;  // 4160 per stage
+
+__device__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Workspace &w,
+                                       const uint16_t *__restrict__ q, int b, int h0, int nh,
+                                       int L, int r, int32_t *err) {
+  constexpr int CPH = 4;  // MMA columns per kv head slot
+  const int G = c.gqa, H = c.num_kv_heads;
+  const int lane = x.lane, gid = x.gid, tig = x.tig;
+  const int S = c.num_sinks, R = c.num_recent;
+  const int n_sink = min(S, L);
+  const int rec_lo = max(S, L - R);
+  const int sink_tiles = (n_sink + kPage - 1) / kPage;
+  const int ring_tiles = rec_lo < L ? (R + kPage - 1) / kPage : 0;
+  const int nt = sink_tiles + ring_tiles;
+  const int nv = 2 * nt;  // copies: the K part, then the V part, of every tile
+  // this lane's C-fragment columns 2tig, 2tig+1: head slot and query index
+  const int hs_c = (2 * tig) / CPH;
+  const int jc0 = (2 * tig) % CPH;
+  const bool head_c_live = hs_c < nh;
+
+  const int set = sink_tiles ? (c.sink_idx ? c.sink_idx[b] : b) : 0;
+  const int ring = ring_tiles ? (c.ring_idx ? c.ring_idx[b] : b) : 0;
+  if ((sink_tiles && (set < 0 || set >= c.num_sink_sets)) ||
+      (ring_tiles && (ring < 0 || ring >= c.num_rings))) {
+    if (lane == 0) set_err(err, KV4_DEVERR_SIDE_IDX);
+    for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+    return;
+  }
+
+  // copy k: tile k/2, K part (k even) or V part (k odd), both heads; a spare slot (one
+  // head left) gets a copy of head h0
+  auto issue = [&](int k) {
+    if (lane == 0) {
+      const int st = k % kStages;
+      uint8_t *dst = x.stage0 + st * kStageBytes;
+      const int tile = k >> 1;
+      const bool vpart = (k & 1) != 0;
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&x.bars[st], kInt8PairBytes);
+      for (int hs = 0; hs < 2; ++hs) {
+        const int h = h0 + (hs < nh ? hs : 0);
+        const int8_t *codes;
+        const uint16_t *scales;
+        if (tile < sink_tiles) {
+          const size_t t = (static_cast<size_t>(set) * H + h) * c.sink_tiles + tile;
+          codes = (vpart ? c.sink_v : c.sink_k) + t * kInt8CodeBytes;
+          scales = (vpart ? c.sink_vs : c.sink_ks) + t * kPage;
+        } else {
+          const size_t t =
+              (static_cast<size_t>(ring) * H + h) * c.ring_tiles + (tile - sink_tiles);
+          codes = (vpart ? c.ring_v : c.ring_k) + t * kInt8CodeBytes;
+          scales = (vpart ? c.ring_vs : c.ring_ks) + t * kPage;
+        }
+        bulk_g2s(dst + hs * kInt8CodeBytes, codes, kInt8CodeBytes, &x.bars[st]);
+        bulk_g2s(dst + kOffScale8P + hs * kInt8ScaleBytes, scales, kInt8ScaleBytes, &x.bars[st]);
+      }
+    }
+  };
+  int issued = min(nv, kStages);
+  for (int k = 0; k < issued; ++k) issue(k);
+  // A bounded wait gave up on copy k: wait for the later copies in flight, write empty
+  // states.
+  auto give_up = [&](int k) {
+    for (int kk = k + 1; kk < issued; ++kk) wait_stage(x, kk % kStages, err);
+    for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+  };
+
+  // ---- query fragments (B operand of QK^T, m16n8k32): lane column gid = (slot gid/4,
+  // query gid%4); k-step ks: b0 = dims 32ks+4tig..+3, b1 = dims 32ks+16+4tig..+3, as bytes
+  // of q / qstep = 256*hi + lo; a slot's fragments are zero outside its columns.
+  uint32_t qh[2][4][2], ql[2][4][2];
+  float qstep_own;
+  {
+    const int hs_b = gid / CPH, jb = gid % CPH;
+    const bool live = jb < G && hs_b < nh;
+    const uint16_t *qrow =
+        q + (static_cast<size_t>(b) * H * G + (h0 + hs_b) * G + jb) * kHeadDim;
+    float qv[4][2][4];
+    float amax = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint2 v = live ? *reinterpret_cast<const uint2 *>(qrow + 32 * ks + 16 * hf + 4 * tig)
+                             : make_uint2(0u, 0u);
+        qv[ks][hf][0] = __uint_as_float(v.x << 16);
+        qv[ks][hf][1] = __uint_as_float(v.x & 0xFFFF0000u);
+        qv[ks][hf][2] = __uint_as_float(v.y << 16);
+        qv[ks][hf][3] = __uint_as_float(v.y & 0xFFFF0000u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(qv[ks][hf][i]));
+      }
+    qstep_own = query_step(amax);
+    const float inv = 1.0f / qstep_own;  // a power of two: exact
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t hb = 0u, lb = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int qi = __float2int_rn(qv[ks][hf][i] * inv);
+          lb |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * i);
+          hb |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * i);
+        }
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+          qh[hs][ks][hf] = hs == hs_b ? hb : 0u;
+          ql[hs][ks][hf] = hs == hs_b ? lb : 0u;
+        }
+      }
+  }
+  float2 kq;  // qstep * log2(e)/sqrt(d) of the C-fragment columns (2tig, 2tig+1)
+  kq.x = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig)) * kScaleLog2;
+  kq.y = __shfl_sync(0xffffffffu, qstep_own, 4 * (2 * tig + 1)) * kScaleLog2;
+
+  float m[2] = {kNegBig, kNegBig}, l[2] = {0.f, 0.f};
+  float o[8][4];
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) o[cc][0] = o[cc][1] = o[cc][2] = o[cc][3] = 0.f;
+  const int ld_off = ((lane >> 4) * 256) + ((lane >> 3) & 1) * 128 + (lane & 7) * 16;
+  const int ring_base = L - R;  // ring slot s holds position ring_base + ((s - ring_base) mod R)
+  const bool write_p0 = head_c_live && jc0 < G, write_p1 = head_c_live && jc0 + 1 < G;
+  const bool col_live = (gid % CPH) < G && (gid / CPH) < nh;  // this lane's B column
+
+  for (int j = 0; j < nt; ++j) {
+    // ---- K part: logits ----
+    const int kk = 2 * j;
+    if (!wait_stage(x, kk % kStages, err)) {
+      give_up(kk);
+      return;
+    }
+    const uint8_t *spk = x.stage0 + (kk % kStages) * kStageBytes;
+    const uint32_t sak = smem_u32(spk);
+    int32_t ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        uint32_t kw[4];  // rows = positions, k = dims 32ks..32ks+31
+        ldsm_x4(kw, sak + hs * kInt8CodeBytes + ks * 512 + ld_off);
+        mma_s8s8(ah, kw[0], kw[1], kw[2], kw[3], qh[hs][ks][0], qh[hs][ks][1]);
+        mma_s8u8(al, kw[0], kw[1], kw[2], kw[3], ql[hs][ks][0], ql[hs][ks][1]);
+      }
+    const uint16_t *ksc =
+        reinterpret_cast<const uint16_t *>(spk + kOffScale8P + hs_c * kInt8ScaleBytes);
+    const float sk[2] = {__half2float(__ushort_as_half(ksc[gid])),
+                         __half2float(__ushort_as_half(ksc[gid + 8]))};
+    __syncwarp();
+    if (issued < nv) issue(issued++);  // the K stage is free again
+
+    float s[2][2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int slot = gid + 8 * hf;
+      bool valid;
+      if (j < sink_tiles) {
+        valid = j * kPage + slot < n_sink;
+      } else {
+        const int rs = (j - sink_tiles) * kPage + slot;
+        int d = (rs - ring_base) % R;
+        if (d < 0) d += R;
+        valid = rs < R && ring_base + d >= S;
+      }
+      // exact integer dot products: |.| < 2^29
+      const float d0 = static_cast<float>(ah[2 * hf] * 256 + al[2 * hf]);
+      const float d1 = static_cast<float>(ah[2 * hf + 1] * 256 + al[2 * hf + 1]);
+      s[hf][0] = valid ? d0 * sk[hf] * kq.x : -CUDART_INF_F;
+      s[hf][1] = valid ? d1 * sk[hf] * kq.y : -CUDART_INF_F;
+    }
+    // ---- online softmax; the rescale is skipped while no running max moves ----
+    float a[2];
+    bool moved = false;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float t = fmaxf(s[0][e], s[1][e]);
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+      const float mn = fmaxf(m[e], t);
+      const bool mv = mn != m[e];
+      a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
+      moved |= mv;
+      m[e] = mn;
+      s[0][e] = fast_exp2(s[0][e] - mn);
+      s[1][e] = fast_exp2(s[1][e] - mn);
+      l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
+    }
+    if (__any_sync(0xffffffffu, moved)) {
+      const float2 a2 = make_float2(a[0], a[1]);
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const float2 u = fmul2(make_float2(o[cc][0], o[cc][1]), a2);
+        const float2 v = fmul2(make_float2(o[cc][2], o[cc][3]), a2);
+        o[cc][0] = u.x; o[cc][1] = u.y; o[cc][2] = v.x; o[cc][3] = v.y;
+      }
+    }
+
+    // ---- V part: P' = p * vscale (fp16), O^T += V^T P' per 16-dim strip and head ----
+    const int kvc = 2 * j + 1;
+    if (!wait_stage(x, kvc % kStages, err)) {
+      give_up(kvc);
+      return;
+    }
+    const uint8_t *spv = x.stage0 + (kvc % kStages) * kStageBytes;
+    const uint32_t sav = smem_u32(spv);
+    const uint16_t *vsc =
+        reinterpret_cast<const uint16_t *>(spv + kOffScale8P + hs_c * kInt8ScaleBytes);
+    const float sv0 = __half2float(__ushort_as_half(vsc[gid]));
+    const float sv1 = __half2float(__ushort_as_half(vsc[gid + 8]));
+    if (write_p0) {
+      x.ptile8[(2 * tig) * 16 + gid] = __half_as_ushort(__float2half_rn(s[0][0] * sv0));
+      x.ptile8[(2 * tig) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(s[1][0] * sv1));
+    }
+    if (write_p1) {
+      x.ptile8[(2 * tig + 1) * 16 + gid] = __half_as_ushort(__float2half_rn(s[0][1] * sv0));
+      x.ptile8[(2 * tig + 1) * 16 + gid + 8] = __half_as_ushort(__float2half_rn(s[1][1] * sv1));
+    }
+    __syncwarp();
+    uint32_t b01 = 0u, b23 = 0u;  // column gid's P' (k = positions 2tig.., 2tig+8..)
+    if (col_live) {
+      b01 = *reinterpret_cast<const uint32_t *>(&x.ptile8[gid * 16 + 2 * tig]);
+      b23 = *reinterpret_cast<const uint32_t *>(&x.ptile8[gid * 16 + 2 * tig + 8]);
+    }
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr)
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        uint32_t vw[4];
+        ldsm_x4_t(vw, sav + hs * kInt8CodeBytes + pr * 512 + ld_off);
+        const uint32_t c01 = gid / CPH == hs ? b01 : 0u, c23 = gid / CPH == hs ? b23 : 0u;
+#pragma unroll
+        for (int sp2 = 0; sp2 < 2; ++sp2) {
+          const int cc = 2 * pr + sp2;
+          const uint32_t ulo = vw[2 * sp2] ^ 0x80808080u, uhi = vw[2 * sp2 + 1] ^ 0x80808080u;
+          mma_f16(o[cc], s8_pair<0x4240>(ulo), s8_pair<0x4341>(ulo), s8_pair<0x4240>(uhi),
+                  s8_pair<0x4341>(uhi), c01, c23);
+        }
+      }
+    __syncwarp();
+    if (issued < nv) issue(issued++);  // the V stage is free again
+  }
+
+  // ---- finish: reduce the denominators over the 8 position lanes, write the partials ----
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], off);
+  if (head_c_live) {
+    float *rec = record_of(w, H, G, b, h0 + hs_c, r);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = jc0 + e;
+      if (j < G) {
+        float *rr = rec + j * kRecordFloats;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)  // rows: dim 16cc+2gid (c0/c1) and +1 (c2/c3)
+          *reinterpret_cast<float2 *>(rr + 16 * cc + 2 * gid) = make_float2(o[cc][e], o[cc][2 + e]);
+        if (gid == 0) {
+          rr[kHeadDim] = m[e] * kLn2;
+          rr[kHeadDim + 1] = l[e];
+        }
+      }
+    }
+  }
+}
 
 // ---------------------------- INT4 chunk --------------------------------
 // Token order of the QK^T M-tile rows: rows 0-7 are tokens 0-7, rows 8-11 tokens 12-15,
@@ -552,10 +855,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 
   // ---- query fragments (B operand of QK^T). Lane column gid = (slot gid/CPH, query
   // gid%CPH); slot hs's fragments are zero unless the column is in slot hs.
-  // group g, with the fp8-conversion unpack: k-tile 0 b01 = (q[32g+8tig], q[..+2]),
-  // b23 = (q[..+4], q[..+6]); k-tile 1 b01 = (q[..+1], q[..+3]), b23 = (q[..+5], q[..+7]).
-  // With the exponent-bias unpack the pairs are (0,4) (1,5) | (2,6) (3,7).
-  // Integer path: q = qstep * (256*hi + lo) with qstep = 2^e chosen per query so that
+  // q = qstep * (256*hi + lo) with qstep = 2^e chosen per query so that
   // |256*hi + lo| < 2^14; b0 holds dims 8tig+{0,2,4,6} and b1 dims 8tig+{1,3,5,7} of a
   // group (the low and high nibbles of the lane's K word), as bytes.
   uint32_t qh[HPW][4][2], ql[HPW][4][2];
@@ -937,9 +1237,12 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
     const int b = en.x, r = en.y, h0 = en.z, nh = en.w;
     const int L = c.seq_lens[b];
     const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages);
-    if (r < rg.has_prot)
-      process_protected(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
-    else
+    if (r < rg.has_prot) {
+      if constexpr (HPW == 2)
+        process_protected_pair(x, c, w, q, b, h0, nh, L, r, err);
+      else
+        process_protected(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
+    } else
       process_int4<HPW>(x, c, w, q, b, h0, nh, r, r - rg.has_prot, rg, err);
     if (x.dead) break;
   }

@@ -51,6 +51,9 @@ struct Outputs {
   float *lse;      // optional fp32 [B][Hq]
 };
 
+// kv heads one attention warp serves for a GQA ratio (2 when G <= 4).
+int heads_per_warp_for(int gqa);
+
 size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads,
                        int32_t gqa, int32_t chunk_pages, Workspace *carve, void *base);
 

@@ -127,9 +127,18 @@ def test_merge_argument_checks(kv4):
     assert lib.kv4_regional_merge(None, None, 2, 4, 128, None, None, None, None) == -1
 
 
+def test_automatic_chunk_splits_small_batches_finer(kv4):
+    auto, c32 = _cfg(kv4), _cfg(kv4, chunk_pages=32)
+    # a small batch gets a finer split (more partial states) than 32-page chunks ...
+    assert kv4.workspace_size(auto, 2, 1000) > kv4.workspace_size(c32, 2, 1000)
+    # ... a large one keeps 32-page chunks
+    assert kv4.workspace_size(auto, 1024, 14348) == kv4.workspace_size(c32, 1024, 14348)
+
+
 def test_workspace_too_small_is_reported(kv4):
     c = _cfg(kv4)
-    need = kv4.workspace_size(c, 2, 1000)
+    # too small even for 32-page chunks, the fallback of the automatic choice
+    need = kv4.workspace_size(_cfg(kv4, chunk_pages=32), 2, 1000)
     pool = kv4.Int4Pool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
     side = kv4.Int8Side(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1 << 20, 1 << 20, 1 << 20,
                         1 << 20, 2)
