@@ -214,6 +214,7 @@ def run_gpu(args, rank, world, local_rank):
     build.build()
     from quantized_kv_cache_kv4_b200 import kv4
     from quantized_kv_cache_kv4_b200.session import DecodeSession
+    from quantized_kv_cache_kv4_b200.host_io import HostStepPipeline
     from quantized_kv_cache_kv4_b200.workload import make_workload
 
     torch.cuda.set_device(local_rank)
@@ -285,26 +286,13 @@ def run_gpu(args, rank, world, local_rank):
     hq = sess.q.cpu().pin_memory()
     hl = sess.step_lens.cpu().pin_memory()
     hout = torch.empty((K, B, Hq, D), dtype=torch.bfloat16).pin_memory()
-    dk = torch.empty_like(sess.step_k[0])
-    dv = torch.empty_like(sess.step_v[0])
-    dq = torch.empty_like(sess.q[0])
-    dl = torch.empty_like(sess.step_lens[0])
-    dout = torch.empty_like(sess.out)
-    h2d = (dk.numel() + dv.numel() + dq.numel()) * 2 + dl.numel() * 4
-    d2h = dout.numel() * 2
+    pipe = HostStepPipeline(sess)
+    h2d, d2h = pipe.bytes_per_step()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for i, s in enumerate(range(W, W + K)):
-        dk.copy_(hk[s], non_blocking=True)
-        dv.copy_(hv[s], non_blocking=True)
-        dq.copy_(hq[s], non_blocking=True)
-        dl.copy_(hl[s], non_blocking=True)
-        b = sess.batch(dl)
-        kv4.quantize_append(sess.cache, b, dk, dv, None, sess.err)
-        kv4.decode_attention(sess.cache, b, dq, dout, sess.workspace, err=sess.err)
-        hout[i].copy_(dout, non_blocking=True)
+    pipe.run(hk, hv, hq, hl, hout, range(W, W + K), start_event=e0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()

@@ -186,6 +186,34 @@ def test_several_decode_steps_demote_and_stay_exact():
     check_cache(sess, range(3))
 
 
+def test_host_pipeline_matches_serial_steps():
+    """Double-buffered host<->device steps give the outputs of plain serial steps."""
+    _, session, W = _mods()
+    from quantized_kv_cache_kv4_b200.host_io import HostStepPipeline
+    wl = W.custom_workload([37, 150, 161, 600], num_sinks=4, num_recent=32, seed=5)
+    n = 5
+    ref = session.DecodeSession(wl, steps=n)
+    want = []
+    for s in range(n):
+        ref.step(s)
+        want.append(ref.out.clone())
+    torch.cuda.synchronize()
+    ref.check_err()
+
+    sess = session.DecodeSession(wl, steps=n)
+    hk, hv = sess.step_k.cpu().pin_memory(), sess.step_v.cpu().pin_memory()
+    hq, hl = sess.q.cpu().pin_memory(), sess.step_lens.cpu().pin_memory()
+    hout = torch.empty((n,) + tuple(sess.out.shape), dtype=torch.bfloat16).pin_memory()
+    pipe = HostStepPipeline(sess)
+    pipe.run(hk, hv, hq, hl, hout, range(n))
+    torch.cuda.synchronize()
+    sess.check_err()
+    for s in range(n):
+        assert torch.equal(hout[s], want[s].cpu()), s
+    h2d, d2h = pipe.bytes_per_step()
+    assert d2h == sess.out.numel() * 2 and h2d > d2h
+
+
 def test_empty_sequence_and_determinism():
     kv4, _, W = _mods()
     wl = W.custom_workload([50, 300], seed=11)
