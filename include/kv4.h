@@ -98,9 +98,9 @@ typedef struct {
   int32_t group_size;   /* must be 32 */
   int32_t num_sinks;    /* S >= 0 */
   int32_t num_recent;   /* R >= 0, S + R <= 144 */
-  int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region, 1..32; 0 = chosen
-                           per call from num_seqs and max_seq_len: 32 for large batches, down
-                           to 8 when 32-page chunks would leave the GPU's warps idle (and 32
+  int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region, 1..64; 0 = chosen
+                           per call from num_seqs and max_seq_len: 64 for large batches, down
+                           to 8 when long chunks would leave the GPU's warps idle (and 64
                            whenever the workspace passed is too small for the finer split) */
 } kv4_config;
 

@@ -10,8 +10,6 @@
 
 namespace {
 
-constexpr int kDefaultChunkPages = 32;  // automatic choice when the workspace is small
-
 kv4_status check_config(const kv4_config *cfg) {
   if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
   if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_sinks < 0 ||
@@ -23,17 +21,17 @@ kv4_status check_config(const kv4_config *cfg) {
   if (cfg->num_q_heads % cfg->num_kv_heads != 0 ||
       cfg->num_q_heads / cfg->num_kv_heads > kv4::kMaxGqa)
     return KV4_ERR_UNSUPPORTED_SHAPE;
-  if (cfg->chunk_pages > 32) return KV4_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->chunk_pages > kv4::kMaxChunkPages) return KV4_ERR_UNSUPPORTED_SHAPE;
   if (cfg->num_sinks + cfg->num_recent > KV4_MAX_PROTECTED) return KV4_ERR_PROTECTED_TOO_LARGE;
   return KV4_OK;
 }
 
 // Automatic chunk length (chunk_pages == 0): the longest chunk in kAutoChunks that still
 // gives the persistent attention grid about one entry per resident warp (148 SMs x 3
-// CTAs x 4 warps) for num_seqs sequences of max_seq_len tokens. Long batches get 32-page
+// CTAs x 4 warps) for num_seqs sequences of max_seq_len tokens. Large batches get 64-page
 // chunks (fewest partial states to merge); small batches are split finer so every warp
 // has work.
-constexpr int kAutoChunks[] = {32, 24, 16, 12, 8};
+constexpr int kAutoChunks[] = {64, 48, 32, 24, 16, 12, 8};
 constexpr long long kAutoTargetEntries = 148LL * 3 * 4;
 
 int chunk_of(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
@@ -159,12 +157,13 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
                                      chunk_of(cfg, batch->num_seqs, batch->max_seq_len), &w,
                                      workspace);
-  // A workspace sized for a larger batch or longer sequences (where the automatic choice
-  // is 32 pages) may be too small for a finer automatic split of this one: fall back to
-  // 32-page chunks, for which it is large enough.
+  // A workspace sized for a larger batch or longer sequences (and so for longer automatic
+  // chunks) may be too small for a finer automatic split of this one: fall back to the
+  // longest chunks, for which any workspace sized with this config at larger or equal
+  // (num_seqs, max_seq_len) is large enough.
   if (ws_bytes < need && cfg->chunk_pages == 0)
     need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
-                                kDefaultChunkPages, &w, workspace);
+                                kv4::kMaxChunkPages, &w, workspace);
   if (ws_bytes < need) return KV4_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);

@@ -806,9 +806,14 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   const int jc0 = (2 * tig) % CPH;
   const bool head_c_live = hs_c < nh;
 
-  int pid = 0;
-  if (lane < np) pid = c.page_table[static_cast<size_t>(b) * c.max_pages + p0 + lane];
-  const bool bad = lane < np && (pid < 0 || pid >= c.num_pages);
+  // page ids of the chunk: page k in lane k (k < 32) or in the second register of lane
+  // k - 32 (chunks of up to 64 pages)
+  const int *pt = c.page_table + static_cast<size_t>(b) * c.max_pages + p0;
+  int pid = 0, pid2 = 0;
+  if (lane < np) pid = pt[lane];
+  if (lane + 32 < np) pid2 = pt[lane + 32];
+  const bool bad = (lane < np && (pid < 0 || pid >= c.num_pages)) ||
+                   (lane + 32 < np && (pid2 < 0 || pid2 >= c.num_pages));
   if (__any_sync(0xffffffffu, bad)) {
     if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
     for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
@@ -820,7 +825,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   constexpr int kOffKp = 2 * HPW * kInt4CodeBytes;
   constexpr int kOffVp = kOffKp + HPW * kInt4ParamBytes;
   auto issue = [&](int k) {
-    const int pk = __shfl_sync(0xffffffffu, pid, k);
+    const int pk = __shfl_sync(0xffffffffu, k < 32 ? pid : pid2, k & 31);
     if (lane == 0) {
       const int st = k % kStages;
       uint8_t *dst = x.stage0 + st * kStageBytes;

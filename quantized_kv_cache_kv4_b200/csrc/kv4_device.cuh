@@ -14,6 +14,7 @@ namespace kv4 {
 constexpr int kHeadDim = 128;
 constexpr int kPage = 16;       // tokens per INT4 page and per INT8 tile
 constexpr int kGroup = 32;      // INT4 group length along head_dim
+constexpr int kMaxChunkPages = 64;  // INT4 pages per work entry (page ids in two registers)
 constexpr int kMaxGqa = 8;      // query heads per kv head handled by one warp (MMA N = 8)
 constexpr int kRecordFloats = kHeadDim + 4;  // partial record: acc[128], m, l, pad, pad
 

@@ -58,7 +58,7 @@ def _cfg(kv4, **kw):
 
 
 def test_workspace_size_host_only(kv4):
-    c = _cfg(kv4)
+    c = _cfg(kv4, chunk_pages=32)
     n1 = kv4.workspace_size(c, 64, 2048)
     n2 = kv4.workspace_size(c, 128, 2048)
     assert 0 < n1 < n2
@@ -74,7 +74,7 @@ def test_workspace_size_host_only(kv4):
     (dict(num_sinks=145, num_recent=0), -3),
     (dict(num_q_heads=30), -2),
     (dict(num_q_heads=128, num_kv_heads=8), -2),
-    (dict(chunk_pages=33), -2),
+    (dict(chunk_pages=65), -2),
     (dict(num_sinks=-1), -1),
 ])
 def test_config_rejected_before_launch(kv4, kw, status):
@@ -128,17 +128,17 @@ def test_merge_argument_checks(kv4):
 
 
 def test_automatic_chunk_splits_small_batches_finer(kv4):
-    auto, c32 = _cfg(kv4), _cfg(kv4, chunk_pages=32)
-    # a small batch gets a finer split (more partial states) than 32-page chunks ...
-    assert kv4.workspace_size(auto, 2, 1000) > kv4.workspace_size(c32, 2, 1000)
-    # ... a large one keeps 32-page chunks
-    assert kv4.workspace_size(auto, 1024, 14348) == kv4.workspace_size(c32, 1024, 14348)
+    auto, c64 = _cfg(kv4), _cfg(kv4, chunk_pages=64)
+    # a small batch gets a finer split (more partial states) than 64-page chunks ...
+    assert kv4.workspace_size(auto, 2, 1000) > kv4.workspace_size(c64, 2, 1000)
+    # ... a large one gets 64-page chunks
+    assert kv4.workspace_size(auto, 1024, 14348) == kv4.workspace_size(c64, 1024, 14348)
 
 
 def test_workspace_too_small_is_reported(kv4):
     c = _cfg(kv4)
-    # too small even for 32-page chunks, the fallback of the automatic choice
-    need = kv4.workspace_size(_cfg(kv4, chunk_pages=32), 2, 1000)
+    # too small even for 64-page chunks, the fallback of the automatic choice
+    need = kv4.workspace_size(_cfg(kv4, chunk_pages=64), 2, 1000)
     pool = kv4.Int4Pool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
     side = kv4.Int8Side(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1 << 20, 1 << 20, 1 << 20,
                         1 << 20, 2)

@@ -137,6 +137,8 @@ EDGE = [
     ("chunk1", [700, 40, 260], 8, 2, 16, 128, 1),
     ("chunk3", [700, 40, 260], 8, 2, 16, 128, 3),
     ("odd-S-R", [23, 64, 511], 8, 2, 7, 13, 2),
+    ("chunk64", [2100, 1030, 40, 1500], 8, 2, 16, 128, 64),
+    ("chunk48-three-kv-heads", [1800, 777, 150], 12, 3, 4, 32, 48),
 ]
 
 
