@@ -198,6 +198,30 @@ def run_reference(args, rank, world):
 # GPU arm
 # ----------------------------------------------------------------------------
 
+def rank_workload(name, rank):
+    """The workload of one rank: the named shape with its own data seed, so that N ranks
+    run N independent replica batches (weak scaling, no exchange)."""
+    from quantized_kv_cache_kv4_b200.workload import make_workload
+    wl = make_workload(name)
+    wl.seed = wl.seed + 7919 * rank
+    return wl
+
+
+def combine_ranks(ms, units, world, device):
+    """(max over ranks of a timed region in ms, sum over ranks of the units processed).
+    Every rank calls this the same number of times, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms), float(units)], dtype=torch.float64, device=device)
+    if world > 1:
+        tmax = t[:1].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        usum = t[1:].clone()
+        dist.all_reduce(usum, op=dist.ReduceOp.SUM)
+        return float(tmax.item()), float(usum.item())
+    return float(t[0].item()), float(t[1].item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -215,7 +239,6 @@ def run_gpu(args, rank, world, local_rank):
     from quantized_kv_cache_kv4_b200 import kv4
     from quantized_kv_cache_kv4_b200.session import DecodeSession
     from quantized_kv_cache_kv4_b200.host_io import HostStepPipeline
-    from quantized_kv_cache_kv4_b200.workload import make_workload
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -224,8 +247,7 @@ def run_gpu(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    wl = make_workload(args.workload)
-    wl.seed = wl.seed + 7919 * rank  # each rank: its own replica batch (same shape)
+    wl = rank_workload(args.workload, rank)
     W, K = args.warmup, args.steps
     sess = DecodeSession(wl, steps=W + K, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -262,15 +284,7 @@ def run_gpu(args, rank, world, local_rank):
     ms = ev[0].elapsed_time(ev[1])
     att_ms = [a.elapsed_time(b) for a, b in att]
     units_local = sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
-    t = torch.tensor([ms, float(units_local)], dtype=torch.float64, device=dev)
-    if world > 1:
-        tmax = t[:1].clone()
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        usum = t[1:].clone()
-        dist.all_reduce(usum, op=dist.ReduceOp.SUM)
-        ms_max, units_all = float(tmax.item()), float(usum.item())
-    else:
-        ms_max, units_all = ms, float(units_local)
+    ms_max, units_all = combine_ranks(ms, units_local, world, dev)
     value = units_all / (ms_max / 1000.0)
 
     # ---- roofline of the attention call (plan + split-K attention + merge) ----
@@ -297,10 +311,8 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     barrier()
     sess.check_err()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = units_all / (float(e2e_ms.item()) / 1000.0)
+    e2e_ms, _ = combine_ranks(e0.elapsed_time(e1), 0, world, dev)
+    e2e_value = units_all / (e2e_ms / 1000.0)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

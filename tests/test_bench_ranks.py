@@ -1,0 +1,64 @@
+"""The multi-rank logic of bench.py on CPU: two gloo ranks, as torchrun would start them.
+
+Each rank runs its own replica batch (same shape, its own seed) and reports its timed
+region; rank 0's line carries the max time over ranks and the sum of the units, which is
+what `value` divides. Nothing here needs a GPU.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms, units = bench.combine_ranks(10.0 + 5.0 * rank, 1000 * (rank + 1), world, "cpu")
+        e2e, zero = bench.combine_ranks(20.0 - rank, 0, world, "cpu")
+        wl = bench.rank_workload("tiny", rank)
+        out.put((rank, ms, units, e2e, zero, wl.seed, tuple(wl.seq_lens)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_time_and_summed_units():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        r = out.get(timeout=120)
+        got[r[0]] = r
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        _, ms, units, e2e, zero, _, _ = got[r]
+        assert ms == 15.0 and units == 3000.0  # max of 10 and 15 ms; 1000 + 2000 units
+        assert e2e == 20.0 and zero == 0.0
+    # same shape on every rank, different data
+    assert got[0][6] == got[1][6]
+    assert got[0][5] != got[1][5]
+
+
+def test_single_rank_passes_values_through():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.combine_ranks(12.5, 77, 1, "cpu") == (12.5, 77.0)
