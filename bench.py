@@ -7,6 +7,11 @@ merge). The workload defaults to the 1024-sequence async-rollout batch (128 grou
 responses sharing a 256-token prompt, lognormal response lengths with mean 1450).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kv4|reference]
+                  [--launch graph|eager]
+
+The timed steps are replayed from CUDA graphs captured once per step (the same kernels
+on the same per-step inputs, without host launch gaps between them); the eager numbers
+are reported beside them.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own full batch (data-parallel
 rollout replicas, no collective in the data path: weak scaling); the timed region is the
@@ -265,27 +270,51 @@ def run_gpu(args, rank, world, local_rank):
     sess.check_err()
 
     # ---- timed region: K full steps (append + attention), device events ----
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
+    steps = list(range(W, W + K))
+
+    def timed(run_append, run_attention):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in steps]
+        barrier()
+        torch.cuda.synchronize(dev)
         ev[0].record(stream)
-        for i, s in enumerate(range(W, W + K)):
-            sess.append_step(s)
+        for i, s in enumerate(steps):
+            run_append(i, s)
             att[i][0].record(stream)
-            sess.attention_step(s)
+            run_attention(i, s)
             att[i][1].record(stream)
         ev[1].record(stream)
         torch.cuda.synchronize(dev)
-    barrier()
-    sess.check_err()
-    ms = ev[0].elapsed_time(ev[1])
-    att_ms = [a.elapsed_time(b) for a, b in att]
+        barrier()
+        sess.check_err()
+        return ev[0].elapsed_time(ev[1]), [a.elapsed_time(b) for a, b in att]
+
+    # eager: every call launches its kernels from the host
+    with ClockSampler(local_rank) as clocks_eager:
+        ms_eager, att_eager = timed(lambda i, s: sess.append_step(s),
+                                    lambda i, s: sess.attention_step(s))
+    # graphs: each step's append and attention call captured once (outside the timed
+    # region) and replayed; the same kernels on the same per-step inputs
+    g_app, g_att = [], []
+    if args.launch == "graph":
+        for s in steps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                sess.append_step(s)
+            g_app.append(g)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                sess.attention_step(s)
+            g_att.append(g)
+        with ClockSampler(local_rank) as clocks:
+            ms, att_ms = timed(lambda i, s: g_app[i].replay(), lambda i, s: g_att[i].replay())
+    else:
+        clocks, ms, att_ms = clocks_eager, ms_eager, att_eager
     units_local = sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
     ms_max, units_all = combine_ranks(ms, units_local, world, dev)
     value = units_all / (ms_max / 1000.0)
+    ms_eager_max, _ = combine_ranks(ms_eager, 0, world, dev)
 
     # ---- roofline of the attention call (plan + split-K attention + merge) ----
     uniq = [attention_bytes(wl, L0 + s) for s in range(W, W + K)]
@@ -306,8 +335,10 @@ def run_gpu(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
+    t_host = time.perf_counter()
     pipe.run(hk, hv, hq, hl, hout, range(W, W + K), start_event=e0)
     e1.record(stream)
+    host_ms = (time.perf_counter() - t_host) * 1000.0  # host time to issue the K steps
     torch.cuda.synchronize(dev)
     barrier()
     sess.check_err()
@@ -331,8 +362,13 @@ def run_gpu(args, rank, world, local_rank):
             "config": {"workload": wl.name, **wl.describe(),
                        "l2": "inputs larger than L2: the cache read per step is "
                              f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
-                       "parallelism": f"dp{world} (independent replica batches)"},
+                       "parallelism": f"dp{world} (independent replica batches)",
+                       "launch": ("cuda graph per step (append call, attention call)"
+                                  if args.launch == "graph" else "eager")},
             "attention_ms": statistics.mean(att_ms),
+            "eager": {"value": units_all / (ms_eager_max / 1000.0),
+                      "ms_per_step": ms_eager_max / K,
+                      "attention_ms": statistics.mean(att_eager)},
             "attention_gbs_unique": ub / mean_att_s / 1e9,
             "attention_gbs_logical": lb / mean_att_s / 1e9,
             "roofline": {"kernel": "kv4_decode_attention (plan + attention + merge launches)",
@@ -340,12 +376,14 @@ def run_gpu(args, rank, world, local_rank):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": None},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
+                    "host_issue_ms_per_step": host_ms / K},
             "gpu_launches": 4 * K,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    del g_app, g_att
     if world > 1:
         dist.destroy_process_group()
 
@@ -359,6 +397,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="rollout")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
+                    help="timed steps replayed from CUDA graphs (default) or launched eagerly")
     args = ap.parse_args(argv)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -178,7 +178,7 @@ kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
  *
  *   q:       bf16 [num_seqs][Hq][128], finite. Each query enters the dot products as
  *            15-bit fixed point with a power-of-two step set by its largest element
- *            (relative rounding at most 2^-15 of that element).
+ *            (rounding at most 2^-14 of that element's magnitude).
  *   out:     bf16 [num_seqs][Hq][128].
  *   out_f32: optional fp32 [num_seqs][Hq][128] (NULL to skip).
  *   lse:     optional fp32 [num_seqs][Hq], natural log of the softmax denominator
