@@ -134,10 +134,37 @@ __device__ void block_scan_n(int (&v)[kScanN], int (&tot)[kScanN], int (*warp_su
   __syncthreads();
 }
 
+// Ranks of the threads' keys within one block of 1024 sequences, stable in sequence
+// order: rank = earlier threads with the same key. Keys are in [0, 32) or -1 (none).
+// cnt: shared scratch; chunk_tot[k] receives the block's count of key k.
+__device__ int key_rank(int key, int (*cnt)[33], int *chunk_tot) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 32 * 33; i += blockDim.x) (&cnt[0][0])[i] = 0;
+  __syncthreads();
+  const unsigned same = __match_any_sync(0xffffffffu, key);
+  const int lr = __popc(same & ((1u << lane) - 1u));
+  if (key >= 0 && lr == 0) cnt[key][wid] = __popc(same);
+  __syncthreads();
+  if (threadIdx.x < 32) {  // per key: exclusive scan over the 32 warps
+    int sum = 0;
+    for (int wi = 0; wi < 32; ++wi) {
+      const int v = cnt[threadIdx.x][wi];
+      cnt[threadIdx.x][wi] = sum;
+      sum += v;
+    }
+    chunk_tot[threadIdx.x] = sum;
+  }
+  __syncthreads();
+  const int rank = key >= 0 ? cnt[key][wid] + lr : 0;
+  __syncthreads();
+  return rank;
+}
+
 struct SeqPlan {
   Regions g;
   int pages;   // INT4 pages of the sequence's INT4 range
   int nfull;   // INT4 chunks of exactly chunk_pages pages
+  int key = -1;  // short last chunk: 31 - its pages (sort key), else -1
   bool last_long;  // the shorter last chunk (if any) has at least half the pages
   // scanned values: regions (protected set + INT4 chunks), then entries per class
   // (full chunks, long partial chunks, protected sets, short chunks)
@@ -147,6 +174,10 @@ struct SeqPlan {
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspace w,
                                                             int32_t *err) {
   __shared__ int warp_sums[kScanN][32];
+  // the short class is ordered by decreasing chunk length (key = 31 - pages), so that
+  // the last entries of the kernel are the shortest
+  __shared__ int key_cnt[32][33];
+  __shared__ int key_chunk[32], key_tot[32], key_run[32];
   const int B = c.num_seqs, H = c.num_kv_heads, C = w.chunk_pages;
   const int S = c.num_sinks, R = c.num_recent;
   const int hpw = w.heads_per_warp;
@@ -173,18 +204,31 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     sp.n[2] = has_last && sp.last_long ? nslots : 0;
     sp.n[3] = sp.g.has_prot * nslots;
     sp.n[4] = has_last && !sp.last_long ? nslots : 0;
+    sp.key = sp.n[4] ? 31 - (sp.pages - sp.nfull * C) : -1;
     return sp;
   };
 
   // pass 1: totals over every sequence
   int tot[kScanN] = {0, 0, 0, 0, 0};
+  if (threadIdx.x < 32) key_tot[threadIdx.x] = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
     SeqPlan sp = plan_of(base + threadIdx.x);
     int t[kScanN];
     block_scan_n(sp.n, t, warp_sums);
 #pragma unroll
     for (int i = 0; i < kScanN; ++i) tot[i] += t[i];
+    key_rank(sp.key, key_cnt, key_chunk);
+    if (threadIdx.x < 32) key_tot[threadIdx.x] += key_chunk[threadIdx.x];
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // first rank of every key: exclusive scan over the keys
+    int sum = 0;
+    for (int k = 0; k < 32; ++k) {
+      key_run[k] = sum;
+      sum += key_tot[k];
+    }
+  }
+  __syncthreads();
   const int te_all = tot[1] + tot[2] + tot[3] + tot[4];
   const bool fits = tot[0] <= w.cap_pairs && te_all <= w.cap_entries;
 
@@ -204,12 +248,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
       off[i] += run[i];
       run[i] += t[i];
     }
+    const int krank = key_rank(sp.key, key_cnt, key_chunk);
+    const int short_rank = sp.key >= 0 ? key_run[sp.key] + krank : 0;
+    __syncthreads();
+    if (threadIdx.x < 32) key_run[threadIdx.x] += key_chunk[threadIdx.x];
+    __syncthreads();
     if (b < my_lo || b >= my_hi) continue;
     const int pairs = sp.n[0];
     for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * off[0] + h * pairs;
     if (pairs == 0) continue;
     const Regions &g = sp.g;
-    int ef = off[1], el = off[2], epr = off[3], es = off[4];
+    int ef = off[1], el = off[2], epr = off[3];
+    const int es = tot[1] + tot[2] + tot[3] + short_rank * nslots;
     if (g.has_prot)
       for (int s = 0; s < nslots; ++s)
         w.entries[epr++] = make_int4(b, 0, s * hpw, min(hpw, H - s * hpw));
