@@ -227,6 +227,24 @@ def combine_ranks(ms, units, world, device):
     return float(t[0].item()), float(t[1].item())
 
 
+def recorded_traffic(workload):
+    """DRAM bytes (read + write) of one attention-kernel launch on `workload`, from the ncu
+    capture recorded under profiles/, or None when the kernel sources have changed since
+    that capture (or none was recorded for this workload)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_kernel_rollout1024.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    if rec.get("workload") != workload:
+        return None
+    for rel, digest in rec["sources_sha256"].items():
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -374,7 +392,7 @@ def run_gpu(args, rank, world, local_rank):
             "roofline": {"kernel": "kv4_decode_attention (plan + attention + merge launches)",
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": None},
+                         "traffic": recorded_traffic(wl.name)},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
