@@ -203,12 +203,17 @@ def run_reference(args, rank, world):
 # GPU arm
 # ----------------------------------------------------------------------------
 
-def rank_workload(name, rank):
+def rank_workload(name, rank, sinks=None, recent=None):
     """The workload of one rank: the named shape with its own data seed, so that N ranks
-    run N independent replica batches (weak scaling, no exchange)."""
+    run N independent replica batches (weak scaling, no exchange). sinks / recent
+    override the protected-set widths (the name then says so)."""
     from quantized_kv_cache_kv4_b200.workload import make_workload
     wl = make_workload(name)
     wl.seed = wl.seed + 7919 * rank
+    if sinks is not None or recent is not None:
+        wl.num_sinks = wl.num_sinks if sinks is None else int(sinks)
+        wl.num_recent = wl.num_recent if recent is None else int(recent)
+        wl.name = f"{wl.name}-S{wl.num_sinks}-R{wl.num_recent}"
     return wl
 
 
@@ -270,9 +275,14 @@ def run_gpu(args, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    wl = rank_workload(args.workload, rank)
+    wl = rank_workload(args.workload, rank, args.sinks, args.recent)
     W, K = args.warmup, args.steps
+    # one session per layer (same lengths and paging, own data); they share a workspace
     sess = DecodeSession(wl, steps=W + K, device=dev)
+    layers = [sess] + [DecodeSession(wl, layer=li, steps=W + K, device=dev,
+                                     workspace=sess.workspace)
+                       for li in range(1, wl.num_layers)]
+    nl = len(layers)
     stream = torch.cuda.current_stream(dev)
     H = wl.num_kv_heads
     L0 = wl.seq_lens.astype(np.int64)
@@ -283,53 +293,61 @@ def run_gpu(args, rank, world, local_rank):
 
     # warm-up
     for s in range(W):
-        sess.step(s)
+        for ls in layers:
+            ls.step(s)
     torch.cuda.synchronize(dev)
-    sess.check_err()
+    for ls in layers:
+        ls.check_err()
 
-    # ---- timed region: K full steps (append + attention), device events ----
+    # ---- timed region: K full steps (append + attention of every layer), device events ----
     steps = list(range(W, W + K))
 
     def timed(run_append, run_attention):
+        """run_append(i, s, l) / run_attention(i, s, l) launch step s's calls of layer l;
+        every attention call is bracketed by events."""
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in steps]
+               for _ in range(len(steps) * nl)]
         barrier()
         torch.cuda.synchronize(dev)
         ev[0].record(stream)
         for i, s in enumerate(steps):
-            run_append(i, s)
-            att[i][0].record(stream)
-            run_attention(i, s)
-            att[i][1].record(stream)
+            for li in range(nl):
+                run_append(i, s, li)
+                att[i * nl + li][0].record(stream)
+                run_attention(i, s, li)
+                att[i * nl + li][1].record(stream)
         ev[1].record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        sess.check_err()
+        for ls in layers:
+            ls.check_err()
         return ev[0].elapsed_time(ev[1]), [a.elapsed_time(b) for a, b in att]
 
     # eager: every call launches its kernels from the host
     with ClockSampler(local_rank) as clocks_eager:
-        ms_eager, att_eager = timed(lambda i, s: sess.append_step(s),
-                                    lambda i, s: sess.attention_step(s))
-    # graphs: each step's append and attention call captured once (outside the timed
-    # region) and replayed; the same kernels on the same per-step inputs
+        ms_eager, att_eager = timed(lambda i, s, li: layers[li].append_step(s),
+                                    lambda i, s, li: layers[li].attention_step(s))
+    # graphs: each step's append and attention calls captured once per layer (outside the
+    # timed region) and replayed; the same kernels on the same per-step inputs
     g_app, g_att = [], []
     if args.launch == "graph":
         for s in steps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                sess.append_step(s)
-            g_app.append(g)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                sess.attention_step(s)
-            g_att.append(g)
+            for ls in layers:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    ls.append_step(s)
+                g_app.append(g)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    ls.attention_step(s)
+                g_att.append(g)
         with ClockSampler(local_rank) as clocks:
-            ms, att_ms = timed(lambda i, s: g_app[i].replay(), lambda i, s: g_att[i].replay())
+            ms, att_ms = timed(lambda i, s, li: g_app[i * nl + li].replay(),
+                               lambda i, s, li: g_att[i * nl + li].replay())
     else:
         clocks, ms, att_ms = clocks_eager, ms_eager, att_eager
-    units_local = sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
+    units_local = nl * sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
     ms_max, units_all = combine_ranks(ms, units_local, world, dev)
     value = units_all / (ms_max / 1000.0)
     ms_eager_max, _ = combine_ranks(ms_eager, 0, world, dev)
@@ -342,24 +360,23 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---- e2e through the public API with host buffers (H2D inputs, D2H output) ----
     B, Hq, D = wl.num_seqs, wl.num_q_heads, wl.head_dim
-    hk = sess.step_k.cpu().pin_memory()
-    hv = sess.step_v.cpu().pin_memory()
-    hq = sess.q.cpu().pin_memory()
-    hl = sess.step_lens.cpu().pin_memory()
-    hout = torch.empty((K, B, Hq, D), dtype=torch.bfloat16).pin_memory()
-    pipe = HostStepPipeline(sess)
+    host_inputs = [(ls.step_k.cpu().pin_memory(), ls.step_v.cpu().pin_memory(),
+                    ls.q.cpu().pin_memory(), ls.step_lens.cpu().pin_memory()) for ls in layers]
+    hout = [torch.empty((K, B, Hq, D), dtype=torch.bfloat16).pin_memory() for _ in layers]
+    pipe = HostStepPipeline(layers)
     h2d, d2h = pipe.bytes_per_step()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     t_host = time.perf_counter()
-    pipe.run(hk, hv, hq, hl, hout, range(W, W + K), start_event=e0)
+    pipe.run(host_inputs, hout, range(W, W + K), start_event=e0)
     e1.record(stream)
     host_ms = (time.perf_counter() - t_host) * 1000.0  # host time to issue the K steps
     torch.cuda.synchronize(dev)
     barrier()
-    sess.check_err()
+    for ls in layers:
+        ls.check_err()
     e2e_ms, _ = combine_ranks(e0.elapsed_time(e1), 0, world, dev)
     e2e_value = units_all / (e2e_ms / 1000.0)
 
@@ -381,8 +398,8 @@ def run_gpu(args, rank, world, local_rank):
                        "l2": "inputs larger than L2: the cache read per step is "
                              f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
                        "parallelism": f"dp{world} (independent replica batches)",
-                       "launch": ("cuda graph per step (append call, attention call)"
-                                  if args.launch == "graph" else "eager")},
+                       "launch": ("cuda graph per call (each layer's append and attention "
+                                  "call of every step)" if args.launch == "graph" else "eager")},
             "attention_ms": statistics.mean(att_ms),
             "eager": {"value": units_all / (ms_eager_max / 1000.0),
                       "ms_per_step": ms_eager_max / K,
@@ -396,12 +413,12 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
-            "gpu_launches": 4 * K,
+            "gpu_launches": 4 * K * nl,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g_app, g_att
+    del g_app, g_att, layers
     if world > 1:
         dist.destroy_process_group()
 
@@ -415,6 +432,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="rollout")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sinks", type=int, default=None, help="override S (protection sweep)")
+    ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
     ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
                     help="timed steps replayed from CUDA graphs (default) or launched eagerly")
     args = ap.parse_args(argv)

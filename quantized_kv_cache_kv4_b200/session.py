@@ -23,7 +23,7 @@ from .workload import Workload, make_paging, queries, seq_kv
 class DecodeSession:
     def __init__(self, wl: Workload, layer: int = 0, steps: int = 1, device="cuda",
                  chunk_pages: int = 0, keep_streams=(), build: bool = True,
-                 max_rows_per_call: int = 1 << 20):
+                 max_rows_per_call: int = 1 << 20, workspace: torch.Tensor | None = None):
         self.wl = wl
         self.layer = layer
         self.steps = steps
@@ -52,7 +52,10 @@ class DecodeSession:
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_rows = max_rows_per_call
         ws = kv4.workspace_size(self.cfg, B, self.max_len)
-        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        if workspace is not None and workspace.numel() >= ws:
+            self.workspace = workspace  # shared with other layers (calls run in stream order)
+        else:
+            self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.q = torch.stack([queries(wl, s, layer, dev) for s in range(steps)])
         self.out = torch.empty((B, wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
         if build:

@@ -207,7 +207,7 @@ def test_host_pipeline_matches_serial_steps():
     hq, hl = sess.q.cpu().pin_memory(), sess.step_lens.cpu().pin_memory()
     hout = torch.empty((n,) + tuple(sess.out.shape), dtype=torch.bfloat16).pin_memory()
     pipe = HostStepPipeline(sess)
-    pipe.run(hk, hv, hq, hl, hout, range(n))
+    pipe.run([(hk, hv, hq, hl)], [hout], range(n))
     torch.cuda.synchronize()
     sess.check_err()
     for s in range(n):
