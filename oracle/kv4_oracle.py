@@ -206,6 +206,30 @@ def decode_reference(q, k, v, S: int, R: int):
     return attention(q, K, V)
 
 
+# ----------------------------------------------------------------------------
+# comparison baselines: the same decode attention over a BF16 cache and over an
+# all-INT8 (KV8) cache.  The pages compare KV4 against both: KV8 "tracks BF16
+# closely" (ai4snews summary, "Interpretation" para. 2) and the replay throughput
+# ratios are quoted against BF16 (ai4snews summary, "Interpretation" paras. 1-2).
+# ----------------------------------------------------------------------------
+
+def decode_reference_bf16(q, k, v):
+    """Decode output over an unquantised BF16 cache: plain softmax attention on the
+    bf16 values themselves.  q float32 [Hq, D]; k, v float32 (bf16 values) [L, Hkv, D]."""
+    return attention(q, k.astype(np.float64), v.astype(np.float64))
+
+
+def decode_reference_kv8(q, k, v):
+    """Decode output over an all-INT8 cache: every position quantised with the INT8
+    quantiser of the protected set (symmetric, per token and kv head, fp16 scale),
+    dequantised, then softmax attention."""
+    out = []
+    for x in (k, v):
+        c8, s8 = quantize_int8(x)
+        out.append(dequant_int8(c8, s8))
+    return attention(q, out[0], out[1])
+
+
 def partial_state(q_row: np.ndarray, K: np.ndarray, V: np.ndarray):
     """Unnormalised softmax state of one query over one region of keys.
 

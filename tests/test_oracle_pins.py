@@ -426,6 +426,39 @@ def test_all_int8_tracks_bf16_within_derived_bound():
         assert np.abs(got - ref).max() < 0.05  # and it is small in absolute terms
 
 
+def test_baseline_references_reduce_to_pinned_cases():
+    """BF16 reference = the brute-force loop on the bf16 values; KV8 reference = the
+    KV4-RL reference with every position protected (L <= S + R), and for longer
+    contexts the same INT8 quantiser applied to every position (checked against a
+    per-token loop of the pinned INT8 quantiser)."""
+    rng = np.random.default_rng(12)
+    for L in (1, 7, 100):
+        k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+        v = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+        q = _bf16(rng.normal(0, 1, (8, 128)).astype(np.float32))
+        got, _ = O.decode_reference_bf16(q, k, v)
+        assert np.max(np.abs(got - _loop_attention(q, k.astype(np.float64),
+                                                   v.astype(np.float64)))) < 1e-12
+        kv8, _ = O.decode_reference_kv8(q, k, v)
+        if L <= 144:
+            want, _ = O.decode_reference(q, k, v, 16, 128)
+            assert np.array_equal(kv8, want)
+    L = 400  # beyond any protected set: quantise token by token
+    k = _bf16(rng.normal(0, 2, (L, 2, 128)).astype(np.float32))
+    v = _bf16(rng.normal(0, 2, (L, 2, 128)).astype(np.float32))
+    q = _bf16(rng.normal(0, 1, (8, 128)).astype(np.float32))
+    Kd = np.zeros((L, 2, 128))
+    Vd = np.zeros((L, 2, 128))
+    for t in range(L):
+        for h in range(2):
+            c, sc = O.quantize_int8(k[t:t + 1, h:h + 1])
+            Kd[t, h] = O.dequant_int8(c, sc)[0, 0]
+            c, sc = O.quantize_int8(v[t:t + 1, h:h + 1])
+            Vd[t, h] = O.dequant_int8(c, sc)[0, 0]
+    got, _ = O.decode_reference_kv8(q, k, v)
+    assert np.max(np.abs(got - _loop_attention(q, Kd, Vd))) < 1e-12
+
+
 def test_expected_pages_layout():
     rng = np.random.default_rng(11)
     L = 21
