@@ -236,6 +236,55 @@ kv4_status kv4_decode_attention_noalloc(const kv4_config *cfg, const kv4_int4_po
 /* Size of the fixed scratch array kv4_decode_attention_noalloc uses, in bytes. */
 size_t kv4_noalloc_scratch_bytes(void);
 
+/* ---------------------------------------------------------------------------------------
+ * Comparison baselines: the same paged decode attention over an unquantised BF16 cache
+ * and over an all-INT8 (KV8) cache, for the throughput comparison the pages make between
+ * KV4, KV8 and BF16 caches (ai4snews summary, "Interpretation" paras. 1-2: KV8 tracks
+ * BF16 closely; replay throughput ratios against BF16). No protected set: cfg's num_sinks
+ * and num_recent are ignored (taken as 0); the other cfg fields, the batch (sink_idx and
+ * ring_idx unused), the workspace, the error bits and the output contract are those of
+ * kv4_decode_attention. KV8 quantises every position with the INT8 quantiser of the
+ * protected set (symmetric per token and kv head, fp16 scale = RN(amax/127), codes
+ * RNE-clamped to [-127, 127]).
+ * ------------------------------------------------------------------------------------- */
+typedef enum {
+  KV4_BASELINE_BF16 = 1,
+  KV4_BASELINE_KV8 = 2
+} kv4_baseline_format;
+
+/* Paged baseline cache, per (page, kv head) block of 16 positions:
+ *   BF16: k, v: bf16 [num_pages][Hkv][16 octets][16 slots][8]; element (slot t, dim d) at
+ *         [d/8][t][d%8] (4 KiB per block); k_scales, v_scales unused (may be NULL).
+ *   KV8:  k, v: int8 [num_pages][Hkv][8 strips][16 slots][16]; element (t, d) at
+ *         [d/16][t][d%16] (2 KiB per block); k_scales, v_scales: fp16 [num_pages][Hkv][16].
+ * All pointers 16-byte aligned device memory owned by the caller. */
+typedef struct {
+  void *k;
+  void *v;
+  uint16_t *k_scales;
+  uint16_t *v_scales;
+  int32_t num_pages;
+} kv4_paged_pool;
+
+/* Append new tokens (same CSR contract as kv4_quantize_append): BF16 copies each row into
+ * its page slot; KV8 quantises it. Data-dependent errors as for kv4_quantize_append. */
+kv4_status kv4_baseline_append(kv4_baseline_format fmt, const kv4_config *cfg,
+                               const kv4_paged_pool *pool, const kv4_batch *batch,
+                               const void *k_new, const void *v_new, const int32_t *new_indptr,
+                               int32_t total_new, int32_t *err_flag, kv4_stream_t stream);
+
+/* Workspace bytes for kv4_baseline_decode_attention (0 on invalid arguments). */
+size_t kv4_baseline_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len);
+
+/* Decode attention over the baseline cache: O[b, j] = softmax(K q / sqrt(128)) V over
+ * positions [0, seq_lens[b]) with K, V the stored bf16 values (BF16) or the dequantised
+ * INT8 codes (KV8). Outputs, workspace and errors as for kv4_decode_attention. */
+kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_config *cfg,
+                                         const kv4_paged_pool *pool, const kv4_batch *batch,
+                                         const void *q, void *out, float *out_f32, float *lse,
+                                         void *workspace, size_t ws_bytes, int32_t *err_flag,
+                                         kv4_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *kv4_status_string(kv4_status status);
 

@@ -112,6 +112,73 @@ kv4_status make_view(const kv4_config *cfg, const kv4_int4_pool *pool, const kv4
   return KV4_OK;
 }
 
+// The comparison baselines have no protected set: the config is used with S = R = 0.
+kv4_config without_protection(const kv4_config *cfg) {
+  kv4_config c = *cfg;
+  c.num_sinks = 0;
+  c.num_recent = 0;
+  return c;
+}
+
+kv4_status make_baseline_view(kv4_baseline_format fmt, const kv4_config *cfg,
+                              const kv4_paged_pool *pool, const kv4_batch *batch,
+                              kv4::CacheView *v) {
+  if (fmt != KV4_BASELINE_BF16 && fmt != KV4_BASELINE_KV8) return KV4_ERR_INVALID_ARG;
+  kv4_status st = check_config(cfg);
+  if (st != KV4_OK) return st;
+  if (pool == nullptr || batch == nullptr) return KV4_ERR_INVALID_ARG;
+  if (batch->num_seqs < 0 || batch->max_pages <= 0 || batch->max_seq_len < 0 ||
+      pool->num_pages < 0)
+    return KV4_ERR_INVALID_ARG;
+  if (batch->num_seqs > 0 && (batch->page_table == nullptr || batch->seq_lens == nullptr))
+    return KV4_ERR_INVALID_ARG;
+  if (!pool->k || !pool->v || misaligned16(pool->k) || misaligned16(pool->v))
+    return KV4_ERR_INVALID_ARG;
+  if (fmt == KV4_BASELINE_KV8 && (!pool->k_scales || !pool->v_scales ||
+                                  misaligned16(pool->k_scales) || misaligned16(pool->v_scales)))
+    return KV4_ERR_INVALID_ARG;
+  *v = kv4::CacheView{};
+  v->k_codes = static_cast<uint8_t *>(pool->k);
+  v->v_codes = static_cast<uint8_t *>(pool->v);
+  v->k_params = pool->k_scales;
+  v->v_params = pool->v_scales;
+  v->num_pages = pool->num_pages;
+  v->page_table = batch->page_table;
+  v->max_pages = batch->max_pages;
+  v->seq_lens = batch->seq_lens;
+  v->num_seqs = batch->num_seqs;
+  v->num_kv_heads = cfg->num_kv_heads;
+  v->gqa = cfg->num_q_heads / cfg->num_kv_heads;
+  return KV4_OK;
+}
+
+// Carve the workspace for (cfg, batch): the automatic chunk choice, falling back to the
+// longest chunks when the caller's workspace is too small for a finer split.
+kv4_status carve_workspace(const kv4_config *cfg, const kv4::CacheView &v,
+                           const kv4_batch *batch, void *workspace, size_t ws_bytes,
+                           kv4::Workspace *w) {
+  size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
+                                     chunk_of(cfg, batch->num_seqs, batch->max_seq_len), w,
+                                     workspace);
+  // A workspace sized for a larger batch or longer sequences (and so for longer automatic
+  // chunks) may be too small for a finer automatic split of this one: fall back to the
+  // longest chunks, for which any workspace sized with this config at larger or equal
+  // (num_seqs, max_seq_len) is large enough.
+  if (ws_bytes < need && cfg->chunk_pages == 0)
+    need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
+                                kv4::kMaxChunkPages, w, workspace);
+  return ws_bytes < need ? KV4_ERR_WORKSPACE_TOO_SMALL : KV4_OK;
+}
+
+kv4_status check_attention_args(const kv4_batch *batch, const void *q, const void *out,
+                                const float *out_f32, const void *workspace) {
+  if (q == nullptr || out == nullptr || workspace == nullptr) return KV4_ERR_INVALID_ARG;
+  if (misaligned16(q) || misaligned16(out) || misaligned16(out_f32) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return KV4_ERR_INVALID_ARG;
+  return batch->num_seqs >= 0 ? KV4_OK : KV4_ERR_INVALID_ARG;
+}
+
 }  // namespace
 
 extern "C" {
@@ -149,22 +216,11 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   kv4_status st = make_view(cfg, pool, side, batch, &v);
   if (st != KV4_OK) return st;
   if (batch->num_seqs == 0) return KV4_OK;
-  if (q == nullptr || out == nullptr || workspace == nullptr) return KV4_ERR_INVALID_ARG;
-  if (misaligned16(q) || misaligned16(out) || misaligned16(out_f32) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return KV4_ERR_INVALID_ARG;
+  st = check_attention_args(batch, q, out, out_f32, workspace);
+  if (st != KV4_OK) return st;
   kv4::Workspace w;
-  size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
-                                     chunk_of(cfg, batch->num_seqs, batch->max_seq_len), &w,
-                                     workspace);
-  // A workspace sized for a larger batch or longer sequences (and so for longer automatic
-  // chunks) may be too small for a finer automatic split of this one: fall back to the
-  // longest chunks, for which any workspace sized with this config at larger or equal
-  // (num_seqs, max_seq_len) is large enough.
-  if (ws_bytes < need && cfg->chunk_pages == 0)
-    need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
-                                kv4::kMaxChunkPages, &w, workspace);
-  if (ws_bytes < need) return KV4_ERR_WORKSPACE_TOO_SMALL;
+  st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
+  if (st != KV4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
   if (e == cudaSuccess)
@@ -191,6 +247,61 @@ kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offse
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
+size_t kv4_baseline_workspace_size(const kv4_config *cfg, int32_t num_seqs,
+                                   int32_t max_seq_len) {
+  if (cfg == nullptr) return 0;
+  const kv4_config c = without_protection(cfg);
+  return kv4_workspace_size(&c, num_seqs, max_seq_len);
+}
+
+kv4_status kv4_baseline_append(kv4_baseline_format fmt, const kv4_config *cfg,
+                               const kv4_paged_pool *pool, const kv4_batch *batch,
+                               const void *k_new, const void *v_new, const int32_t *new_indptr,
+                               int32_t total_new, int32_t *err_flag, kv4_stream_t stream) {
+  if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
+  const kv4_config c = without_protection(cfg);
+  kv4::CacheView v;
+  kv4_status st = make_baseline_view(fmt, &c, pool, batch, &v);
+  if (st != KV4_OK) return st;
+  if (total_new < 0) return KV4_ERR_INVALID_ARG;
+  if (new_indptr == nullptr && total_new != batch->num_seqs) return KV4_ERR_INVALID_ARG;
+  if (total_new > 0 && (k_new == nullptr || v_new == nullptr)) return KV4_ERR_INVALID_ARG;
+  if (misaligned16(k_new) || misaligned16(v_new)) return KV4_ERR_INVALID_ARG;
+  if (total_new == 0 || batch->num_seqs == 0) return KV4_OK;
+  cudaError_t e = kv4::launch_baseline_append(fmt, v, static_cast<const uint16_t *>(k_new),
+                                              static_cast<const uint16_t *>(v_new), new_indptr,
+                                              total_new, err_flag,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_config *cfg,
+                                         const kv4_paged_pool *pool, const kv4_batch *batch,
+                                         const void *q, void *out, float *out_f32, float *lse,
+                                         void *workspace, size_t ws_bytes, int32_t *err_flag,
+                                         kv4_stream_t stream) {
+  if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
+  const kv4_config c = without_protection(cfg);
+  kv4::CacheView v;
+  kv4_status st = make_baseline_view(fmt, &c, pool, batch, &v);
+  if (st != KV4_OK) return st;
+  if (batch->num_seqs == 0) return KV4_OK;
+  st = check_attention_args(batch, q, out, out_f32, workspace);
+  if (st != KV4_OK) return st;
+  kv4::Workspace w;
+  st = carve_workspace(&c, v, batch, workspace, ws_bytes, &w);
+  if (st != KV4_OK) return st;
+  w.heads_per_warp = 1;  // one kv head per warp and entry
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_baseline_attention(fmt, v, w, static_cast<const uint16_t *>(q), err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
+                          static_cast<uint16_t *>(out), out_f32, lse, s);
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
 const char *kv4_status_string(kv4_status status) {
   switch (status) {
     case KV4_OK: return "ok";
@@ -203,6 +314,6 @@ const char *kv4_status_string(kv4_status status) {
   return "unknown status";
 }
 
-int32_t kv4_version(void) { return 100; }
+int32_t kv4_version(void) { return 200; }
 
 }  // extern "C"

@@ -28,22 +28,7 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t
   const int h = warp - row * H;
 
   int b, pos, L;
-  if (new_indptr == nullptr) {
-    b = row;
-    L = c.seq_lens[b];
-    pos = L - 1;
-  } else {
-    int lo = 0, hi = c.num_seqs - 1;  // largest b with new_indptr[b] <= row
-    while (lo < hi) {
-      int mid = (lo + hi + 1) >> 1;
-      if (new_indptr[mid] <= row) lo = mid; else hi = mid - 1;
-    }
-    b = lo;
-    const int n = new_indptr[b + 1] - new_indptr[b];
-    const int i = row - new_indptr[b];
-    L = c.seq_lens[b];
-    pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
-  }
+  locate_new_token(c.seq_lens, c.num_seqs, new_indptr, row, b, pos, L);
   if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
     if (lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
     return;

@@ -29,65 +29,9 @@
 //                the kernel behind kv4_regional_merge.
 #include <math_constants.h>
 
-#include "kv4_device.cuh"
-#include "kv4_internal.h"
+#include "kv4_attn_common.cuh"
 
 namespace kv4 {
-
-constexpr int kWarps = 4;                 // warps per CTA (independent work streams)
-constexpr int kStages = 3;                // shared-memory stages per warp
-constexpr int kStageBytes = 5120;         // two kv heads' INT4 page blocks; >= one INT8 tile
-constexpr int kPWordsPerCol = 12;         // P' tile column stride in words (bank-conflict free)
-constexpr int kPtileBytes = 2 * 4 * 8 * kPWordsPerCol * 4;  // [2 slots][4 groups][8 cols][12 w]
-constexpr int kPtile8Bytes = 8 * 16 * 2;  // INT8 P': [8 heads][16 tokens] fp16
-constexpr int kWarpSmem = kStages * kStageBytes + kPtileBytes + kPtile8Bytes + 64;
-constexpr int kCtaSmem = kWarps * kWarpSmem;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kNegBig = -1.0e30f;  // running-max start: finite, so e^(m_old-m_new) is 0 not NaN
-constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
-
-// V codes enter the PV product through the fp8 conversion: a byte b in 0..15 read as
-// e4m3 is exactly b * 2^-9, so the products are scaled by 2^-9 and the 2^9 is applied
-// once to the output.
-constexpr float kUnscaleV = kCvtUnscale;
-
-// INT8 stage: K codes | V codes | K scales | V scales
-constexpr int kOffVc8 = 2048, kOffKs8 = 4096, kOffVs8 = 4128, kInt8Bytes = 4160;
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// ---------------------------------------------------------------------------
-// region bookkeeping shared by plan and attention
-// ---------------------------------------------------------------------------
-struct Regions {
-  int has_prot;          // 1 if the INT8 protected set is non-empty
-  int first_page;        // first page of the INT4 range
-  int int4_lo, int4_hi;  // INT4 token range [lo, hi)
-  int n_chunks;
-};
-
-__device__ __forceinline__ Regions regions_of(int L, int S, int R, int C) {
-  Regions g;
-  const int n_sink = min(S, L);
-  const int rec_lo = max(S, L - R);
-  g.has_prot = (n_sink > 0 || rec_lo < L) ? 1 : 0;
-  g.int4_lo = S;
-  g.int4_hi = L - R;
-  if (g.int4_hi > g.int4_lo) {
-    g.first_page = g.int4_lo / kPage;
-    const int last = (g.int4_hi - 1) / kPage;
-    g.n_chunks = (last - g.first_page + 1 + C - 1) / C;
-  } else {
-    g.first_page = 0;
-    g.n_chunks = 0;
-  }
-  return g;
-}
 
 // ---------------------------------------------------------------------------
 // plan: a few CTAs of 1024 threads. Every CTA scans all sequences (a few KB of lengths)
@@ -278,82 +222,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     *w.counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
   }
-}
-
-// ---------------------------------------------------------------------------
-// attention
-// ---------------------------------------------------------------------------
-struct WarpCtx {
-  uint8_t *stage0;     // first stage (generic pointer)
-  uint32_t *ptile;     // INT4 P' tile [2 slots][4 groups][8 cols][12 words], zero padded
-  uint16_t *ptile8;    // INT8 P' tile [8 heads][16 tokens]
-  uint64_t *bars;      // kStages mbarriers
-  uint32_t parity;     // bit s = parity of the next completion of stage s
-  int lane, gid, tig;
-  bool dead;           // a bounded wait gave up: stop taking work
-};
-
-// Online softmax update for this thread's two heads (2tig, 2tig+1) with logits of
-// tokens (gid, gid+8) in log2 units. Returns p in s[][] and the rescale factors.
-__device__ __forceinline__ void softmax_step(float (&s)[2][2], float (&m)[2], float (&l)[2],
-                                             float (&alpha)[2]) {
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    float t = fmaxf(s[0][e], s[1][e]);
-    t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
-    t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
-    t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-    const float mn = fmaxf(m[e], t);
-    alpha[e] = fast_exp2(m[e] - mn);
-    m[e] = mn;
-    s[0][e] = fast_exp2(s[0][e] - mn);
-    s[1][e] = fast_exp2(s[1][e] - mn);
-    l[e] = l[e] * alpha[e] + s[0][e] + s[1][e];
-  }
-}
-
-__device__ __forceinline__ bool wait_stage(WarpCtx &x, int stage, int32_t *err) {
-  const bool ok = mbar_wait_bounded(&x.bars[stage], (x.parity >> stage) & 1u);
-  x.parity ^= 1u << stage;
-  if (!ok) {
-    x.dead = true;
-    if (x.lane == 0) set_err(err, KV4_DEVERR_TIMEOUT);
-  }
-  return ok;
-}
-
-// Write the empty partial state (-inf, 0, 0) for the G heads of a record group.
-__device__ void write_empty(float *rec, int G, int lane) {
-  for (int j = 0; j < G; ++j) {
-    float *r = rec + j * kRecordFloats;
-    reinterpret_cast<float4 *>(r)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane == 0) {
-      r[kHeadDim] = -CUDART_INF_F;
-      r[kHeadDim + 1] = 0.0f;
-    }
-  }
-}
-
-__device__ __forceinline__ float *record_of(const Workspace &w, int H, int G, int b, int h, int r) {
-  return w.partials + static_cast<size_t>(w.unit_offsets[b * H + h] + r) * G * kRecordFloats;
-}
-
-__device__ __forceinline__ uint4 load_q8(const uint16_t *qrow, int dim0, bool live) {
-  if (!live) return make_uint4(0, 0, 0, 0);
-  return *reinterpret_cast<const uint4 *>(qrow + dim0);
-}
-
-// Fixed-point step of a query: 2^e with max|q| < 2^(e+14), so every |q / 2^e| <= 2^14
-// (15 bits with the sign). amax is the lane's max|q|; the 4 lanes of a column combine.
-__device__ __forceinline__ float query_step(float amax) {
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  int ex = 0;
-  if (amax > 0.f) {
-    frexpf(amax, &ex);  // amax < 2^ex
-    ex -= 14;
-  }
-  return ldexpf(1.0f, ex);
 }
 
 // ------------------------- INT8 protected set ----------------------------
@@ -1252,9 +1120,6 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
   if (o.lse && lane == 0) o.lse[row] = lam > 0.f ? M + logf(lam) : -CUDART_INF_F;
 }
 
-#ifndef KV4_MIN_BLOCKS
-#define KV4_MIN_BLOCKS 3  // CTAs per SM the register budget is sized for
-#endif
 
 template <int HPW>
 __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(CacheView c, Workspace w,

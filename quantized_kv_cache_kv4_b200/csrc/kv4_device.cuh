@@ -104,6 +104,15 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a01, uint32_t a2
 //   A: a0 = (row gid, k 4tig..+3), a1 = (row gid+8, k 4tig..+3),
 //      a2 = (row gid, k 16+4tig..+3), a3 = (row gid+8, k 16+4tig..+3)
 //   B: b0 = (k 4tig..+3, col gid), b1 = (k 16+4tig..+3, col gid); C as for mma_f16.
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a01, uint32_t a23, uint32_t a45,
+                                         uint32_t a67, uint32_t b01, uint32_t b23) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a01), "r"(a23), "r"(a45), "r"(a67), "r"(b01), "r"(b23));
+}
+
 __device__ __forceinline__ void mma_u8s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -241,6 +250,32 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 // fp16 round-to-nearest-even with saturation to +-65504.
 __device__ __forceinline__ __half f16_sat(float x) {
   return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
+}
+
+// The sequence and position of new-token row `row` of an append call: one row per
+// sequence (indptr == nullptr: position L-1), or CSR ranges (the rows of sequence b are
+// the last indptr[b+1]-indptr[b] positions before its length L). pos = -1 when the row
+// lies outside every range.
+__device__ __forceinline__ void locate_new_token(const int32_t *__restrict__ seq_lens,
+                                                 int num_seqs,
+                                                 const int32_t *__restrict__ indptr, int row,
+                                                 int &b, int &pos, int &L) {
+  if (indptr == nullptr) {
+    b = row;
+    L = seq_lens[b];
+    pos = L - 1;
+    return;
+  }
+  int lo = 0, hi = num_seqs - 1;  // largest b with indptr[b] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (indptr[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  b = lo;
+  const int n = indptr[b + 1] - indptr[b];
+  const int i = row - indptr[b];
+  L = seq_lens[b];
+  pos = (i >= 0 && i < n) ? L - n + i : -1;
 }
 
 __device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {

@@ -71,4 +71,12 @@ cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int
                          int32_t group, uint16_t *out, float *out_f32, float *lse,
                          cudaStream_t s);
 
+// Comparison baselines (kv4_baseline.cu): fmt is a kv4_baseline_format. The view's
+// k_codes / v_codes hold the BF16 or INT8 pages, k_params / v_params the KV8 scales.
+cudaError_t launch_baseline_append(int fmt, const CacheView &c, const uint16_t *k_new,
+                                   const uint16_t *v_new, const int32_t *new_indptr,
+                                   int32_t total_new, int32_t *err_flag, cudaStream_t s);
+cudaError_t launch_baseline_attention(int fmt, const CacheView &c, const Workspace &w,
+                                      const uint16_t *q, int32_t *err_flag, cudaStream_t s);
+
 }  // namespace kv4

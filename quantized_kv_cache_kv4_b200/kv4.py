@@ -30,7 +30,12 @@ GROUP = 32
 
 EXPORTS = ("kv4_workspace_size", "kv4_quantize_append", "kv4_decode_attention",
            "kv4_regional_merge", "kv4_status_string", "kv4_version",
-           "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes")
+           "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes",
+           "kv4_baseline_append", "kv4_baseline_workspace_size",
+           "kv4_baseline_decode_attention")
+
+BASELINE_BF16 = 1  # kv4_baseline_format
+BASELINE_KV8 = 2
 
 
 class Config(ctypes.Structure):
@@ -62,6 +67,12 @@ class Batch(ctypes.Structure):
                 ("max_seq_len", ctypes.c_int32)]
 
 
+class PagedPool(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32)]
+
+
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(f"libkv4.so not built at {path}: run "
@@ -87,6 +98,18 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  P, P, P, P, P, P]
     lib.kv4_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.kv4_noalloc_scratch_bytes.argtypes = []
+    lib.kv4_baseline_append.restype = ctypes.c_int
+    lib.kv4_baseline_append.argtypes = [ctypes.c_int, ctypes.POINTER(Config),
+                                        ctypes.POINTER(PagedPool), ctypes.POINTER(Batch),
+                                        P, P, P, ctypes.c_int32, P, P]
+    lib.kv4_baseline_workspace_size.restype = ctypes.c_size_t
+    lib.kv4_baseline_workspace_size.argtypes = [ctypes.POINTER(Config), ctypes.c_int32,
+                                                ctypes.c_int32]
+    lib.kv4_baseline_decode_attention.restype = ctypes.c_int
+    lib.kv4_baseline_decode_attention.argtypes = [ctypes.c_int, ctypes.POINTER(Config),
+                                                  ctypes.POINTER(PagedPool),
+                                                  ctypes.POINTER(Batch), P, P, P, P, P,
+                                                  ctypes.c_size_t, P, P]
     lib.kv4_status_string.restype = ctypes.c_char_p
     lib.kv4_status_string.argtypes = [ctypes.c_int]
     lib.kv4_version.restype = ctypes.c_int32
@@ -254,3 +277,73 @@ def regional_merge(partials: torch.Tensor, region_offsets: torch.Tensor, group: 
 
 def decode_err(flag: int) -> list[str]:
     return [name for bit, name in DEVERR.items() if flag & bit]
+
+
+# ----------------------------------------------------------------------------
+# comparison baselines (BF16 and all-INT8 paged caches)
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class BaselineCache:
+    """Device storage of one layer's BF16 or KV8 paged cache (layouts in kv4.h)."""
+
+    fmt: int
+    cfg: Config
+    k: torch.Tensor
+    v: torch.Tensor
+    k_scales: torch.Tensor | None
+    v_scales: torch.Tensor | None
+
+    @property
+    def num_pages(self):
+        return self.k.shape[0]
+
+    def pool_struct(self) -> PagedPool:
+        ks = 0 if self.k_scales is None else self.k_scales.data_ptr()
+        vs = 0 if self.v_scales is None else self.v_scales.data_ptr()
+        return PagedPool(self.k.data_ptr(), self.v.data_ptr(), ks, vs, self.num_pages)
+
+
+def allocate_baseline_cache(fmt: int, cfg: Config, num_pages: int, device="cuda") -> BaselineCache:
+    """Zero-initialised BF16 ([pages, Hkv, 16 octets, 16 slots, 8]) or KV8 ([pages, Hkv,
+    8 strips, 16 slots, 16] int8 + fp16 scales [pages, Hkv, 16]) page pool."""
+    H = cfg.num_kv_heads
+    z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=device)
+    if fmt == BASELINE_BF16:
+        return BaselineCache(fmt, cfg, z((num_pages, H, 16, PAGE, 8), torch.bfloat16),
+                             z((num_pages, H, 16, PAGE, 8), torch.bfloat16), None, None)
+    if fmt == BASELINE_KV8:
+        return BaselineCache(fmt, cfg, z((num_pages, H, 8, PAGE, 16), torch.int8),
+                             z((num_pages, H, 8, PAGE, 16), torch.int8),
+                             z((num_pages, H, PAGE), torch.int16),
+                             z((num_pages, H, PAGE), torch.int16))
+    raise ValueError(f"unknown baseline format {fmt}")
+
+
+def baseline_workspace_size(cfg: Config, num_seqs: int, max_seq_len: int) -> int:
+    n = _lib.kv4_baseline_workspace_size(ctypes.byref(cfg), num_seqs, max_seq_len)
+    if n == 0 and num_seqs > 0:
+        raise KV4Error("kv4_baseline_workspace_size: invalid arguments")
+    return n
+
+
+def baseline_append(cache: BaselineCache, batch: BatchTensors, k_new: torch.Tensor,
+                    v_new: torch.Tensor, new_indptr: torch.Tensor | None = None,
+                    err: torch.Tensor | None = None, stream=None):
+    pool, bs = cache.pool_struct(), batch.struct()
+    st = _lib.kv4_baseline_append(cache.fmt, ctypes.byref(cache.cfg), ctypes.byref(pool),
+                                  ctypes.byref(bs), _ptr(k_new), _ptr(v_new), _ptr(new_indptr),
+                                  int(k_new.shape[0]), _ptr(err), _stream(stream))
+    _check(st, "kv4_baseline_append")
+
+
+def baseline_decode_attention(cache: BaselineCache, batch: BatchTensors, q: torch.Tensor,
+                              out: torch.Tensor, workspace: torch.Tensor,
+                              out_f32: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                              err: torch.Tensor | None = None, stream=None):
+    pool, bs = cache.pool_struct(), batch.struct()
+    st = _lib.kv4_baseline_decode_attention(cache.fmt, ctypes.byref(cache.cfg),
+                                            ctypes.byref(pool), ctypes.byref(bs), _ptr(q),
+                                            _ptr(out), _ptr(out_f32), _ptr(lse), _ptr(workspace),
+                                            workspace.numel(), _ptr(err), _stream(stream))
+    _check(st, "kv4_baseline_decode_attention")

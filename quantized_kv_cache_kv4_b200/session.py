@@ -31,9 +31,7 @@ class DecodeSession:
         self.paging = make_paging(wl, extra_tokens=steps)
         self.cfg = kv4.make_config(wl.num_q_heads, wl.num_kv_heads, wl.num_sinks,
                                    wl.num_recent, chunk_pages)
-        self.cache = kv4.allocate_cache(self.cfg, self.paging.num_pages,
-                                        self.paging.num_sink_sets, self.paging.num_rings,
-                                        device=self.device)
+        self.cache = self._allocate_cache()
         B = wl.num_seqs
         self.L0 = wl.seq_lens.astype(np.int64)  # lengths after step 0's append
         dev = self.device
@@ -51,7 +49,7 @@ class DecodeSession:
         self.step_v = torch.empty_like(self.step_k)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_rows = max_rows_per_call
-        ws = kv4.workspace_size(self.cfg, B, self.max_len)
+        ws = self._workspace_size(B, self.max_len)
         if workspace is not None and workspace.numel() >= ws:
             self.workspace = workspace  # shared with other layers (calls run in stream order)
         else:
@@ -62,6 +60,16 @@ class DecodeSession:
             self.build()
 
     # ------------------------------------------------------------------ helpers
+    def _allocate_cache(self):
+        return kv4.allocate_cache(self.cfg, self.paging.num_pages, self.paging.num_sink_sets,
+                                  self.paging.num_rings, device=self.device)
+
+    def _workspace_size(self, num_seqs, max_len):
+        return kv4.workspace_size(self.cfg, num_seqs, max_len)
+
+    def _append(self, batch, k, v, indptr, stream=None):
+        kv4.quantize_append(self.cache, batch, k, v, indptr, self.err, stream=stream)
+
     def batch(self, lens: torch.Tensor) -> kv4.BatchTensors:
         return kv4.BatchTensors(self.page_table, lens, self.sink_idx, self.ring_idx,
                                 self.max_len)
@@ -78,7 +86,7 @@ class DecodeSession:
         b = kv4.BatchTensors(self.page_table if page_table is None else page_table,
                              torch.as_tensor(lens_after.astype(np.int32), device=dev),
                              self.sink_idx, self.ring_idx, self.max_len)
-        kv4.quantize_append(self.cache, b, k, v, torch.as_tensor(indptr, device=dev), self.err)
+        self._append(b, k, v, torch.as_tensor(indptr, device=dev))
 
     def _gen(self, b):
         end = int(self.L0[b]) + self.steps
@@ -108,6 +116,8 @@ class DecodeSession:
             self._append_rows(rows_k, rows_v, counts, lens)
             # 2. fork the leader's ring to the group's other sequences
             leader_of = {}
+            rings = [] if not hasattr(self.cache, "ring_k") else [
+                self.cache.ring_k, self.cache.ring_v, self.cache.ring_ks, self.cache.ring_vs]
             for b in range(B):
                 g = wl.group_of(b)
                 if lead[b]:
@@ -115,8 +125,7 @@ class DecodeSession:
             for b in range(B):
                 if not lead[b]:
                     src = leader_of[wl.group_of(b)]
-                    for t in (self.cache.ring_k, self.cache.ring_v, self.cache.ring_ks,
-                              self.cache.ring_vs):
+                    for t in rings:
                         t[b].copy_(t[src])
         # 3. every sequence appends its own context up to position L0 - 2
         rows_k, rows_v = [], []
@@ -145,8 +154,8 @@ class DecodeSession:
 
     # ------------------------------------------------------------------ steps
     def append_step(self, s: int = 0, stream=None):
-        kv4.quantize_append(self.cache, self.batch(self.step_lens[s]), self.step_k[s],
-                            self.step_v[s], None, self.err, stream=stream)
+        self._append(self.batch(self.step_lens[s]), self.step_k[s], self.step_v[s], None,
+                     stream=stream)
 
     def attention_step(self, s: int = 0, out=None, out_f32=None, lse=None, stream=None):
         kv4.decode_attention(self.cache, self.batch(self.step_lens[s]), self.q[s],
@@ -161,3 +170,28 @@ class DecodeSession:
         flag = int(self.err.item())
         if flag:
             raise kv4.KV4Error(f"device error flag {flag}: {kv4.decode_err(flag)}")
+
+
+class BaselineSession(DecodeSession):
+    """The same decode batch over a comparison cache: BF16 (kv4.BASELINE_BF16) or all-INT8
+    (kv4.BASELINE_KV8) pages, no protected set. Built and stepped like DecodeSession, with
+    the library's baseline append and attention calls."""
+
+    def __init__(self, wl: Workload, fmt: int, **kw):
+        self.fmt = fmt
+        super().__init__(wl, **kw)
+
+    def _allocate_cache(self):
+        return kv4.allocate_baseline_cache(self.fmt, self.cfg, self.paging.num_pages,
+                                           device=self.device)
+
+    def _workspace_size(self, num_seqs, max_len):
+        return kv4.baseline_workspace_size(self.cfg, num_seqs, max_len)
+
+    def _append(self, batch, k, v, indptr, stream=None):
+        kv4.baseline_append(self.cache, batch, k, v, indptr, self.err, stream=stream)
+
+    def attention_step(self, s: int = 0, out=None, out_f32=None, lse=None, stream=None):
+        kv4.baseline_decode_attention(self.cache, self.batch(self.step_lens[s]), self.q[s],
+                                      self.out if out is None else out, self.workspace,
+                                      out_f32, lse, self.err, stream=stream)

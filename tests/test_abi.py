@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(kv4):
 
 def test_status_strings_and_version(kv4):
     lib = kv4._lib
-    assert lib.kv4_version() == 100
+    assert lib.kv4_version() == 200
     assert lib.kv4_status_string(0) == b"ok"
     assert b"144" in lib.kv4_status_string(-3)
     assert lib.kv4_status_string(-99) == b"unknown status"
@@ -147,4 +147,28 @@ def test_workspace_too_small_is_reported(kv4):
                                        ctypes.byref(batch), ctypes.c_void_p(1 << 20),
                                        ctypes.c_void_p(1 << 20), None, None,
                                        ctypes.c_void_p(1 << 20), need - 256, None, None)
+    assert st == -4
+
+
+def test_baseline_argument_checks(kv4):
+    lib = kv4._lib
+    c = _cfg(kv4)
+    none_prot = _cfg(kv4, num_sinks=0, num_recent=0)
+    # the baselines ignore the protected set: same workspace as KV4-RL without one
+    assert kv4.baseline_workspace_size(c, 64, 2048) == kv4.workspace_size(none_prot, 64, 2048)
+    pool = kv4.PagedPool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
+    batch = kv4.Batch(1 << 20, 64, 1 << 20, 0, 0, 2, 1000)
+    call = lambda fmt, p=pool: lib.kv4_baseline_decode_attention(
+        fmt, ctypes.byref(c), ctypes.byref(p), ctypes.byref(batch), ctypes.c_void_p(1 << 20),
+        ctypes.c_void_p(1 << 20), None, None, ctypes.c_void_p(1 << 20), 1 << 30, None, None)
+    assert call(3) == -1 and call(0) == -1                # unknown format
+    no_scales = kv4.PagedPool(1 << 20, 1 << 20, 0, 0, 10)
+    assert call(kv4.BASELINE_KV8, no_scales) == -1        # KV8 needs its scales
+    misaligned = kv4.PagedPool((1 << 20) + 8, 1 << 20, 0, 0, 10)
+    assert call(kv4.BASELINE_BF16, misaligned) == -1
+    # too small a workspace is reported before anything is launched
+    st = lib.kv4_baseline_decode_attention(
+        kv4.BASELINE_BF16, ctypes.byref(c), ctypes.byref(pool), ctypes.byref(batch),
+        ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 20), None, None,
+        ctypes.c_void_p(1 << 20), 256, None, None)
     assert st == -4
