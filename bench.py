@@ -41,19 +41,42 @@ UNIT = "tokens*kv_heads/s"
 # workload accounting (host arithmetic on lengths only)
 # ----------------------------------------------------------------------------
 
+DTYPE = {"kv4": "f16-mma/f32-acc, int4/int8 codes",
+         "kv8": "f16-mma/f32-acc, int8 codes (comparison cache)",
+         "bf16": "bf16-mma/f32-acc, bf16 cache (comparison cache)"}
+CALL = {"kv4": "kv4_decode_attention", "kv8": "kv4_baseline_decode_attention(KV8)",
+        "bf16": "kv4_baseline_decode_attention(BF16)"}
+
+
 def units_per_step(wl, lens) -> int:
     """Context tokens x KV heads attended in one step."""
     return int(np.asarray(lens, dtype=np.int64).sum()) * wl.num_kv_heads
 
 
-def attention_bytes(wl, lens):
+def attention_bytes(wl, lens, cache="kv4"):
     """Algorithmic HBM bytes of one attention call: (unique, logical).
 
     Per token and KV head: 160 B when read from INT4 (64 B K codes + 16 B K params +
     the same for V), 260 B when read from INT8 (128 B codes + 2 B scale, K and V).
     Plus the query read and the output write (bf16). `unique` counts a group's shared
-    prompt pages and shared sink set once; `logical` counts them per sequence."""
+    prompt pages and shared sink set once; `logical` counts them per sequence.
+    Comparison caches: 512 B per token and head for BF16, 260 B for KV8, at every
+    position; shared prompt positions counted once in `unique`."""
     lens = np.asarray(lens, dtype=np.int64)
+    if cache in ("bf16", "kv8"):
+        per = 512 if cache == "bf16" else 260
+        H = wl.num_kv_heads
+        logical = int(lens.sum()) * per * H
+        io = lens.size * wl.num_q_heads * wl.head_dim * 2 * 2
+        unique = logical
+        if wl.shared_prefix:
+            shared = np.minimum(wl.prompt_len, lens)
+            dup = 0
+            for g in range((lens.size + wl.group_seqs - 1) // wl.group_seqs):
+                sl = slice(g * wl.group_seqs, (g + 1) * wl.group_seqs)
+                dup += int(shared[sl].min()) * per * (lens[sl].size - 1)
+            unique = logical - dup * H
+        return int(unique + io), int(logical + io)
     S, R, H = wl.num_sinks, wl.num_recent, wl.num_kv_heads
     prot = np.minimum(lens, S + R)
     int4 = np.maximum(0, lens - S - R)
@@ -73,6 +96,51 @@ def attention_bytes(wl, lens):
             dup += (shared_int4[sl].min() * 160 + shared_sink[sl].min() * 260) * (n - 1)
         unique = logical - dup * H
     return int(unique + io), int(logical + io)
+
+
+def time_prefill(sess, wl, dev, max_rows=1 << 20, reps=5):
+    """Bulk prefill through the append call: the context rows [0, L-1) of the first
+    sequences (up to max_rows rows) re-appended in one CSR call (the cache ends as it
+    was). Returns a dict with rows, mean ms per call and algorithmic GB/s (read bf16 K/V,
+    write the INT4 records and the INT8 copies of protected positions)."""
+    import torch
+    from quantized_kv_cache_kv4_b200.workload import seq_kv
+    B, H = wl.num_seqs, wl.num_kv_heads
+    L0 = wl.seq_lens.astype(np.int64)
+    ks, vs, counts, n = [], [], np.zeros(B, np.int64), 0
+    for b in range(B):
+        if n >= max_rows:
+            break
+        m = int(L0[b]) - 1
+        k, v = seq_kv(wl, b, m, sess.layer, dev)
+        ks.append(k); vs.append(v)
+        counts[b] = m
+        n += m
+    k, v = torch.cat(ks), torch.cat(vs)
+    del ks, vs
+    indptr = np.zeros(B + 1, dtype=np.int32)
+    indptr[1:] = np.cumsum(counts)
+    lens = torch.as_tensor(np.where(counts > 0, L0 - 1, 0).astype(np.int32), device=dev)
+    batch = sess.batch(lens)
+    ip = torch.as_tensor(indptr, device=dev)
+    S, R = wl.num_sinks, wl.num_recent
+    prot = sum(min(int(c), S + R) for c in counts if c > 0)
+    nbytes = n * H * (2 * 2 * wl.head_dim + 160) + prot * H * 260
+    if getattr(sess, "fmt", None) is not None:  # comparison cache: bf16 or int8 copy
+        per = 512 if sess.fmt == 1 else 260
+        nbytes = n * H * (2 * 2 * wl.head_dim + per)
+    sess.append(batch, k, v, ip)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        sess.append(batch, k, v, ip)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sess.check_err()
+    ms = e0.elapsed_time(e1) / reps
+    return {"rows": int(n), "ms": ms, "gbs": nbytes / (ms / 1000.0) / 1e9,
+            "bytes_per_call": int(nbytes)}
 
 
 def append_bytes(wl) -> int:
@@ -140,10 +208,10 @@ class ClockSampler:
 # CPU oracle timing (reference arm and cpu_baseline)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(wl, budget_s: float, start_seq: int = 0):
-    """Time the oracle's decode output (quantise -> dequantise -> softmax attention) on
-    consecutive sequences of the workload until `budget_s` of CPU time is used.
-    Returns (units processed, seconds, description, threads)."""
+def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4"):
+    """Time the oracle's decode output (quantise -> dequantise -> softmax attention; for a
+    comparison cache its BF16 / KV8 reference) on consecutive sequences of the workload
+    until `budget_s` of CPU time is used. Returns (units, seconds, description, threads)."""
     import torch
     from oracle import kv4_oracle as O
     from quantized_kv_cache_kv4_b200.workload import queries, seq_kv
@@ -161,26 +229,32 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0):
         k, v = seq_kv(wl, bb, L, 0, "cpu")
         k, v = k.float().numpy(), v.float().numpy()
         t0 = time.perf_counter()
-        O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent)
+        if cache == "bf16":
+            O.decode_reference_bf16(q_all[bb], k, v)
+        elif cache == "kv8":
+            O.decode_reference_kv8(q_all[bb], k, v)
+        else:
+            O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent)
         spent += time.perf_counter() - t0
         units += L * wl.num_kv_heads
         seqs.append(bb)
         b += 1
-    desc = (f"oracle decode_reference (fp64 numpy: quantise every position, dequantise, "
+    fn = {"bf16": "decode_reference_bf16", "kv8": "decode_reference_kv8"}.get(
+        cache, "decode_reference")
+    desc = (f"oracle {fn} (fp64 numpy: quantise every position, dequantise, "
             f"softmax attention) on {len(seqs)} sequence(s) of the workload "
             f"({units // wl.num_kv_heads} context tokens)")
     return units, spent, desc, threads
 
 
 def run_reference(args, rank, world):
-    from quantized_kv_cache_kv4_b200.workload import make_workload
     if rank != 0:
         return
-    wl = make_workload(args.workload)
+    wl = rank_workload(args.workload, 0, args.sinks, args.recent)
     total_units, total_s, descs, threads = 0, 0.0, [], 1
     per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
-        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3)
+        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3, cache=args.cache)
         if s >= args.warmup:
             total_units += u
             total_s += t
@@ -191,7 +265,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * total_s / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, **wl.describe()},
+        "config": {"workload": wl.name, **wl.describe(), "cache": args.cache},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": descs[0] if descs else ""},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -265,7 +339,7 @@ def run_gpu(args, rank, world, local_rank):
     from quantized_kv_cache_kv4_b200 import build
     build.build()
     from quantized_kv_cache_kv4_b200 import kv4
-    from quantized_kv_cache_kv4_b200.session import DecodeSession
+    from quantized_kv_cache_kv4_b200.session import BaselineSession, DecodeSession
     from quantized_kv_cache_kv4_b200.host_io import HostStepPipeline
 
     torch.cuda.set_device(local_rank)
@@ -278,9 +352,14 @@ def run_gpu(args, rank, world, local_rank):
     wl = rank_workload(args.workload, rank, args.sinks, args.recent)
     W, K = args.warmup, args.steps
     # one session per layer (same lengths and paging, own data); they share a workspace
-    sess = DecodeSession(wl, steps=W + K, device=dev)
-    layers = [sess] + [DecodeSession(wl, layer=li, steps=W + K, device=dev,
-                                     workspace=sess.workspace)
+    if args.cache == "kv4":
+        make_session = DecodeSession
+    else:
+        fmt = kv4.BASELINE_BF16 if args.cache == "bf16" else kv4.BASELINE_KV8
+        make_session = lambda *a, **kw: BaselineSession(*a, fmt=fmt, **kw)
+    sess = make_session(wl, steps=W + K, device=dev)
+    layers = [sess] + [make_session(wl, layer=li, steps=W + K, device=dev,
+                                    workspace=sess.workspace)
                        for li in range(1, wl.num_layers)]
     nl = len(layers)
     stream = torch.cuda.current_stream(dev)
@@ -331,7 +410,20 @@ def run_gpu(args, rank, world, local_rank):
     # graphs: each step's append and attention calls captured once per layer (outside the
     # timed region) and replayed; the same kernels on the same per-step inputs
     g_app, g_att = [], []
-    if args.launch == "graph":
+    if args.launch == "graph-step":
+        # one graph per step: the append and attention calls of every layer
+        for s in steps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for ls in layers:
+                    ls.append_step(s)
+                    ls.attention_step(s)
+            g_app.append(g)
+        with ClockSampler(local_rank) as clocks:
+            ms, _ = timed(lambda i, s, li: g_app[i].replay() if li == 0 else None,
+                          lambda i, s, li: None)
+        att_ms = att_eager  # calls inside one graph are not timed one by one
+    elif args.launch == "graph":
         for s in steps:
             for ls in layers:
                 g = torch.cuda.CUDAGraph()
@@ -353,7 +445,7 @@ def run_gpu(args, rank, world, local_rank):
     ms_eager_max, _ = combine_ranks(ms_eager, 0, world, dev)
 
     # ---- roofline of the attention call (plan + split-K attention + merge) ----
-    uniq = [attention_bytes(wl, L0 + s) for s in range(W, W + K)]
+    uniq = [attention_bytes(wl, L0 + s, args.cache) for s in range(W, W + K)]
     mean_att_s = statistics.mean(att_ms) / 1000.0
     achieved = statistics.mean(u for u, _ in uniq) / mean_att_s / 1e9
     peak, peak_kind = load_peaks()
@@ -380,9 +472,11 @@ def run_gpu(args, rank, world, local_rank):
     e2e_ms, _ = combine_ranks(e0.elapsed_time(e1), 0, world, dev)
     e2e_value = units_all / (e2e_ms / 1000.0)
 
+    prefill = time_prefill(sess, wl, dev) if args.prefill else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget)
+        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget, cache=args.cache)
         cpu = {"value": u / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": desc}
 
@@ -392,24 +486,28 @@ def run_gpu(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc, int4/int8 codes",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[args.cache],
             "data": "synthetic",
             "config": {"workload": wl.name, **wl.describe(),
                        "l2": "inputs larger than L2: the cache read per step is "
                              f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
+                       "cache": args.cache,
                        "parallelism": f"dp{world} (independent replica batches)",
-                       "launch": ("cuda graph per call (each layer's append and attention "
-                                  "call of every step)" if args.launch == "graph" else "eager")},
+                       "launch": {"graph": "cuda graph per call (each layer's append and "
+                                           "attention call of every step)",
+                                  "graph-step": "one cuda graph per step (all calls of all "
+                                                "layers); attention call times from the eager run",
+                                  "eager": "eager"}[args.launch]},
             "attention_ms": statistics.mean(att_ms),
             "eager": {"value": units_all / (ms_eager_max / 1000.0),
                       "ms_per_step": ms_eager_max / K,
                       "attention_ms": statistics.mean(att_eager)},
             "attention_gbs_unique": ub / mean_att_s / 1e9,
             "attention_gbs_logical": lb / mean_att_s / 1e9,
-            "roofline": {"kernel": "kv4_decode_attention (plan + attention + merge launches)",
+            "roofline": {"kernel": CALL[args.cache] + " (plan + attention + merge launches)",
                          "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": recorded_traffic(wl.name)},
+                         "traffic": recorded_traffic(wl.name) if args.cache == "kv4" else None},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
@@ -417,6 +515,8 @@ def run_gpu(args, rank, world, local_rank):
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
+        if prefill is not None:
+            line["prefill"] = {**prefill, "peak_gbs": peak, "frac": prefill["gbs"] / peak}
         print(json.dumps(line), flush=True)
     del g_app, g_att, layers
     if world > 1:
@@ -432,9 +532,13 @@ def main(argv=None):
     ap.add_argument("--workload", default="rollout")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cache", default="kv4", choices=["kv4", "kv8", "bf16"],
+                    help="KV4-RL cache (default) or a comparison cache: all-INT8 or BF16")
     ap.add_argument("--sinks", type=int, default=None, help="override S (protection sweep)")
     ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
-    ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
+    ap.add_argument("--prefill", action="store_true",
+                    help="also time a bulk prefill (one CSR append call of ~1M rows)")
+    ap.add_argument("--launch", default="graph", choices=["graph", "graph-step", "eager"],
                     help="timed steps replayed from CUDA graphs (default) or launched eagerly")
     args = ap.parse_args(argv)
     rank = int(os.environ.get("RANK", 0))

@@ -14,31 +14,17 @@
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 
+#ifndef KV4_APPEND_ROWS
+#define KV4_APPEND_ROWS 4  // new-token rows per warp in bulk appends
+#endif
+
 namespace kv4 {
 
-__global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t *__restrict__ k_new,
-                                                     const uint16_t *__restrict__ v_new,
-                                                     const int32_t *__restrict__ new_indptr,
-                                                     int32_t total_new, int32_t *err) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+// The quantise-append of one token (sequence b, position pos of L) and kv head h; every
+// lane holds 4 dims of the token's K (kraw) and V (vraw).
+__device__ __forceinline__ void append_token(const CacheView &c, int h, int b, int pos, int L,
+                                             uint2 kraw, uint2 vraw, int lane, int32_t *err) {
   const int H = c.num_kv_heads;
-  if (warp >= total_new * H) return;
-  const int row = warp / H;
-  const int h = warp - row * H;
-
-  int b, pos, L;
-  locate_new_token(c.seq_lens, c.num_seqs, new_indptr, row, b, pos, L);
-  if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
-    if (lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
-    return;
-  }
-
-  // ---- load the token's K and V (4 bf16 per lane) ----
-  const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim + 4 * lane;
-  const uint2 kraw = *reinterpret_cast<const uint2 *>(k_new + rowoff);
-  const uint2 vraw = *reinterpret_cast<const uint2 *>(v_new + rowoff);
-
   const int page = c.page_table[static_cast<size_t>(b) * c.max_pages + pos / kPage];
   const bool page_ok = page >= 0 && page < c.num_pages;
   if (!page_ok && lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
@@ -141,15 +127,87 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t
   }
 }
 
+// Largest b in [0, num_seqs) with indptr[b] <= row, by the whole warp: each round the 32
+// lanes probe 32 evenly spaced entries of the remaining range (ranges of 1M sequences
+// resolve in 4 rounds of dependent loads instead of 20).
+__device__ __forceinline__ int find_seq_warp(const int32_t *__restrict__ indptr, int num_seqs,
+                                             int row, int lane) {
+  int lo = 0, hi = num_seqs;  // indptr[lo] <= row holds throughout (indptr[0] = 0)
+  while (hi - lo > 1) {
+    const int step = (hi - lo + 31) / 32;
+    const int idx = lo + lane * step;
+    const bool le = idx < hi && indptr[idx] <= row;
+    const int k = max(__popc(__ballot_sync(0xffffffffu, le)) - 1, 0);
+    lo += k * step;
+    hi = min(hi, lo + step);
+  }
+  return lo;
+}
+
+// One warp per (block of T consecutive new-token rows, kv head); the loads of all T rows
+// are issued before the first is quantised. T = 1 for decode steps (one row per sequence).
+template <int T>
+__global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t *__restrict__ k_new,
+                                                     const uint16_t *__restrict__ v_new,
+                                                     const int32_t *__restrict__ new_indptr,
+                                                     int32_t total_new, int32_t *err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int H = c.num_kv_heads;
+  const int blocks = (total_new + T - 1) / T;
+  if (warp >= blocks * H) return;
+  const int h = warp % H;
+  const int r0 = (warp / H) * T;
+  uint2 kr[T], vr[T];
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int row = r0 + t;
+    if (row < total_new) {
+      const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim + 4 * lane;
+      kr[t] = *reinterpret_cast<const uint2 *>(k_new + rowoff);
+      vr[t] = *reinterpret_cast<const uint2 *>(v_new + rowoff);
+    }
+  }
+  int b = new_indptr ? find_seq_warp(new_indptr, c.num_seqs, r0, lane) : r0;
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int row = r0 + t;
+    if (row >= total_new) break;
+    int pos, L;
+    if (new_indptr == nullptr) {
+      b = row;
+      L = c.seq_lens[b];
+      pos = L - 1;
+    } else {
+      while (b + 1 < c.num_seqs && new_indptr[b + 1] <= row) ++b;  // next sequence's rows
+      const int n = new_indptr[b + 1] - new_indptr[b];
+      const int i = row - new_indptr[b];
+      L = c.seq_lens[b];
+      pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
+    }
+    if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
+      if (lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
+      continue;
+    }
+    append_token(c, h, b, pos, L, kr[t], vr[t], lane, err);
+  }
+}
+
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
                           const int32_t *new_indptr, int32_t total_new, int32_t *err_flag,
                           cudaStream_t s) {
   if (total_new == 0) return cudaSuccess;
-  const long long warps = static_cast<long long>(total_new) * c.num_kv_heads;
   const int threads = 256;
-  const long long blocks = (warps * 32 + threads - 1) / threads;
-  append_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(c, k_new, v_new, new_indptr,
-                                                                  total_new, err_flag);
+  // bulk appends (prefill): KV4_APPEND_ROWS rows per warp; decode-sized appends: one
+  constexpr int TB = KV4_APPEND_ROWS;
+  const bool bulk = new_indptr != nullptr && total_new >= TB * 148 * 64;
+  const int T = bulk ? TB : 1;
+  const long long warps = static_cast<long long>((total_new + T - 1) / T) * c.num_kv_heads;
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + threads - 1) / threads);
+  if (bulk)
+    append_kernel<TB><<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
+  else
+    append_kernel<1><<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
   return cudaGetLastError();
 }
 

@@ -67,8 +67,14 @@ class DecodeSession:
     def _workspace_size(self, num_seqs, max_len):
         return kv4.workspace_size(self.cfg, num_seqs, max_len)
 
-    def _append(self, batch, k, v, indptr, stream=None):
+    def append(self, batch, k, v, indptr=None, stream=None):
+        """Append rows k, v (CSR by indptr, None = one per sequence) into this cache."""
         kv4.quantize_append(self.cache, batch, k, v, indptr, self.err, stream=stream)
+
+    def attend(self, batch, q, out, out_f32=None, lse=None, stream=None):
+        """Decode attention of queries q over this cache."""
+        kv4.decode_attention(self.cache, batch, q, out, self.workspace, out_f32, lse,
+                             self.err, stream=stream)
 
     def batch(self, lens: torch.Tensor) -> kv4.BatchTensors:
         return kv4.BatchTensors(self.page_table, lens, self.sink_idx, self.ring_idx,
@@ -86,7 +92,7 @@ class DecodeSession:
         b = kv4.BatchTensors(self.page_table if page_table is None else page_table,
                              torch.as_tensor(lens_after.astype(np.int32), device=dev),
                              self.sink_idx, self.ring_idx, self.max_len)
-        self._append(b, k, v, torch.as_tensor(indptr, device=dev))
+        self.append(b, k, v, torch.as_tensor(indptr, device=dev))
 
     def _gen(self, b):
         end = int(self.L0[b]) + self.steps
@@ -154,13 +160,12 @@ class DecodeSession:
 
     # ------------------------------------------------------------------ steps
     def append_step(self, s: int = 0, stream=None):
-        self._append(self.batch(self.step_lens[s]), self.step_k[s], self.step_v[s], None,
-                     stream=stream)
+        self.append(self.batch(self.step_lens[s]), self.step_k[s], self.step_v[s], None,
+                    stream=stream)
 
     def attention_step(self, s: int = 0, out=None, out_f32=None, lse=None, stream=None):
-        kv4.decode_attention(self.cache, self.batch(self.step_lens[s]), self.q[s],
-                             self.out if out is None else out, self.workspace, out_f32, lse,
-                             self.err, stream=stream)
+        self.attend(self.batch(self.step_lens[s]), self.q[s], self.out if out is None else out,
+                    out_f32, lse, stream=stream)
 
     def step(self, s: int = 0, **kw):
         self.append_step(s, stream=kw.get("stream"))
@@ -188,10 +193,9 @@ class BaselineSession(DecodeSession):
     def _workspace_size(self, num_seqs, max_len):
         return kv4.baseline_workspace_size(self.cfg, num_seqs, max_len)
 
-    def _append(self, batch, k, v, indptr, stream=None):
+    def append(self, batch, k, v, indptr=None, stream=None):
         kv4.baseline_append(self.cache, batch, k, v, indptr, self.err, stream=stream)
 
-    def attention_step(self, s: int = 0, out=None, out_f32=None, lse=None, stream=None):
-        kv4.baseline_decode_attention(self.cache, self.batch(self.step_lens[s]), self.q[s],
-                                      self.out if out is None else out, self.workspace,
-                                      out_f32, lse, self.err, stream=stream)
+    def attend(self, batch, q, out, out_f32=None, lse=None, stream=None):
+        kv4.baseline_decode_attention(self.cache, batch, q, out, self.workspace, out_f32, lse,
+                                      self.err, stream=stream)
