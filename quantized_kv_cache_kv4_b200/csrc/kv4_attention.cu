@@ -19,8 +19,9 @@
 //                  QK^T  integer MMA (m16n8k32): K codes as bytes times the query in
 //                        15-bit fixed point split into a signed high and an unsigned low
 //                        byte, exact int32 dot products;
-//                  PV    fp16 MMA (m16n8k16, fp32 accumulate): V codes converted exactly
-//                        by the fp8 conversion, P' = p * vscale rounded once to fp16.
+//                  PV    fp16 MMA (m16n8k16, fp32 accumulate): V codes masked into fp16
+//                        subnormals (exact, no conversion), P' = p * vscale rounded once
+//                        to fp16.
 //                With G <= 4 query heads per kv head one warp serves two kv heads: the MMA
 //                N dimension (8) holds head A's queries in columns 0-3 and head B's in
 //                columns 4-7 (zeros in the other half of each B operand), so every lane's
@@ -993,8 +994,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           uint32_t vl[4], vh[4];
-          nib_pairs_v(vw[hs][2 * gg], vl);
-          nib_pairs_v(vw[hs][2 * gg + 1], vh);
+          nib_pairs_v_sub(vw[hs][2 * gg], vl);
+          nib_pairs_v_sub(vw[hs][2 * gg + 1], vh);
           const uint32_t *pb = x.ptile + ((hs * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
           const uint32_t b01 = pb[0], b23 = pb[4];
           mma_f16(o[g][0], vl[0], vl[1], vh[0], vh[1], b01, b23);
@@ -1026,11 +1027,11 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
         float *rr = rec + j * kRecordFloats;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          // V codes may have entered the MMA scaled by 2^-9
+          // rows gid (dims +0, +2) and gid+8 (dims +1, +3) carry their code scale
           const float4 v = make_float4(fmaf(o[g][0][e], kUnscaleV, mt[g][e]),
-                                       fmaf(o[g][0][2 + e], kUnscaleV, mt[g][e]),
+                                       fmaf(o[g][0][2 + e], kUnscaleV1, mt[g][e]),
                                        fmaf(o[g][1][e], kUnscaleV, mt[g][e]),
-                                       fmaf(o[g][1][2 + e], kUnscaleV, mt[g][e]));
+                                       fmaf(o[g][1][2 + e], kUnscaleV1, mt[g][e]));
           *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
         }
         if (gid == 0) {

@@ -27,10 +27,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegBig = -1.0e30f;  // running-max start: finite, so e^(m_old-m_new) is 0 not NaN
 constexpr float kScaleLog2 = kLog2e * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
-// V codes enter the PV product through the fp8 conversion: a byte b in 0..15 read as
-// e4m3 is exactly b * 2^-9, so the products are scaled by 2^-9 and the 2^9 is applied
-// once to the output.
-constexpr float kUnscaleV = kCvtUnscale;
+// V codes enter the PV product as fp16 subnormals (see nib_pairs_v_sub): code c of an
+// even output row is c * 2^-24, of an odd one 16c * 2^-24; the scales are undone on the
+// output.
+constexpr float kUnscaleV = kSubUnscale;     // C rows gid (dims 32g+4gid+2t)
+constexpr float kUnscaleV1 = kSubUnscale16;  // C rows gid+8 (dims 32g+4gid+2t+1)
 
 // INT8 stage: K codes | V codes | K scales | V scales
 constexpr int kOffVc8 = 2048, kOffKs8 = 4096, kOffVs8 = 4128, kInt8Bytes = 4160;

@@ -174,29 +174,21 @@ __device__ __forceinline__ uint32_t h2_sub(uint32_t x, uint32_t y) {
 
 constexpr uint32_t kMagic1152x2 = 0x64806480u;  // (1152.0, 1152.0)
 
-// ---------------------------------------------------------------------------
-// nibble -> fp16 through the fp8 conversion: a byte b in 0..15 read as e4m3 is exactly
-// b * 2^-9 (subnormals 0..7 and the first normal binade 8..15 are evenly spaced), so
-// masking the nibbles into bytes and converting two bytes at a time gives the codes
-// exactly, scaled by 2^-9; the scale is applied once after the dot products.
-// ---------------------------------------------------------------------------
-constexpr float kCvtUnscale = 512.0f;  // 2^9
-
-// Both byte pairs of a word: lo = bytes (0, 1), hi = bytes (2, 3).
-__device__ __forceinline__ void cvt_e4m3x2x2(uint32_t four_bytes, uint32_t &lo, uint32_t &hi) {
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(four_bytes));
-}
-
 // V word from a transposed ldmatrix (token t0's nibbles d0..d3 in bits 0-15, token t1's
-// in bits 16-31): p[k] = (t0 dim k, t1 dim k), scaled by 2^-9.
-__device__ __forceinline__ void nib_pairs_v(uint32_t x, uint32_t (&p)[4]) {
-  uint32_t y;
-  asm("prmt.b32 %0, %1, %1, 0x3120;" : "=r"(y) : "r"(x));  // bytes t0(d0d1) t1(d0d1) t0(d2d3) t1(d2d3)
-  cvt_e4m3x2x2(y & 0x0F0F0F0Fu, p[0], p[2]);
-  cvt_e4m3x2x2((y >> 4) & 0x0F0F0F0Fu, p[1], p[3]);
+// in bits 16-31) as fp16 subnormals, without any conversion: a 16-bit half holding a
+// nibble c in bits 0-3 (exponent field 0) is exactly c * 2^-24, one in bits 4-7 exactly
+// 16c * 2^-24. So p[k] = (t0 dim k, t1 dim k) is a mask for k = 0, 1 and a shift and a
+// mask for k = 2, 3; dims 1 and 3 carry an extra factor 16. The products with P' are
+// exact in the fp32 accumulators; the factors 2^24 (dims 0, 2) and 2^20 (dims 1, 3) are
+// applied once to the output.
+constexpr float kSubUnscale = 16777216.0f;  // 2^24
+constexpr float kSubUnscale16 = 1048576.0f;  // 2^20
+__device__ __forceinline__ void nib_pairs_v_sub(uint32_t x, uint32_t (&p)[4]) {
+  p[0] = x & 0x000F000Fu;
+  p[1] = x & 0x00F000F0u;
+  const uint32_t y = x >> 8;
+  p[2] = y & 0x000F000Fu;
+  p[3] = y & 0x00F000F0u;
 }
 
 // ---------------------------------------------------------------------------
