@@ -155,14 +155,33 @@ def ring_slot(pos: int, R: int) -> int:
 # attention
 # ----------------------------------------------------------------------------
 
-def effective_kv(k: np.ndarray, v: np.ndarray, S: int, R: int):
+def int4_source(x: np.ndarray, reading: str = "A") -> np.ndarray:
+    """The values a position's INT4 copy is quantised from.
+
+    Reading A (the one built by default): the bf16 input itself -- "keeps the whole
+    context in paged INT4" (ai4snews summary, "Interpretation" para. 3), so every position
+    is written to INT4 when it is appended.  Reading B: the position's INT8 copy,
+    dequantised -- the INT4 copy is made when the position is demoted out of the recent
+    window, from what the INT8 side cache holds (aimodeling article, "INT4 as the base,
+    INT8 insurance for critical positions").  code * scale of an INT8 copy has at most 18
+    significant bits, so the float32 value below is exact."""
+    if reading == "A":
+        return x
+    if reading != "B":
+        raise ValueError(f"unknown demotion reading {reading!r}")
+    c8, s8 = quantize_int8(x)
+    return (c8.astype(np.float32) * s8.astype(np.float32)[..., None]).astype(np.float32)
+
+
+def effective_kv(k: np.ndarray, v: np.ndarray, S: int, R: int, reading: str = "A"):
     """Values the cache yields for each position: INT8 dequant where protected,
-    INT4 dequant elsewhere.  k, v: float32 (bf16 values) [L, Hkv, D] -> float64."""
+    INT4 dequant elsewhere.  k, v: float32 (bf16 values) [L, Hkv, D] -> float64.
+    reading: where the INT4 copies come from (see int4_source)."""
     L = k.shape[0]
     prot = protected_mask(L, S, R)
     out = []
     for x in (k, v):
-        c4, s4, m4 = quantize_int4(x)
+        c4, s4, m4 = quantize_int4(int4_source(x, reading))
         y = dequant_int4(c4, s4, m4)
         if prot.any():
             c8, s8 = quantize_int8(x[prot])
@@ -197,12 +216,12 @@ def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray):
     return O, lse
 
 
-def decode_reference(q, k, v, S: int, R: int):
+def decode_reference(q, k, v, S: int, R: int, reading: str = "A"):
     """KV4-RL decode output for one sequence: quantise -> dequantise -> softmax.
 
     q float32 [Hq, D]; k, v float32 [L, Hkv, D] (the whole token stream of the
     sequence including the token appended this step)."""
-    K, V = effective_kv(k, v, S, R)
+    K, V = effective_kv(k, v, S, R, reading)
     return attention(q, K, V)
 
 
@@ -287,8 +306,8 @@ def f16_bits(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float16).view(np.uint16)
 
 
-def token_records(k: np.ndarray, v: np.ndarray):
-    """Per-position stored records of a token stream.
+def token_records(k: np.ndarray, v: np.ndarray, reading: str = "A"):
+    """Per-position stored records of a token stream (INT4 copies per `reading`).
 
     Returns a dict of arrays indexed by position:
       k4, v4   uint8  [L, Hkv, 4, 16]   INT4 strips
@@ -298,7 +317,7 @@ def token_records(k: np.ndarray, v: np.ndarray):
     """
     out = {}
     for name, x in (("k", k), ("v", v)):
-        c4, s4, m4 = quantize_int4(x)
+        c4, s4, m4 = quantize_int4(int4_source(x, reading))
         out[name + "4"] = pack_int4_token(c4)
         out[name + "p"] = np.stack([f16_bits(s4), f16_bits(m4)], axis=-1)
         c8, s8 = quantize_int8(x)

@@ -459,6 +459,45 @@ def test_baseline_references_reduce_to_pinned_cases():
     assert np.max(np.abs(got - _loop_attention(q, Kd, Vd))) < 1e-12
 
 
+def test_demotion_reading_b():
+    """Reading B (INT4 copies quantised from the INT8 copy): (1) with every position
+    protected it is reading A; (2) for tokens already on their INT8 grid (x = c * s, with
+    max |c| = 127 and s an fp16 value that amax/127 reproduces) it is reading A; (3) the
+    INT4 value stays within the INT8 rounding plus the INT4 bound of the INT8 values;
+    (4) on ordinary data it differs from reading A at some positions."""
+    rng = np.random.default_rng(13)
+    L = 60
+    k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    v = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    q = _bf16(rng.normal(0, 1, (8, 128)).astype(np.float32))
+    a, _ = O.decode_reference(q, k, v, 16, 128, "A")
+    b, _ = O.decode_reference(q, k, v, 16, 128, "B")
+    assert np.array_equal(a, b)
+    # tokens on their own INT8 grid: fp16 scales s = 2^-7 m with m in [64, 127]
+    c = rng.integers(-127, 128, (40, 2, 128)).astype(np.float32)
+    c[:, :, 0] = 127.0
+    s = (rng.integers(64, 128, (40, 2)) / 128.0).astype(np.float32)
+    x = (c * s[..., None]).astype(np.float32)
+    assert np.array_equal(O.quantize_int8(x)[0], c.astype(np.int8))
+    assert np.array_equal(O.int4_source(x, "B"), x)
+    ka, _ = O.effective_kv(x, x, 0, 0, "A")
+    kb, _ = O.effective_kv(x, x, 0, 0, "B")
+    assert np.array_equal(ka, kb)
+    # bound: |x - B| <= s8 / 2 + (INT4 reconstruction bound of the INT8 values)
+    xs = _bf16(rng.normal(0, 1, (50, 2, 128)).astype(np.float32))
+    src = O.int4_source(xs, "B")
+    _, s8 = O.quantize_int8(xs)
+    c4, s4, m4 = O.quantize_int4(src)
+    y = O.dequant_int4(c4, s4, m4)
+    g = src.reshape(50, 2, 4, 32).astype(np.float64)
+    rng_g = g.max(-1) - g.min(-1)
+    b4 = np.repeat(s4.astype(np.float64) / 2 + np.abs(15 * s4.astype(np.float64) - rng_g)
+                   + np.abs(m4.astype(np.float64) - g.min(-1)), 32, axis=-1)
+    err = np.abs(xs.astype(np.float64) - y)
+    assert np.all(err <= s8.astype(np.float64)[..., None] / 2 + b4 + 1e-12)
+    assert not np.array_equal(O.quantize_int4(xs)[0], c4)
+
+
 def test_expected_pages_layout():
     rng = np.random.default_rng(11)
     L = 21
