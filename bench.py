@@ -208,7 +208,8 @@ class ClockSampler:
 # CPU oracle timing (reference arm and cpu_baseline)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4"):
+def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
+                  demotion: str = "A"):
     """Time the oracle's decode output (quantise -> dequantise -> softmax attention; for a
     comparison cache its BF16 / KV8 reference) on consecutive sequences of the workload
     until `budget_s` of CPU time is used. Returns (units, seconds, description, threads)."""
@@ -234,7 +235,7 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4"):
         elif cache == "kv8":
             O.decode_reference_kv8(q_all[bb], k, v)
         else:
-            O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent)
+            O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent, demotion)
         spent += time.perf_counter() - t0
         units += L * wl.num_kv_heads
         seqs.append(bb)
@@ -254,7 +255,8 @@ def run_reference(args, rank, world):
     total_units, total_s, descs, threads = 0, 0.0, [], 1
     per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
-        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3, cache=args.cache)
+        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3, cache=args.cache,
+                                         demotion=args.demotion)
         if s >= args.warmup:
             total_units += u
             total_s += t
@@ -350,10 +352,12 @@ def run_gpu(args, rank, world, local_rank):
                                 device_id=dev)
 
     wl = rank_workload(args.workload, rank, args.sinks, args.recent)
+    if args.demotion == "B":
+        wl.name += "-demotionB"
     W, K = args.warmup, args.steps
     # one session per layer (same lengths and paging, own data); they share a workspace
     if args.cache == "kv4":
-        make_session = DecodeSession
+        make_session = lambda *a, **kw: DecodeSession(*a, demotion=args.demotion, **kw)
     else:
         fmt = kv4.BASELINE_BF16 if args.cache == "bf16" else kv4.BASELINE_KV8
         make_session = lambda *a, **kw: BaselineSession(*a, fmt=fmt, **kw)
@@ -476,7 +480,8 @@ def run_gpu(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget, cache=args.cache)
+        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget, cache=args.cache,
+                                               demotion=args.demotion)
         cpu = {"value": u / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": desc}
 
@@ -534,6 +539,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cache", default="kv4", choices=["kv4", "kv8", "bf16"],
                     help="KV4-RL cache (default) or a comparison cache: all-INT8 or BF16")
+    ap.add_argument("--demotion", default="A", choices=["A", "B"],
+                    help="INT4 copies from the bf16 input (A) or from the INT8 copy (B)")
     ap.add_argument("--sinks", type=int, default=None, help="override S (protection sweep)")
     ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
     ap.add_argument("--prefill", action="store_true",

@@ -102,6 +102,10 @@ typedef struct {
                            per call from num_seqs and max_seq_len: 64 for large batches, down
                            to 8 when long chunks would leave the GPU's warps idle (and 64
                            whenever the workspace passed is too small for the finer split) */
+  int32_t demotion;     /* where a position's INT4 copy comes from: 0 = the bf16 input, at
+                           append (reading A, the default); 1 = the position's INT8 copy,
+                           dequantised (reading B: what demotion out of the recent window
+                           would write). Attention is the same for both. */
 } kv4_config;
 
 typedef struct {

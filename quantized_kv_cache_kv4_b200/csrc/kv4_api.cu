@@ -13,7 +13,7 @@ namespace {
 kv4_status check_config(const kv4_config *cfg) {
   if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
   if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_sinks < 0 ||
-      cfg->num_recent < 0 || cfg->chunk_pages < 0)
+      cfg->num_recent < 0 || cfg->chunk_pages < 0 || cfg->demotion < 0 || cfg->demotion > 1)
     return KV4_ERR_INVALID_ARG;
   if (cfg->head_dim != kv4::kHeadDim || cfg->page_size != kv4::kPage ||
       cfg->group_size != kv4::kGroup)
@@ -109,6 +109,7 @@ kv4_status make_view(const kv4_config *cfg, const kv4_int4_pool *pool, const kv4
   v->gqa = cfg->num_q_heads / cfg->num_kv_heads;
   v->num_sinks = S;
   v->num_recent = R;
+  v->int4_from_int8 = cfg->demotion == 1;
   return KV4_OK;
 }
 
@@ -314,6 +315,6 @@ const char *kv4_status_string(kv4_status status) {
   return "unknown status";
 }
 
-int32_t kv4_version(void) { return 200; }
+int32_t kv4_version(void) { return 300; }
 
 }  // extern "C"

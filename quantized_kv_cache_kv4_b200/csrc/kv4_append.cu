@@ -7,6 +7,10 @@
 // a fixed set of attention-sink and recent positions" (ai4snews summary,
 // "Interpretation" para. 3); INT8 side cache (aimodeling article, "INT4 as the base").
 //
+// Demotion reading B (kv4_config.demotion = 1): the INT4 copy is quantised from the
+// token's INT8 copy (code * scale) instead of its bf16 values, which is what demotion out
+// of the recent window would write; the attention reads the same regions either way.
+//
 // One warp per (new token, kv head); lane i owns dims 4i..4i+3, so an INT4 group of 32
 // dims is 8 lanes and its min/max is a 3-step shuffle reduction. The code decisions are
 // taken in IEEE fp32 (__fsub_rn / __fdiv_rn / rintf = nearest-even) so they are unique
@@ -69,6 +73,30 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
     x[2] = bf16_bits_to_f32(static_cast<uint16_t>(raw.y & 0xFFFFu));
     x[3] = bf16_bits_to_f32(static_cast<uint16_t>(raw.y >> 16));
 
+    // ---- INT8 (symmetric, per token and head): the protected copy, and in demotion
+    // reading B also the values the INT4 copy is quantised from ----
+    const bool need8 = side_k != nullptr || c.int4_from_int8;  // uniform over the warp
+    float q8[4] = {0.f, 0.f, 0.f, 0.f};
+    __half s8h = __float2half(0.f);
+    float s8 = 0.f;
+    if (need8) {
+      float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      s8h = f16_sat(__fdiv_rn(amax, 127.0f));
+      s8 = __half2float(s8h);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float qv = s8 == 0.0f ? 0.0f : rintf(__fdiv_rn(x[i], s8));
+        q8[i] = fminf(fmaxf(qv, -127.0f), 127.0f);
+      }
+    }
+    if (c.int4_from_int8) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = q8[i] * s8;  // code * fp16 scale: exact in fp32
+    }
+
     // ---- INT4: per 32-dim group (8 lanes), asymmetric, fp16 scale and min ----
     float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
     float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
@@ -103,21 +131,12 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
       }
     }
 
-    // ---- INT8 copy of a protected position: symmetric, per token and head ----
+    // ---- INT8 copy of a protected position ----
     if (side_k != nullptr) {
-      float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s8h = f16_sat(__fdiv_rn(amax, 127.0f));
-      const float s8 = __half2float(s8h);
       uint32_t word = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float q = s8 == 0.0f ? 0.0f : rintf(__fdiv_rn(x[i], s8));
-        q = fminf(fmaxf(q, -127.0f), 127.0f);
-        word |= (static_cast<uint32_t>(static_cast<int32_t>(q)) & 0xFFu) << (8 * i);
-      }
+      for (int i = 0; i < 4; ++i)
+        word |= (static_cast<uint32_t>(static_cast<int32_t>(q8[i])) & 0xFFu) << (8 * i);
       int8_t *dst = (which == 0 ? side_k : side_v) + tile_base;
       // lane i holds dims 4i..4i+3: strip i/4, byte offset 4*(i%4)
       *reinterpret_cast<uint32_t *>(dst + (lane >> 2) * (kPage * 16) + side_slot * 16 +

@@ -29,6 +29,7 @@ struct CacheView {
   int32_t num_kv_heads;
   int32_t gqa;  // query heads per kv head
   int32_t num_sinks, num_recent;
+  bool int4_from_int8;  // demotion reading B: INT4 copies quantised from the INT8 copy
 };
 
 // Workspace carve-up for one decode-attention call.

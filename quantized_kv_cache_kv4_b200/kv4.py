@@ -42,7 +42,8 @@ class Config(ctypes.Structure):
     _fields_ = [("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("group_size", ctypes.c_int32), ("num_sinks", ctypes.c_int32),
-                ("num_recent", ctypes.c_int32), ("chunk_pages", ctypes.c_int32)]
+                ("num_recent", ctypes.c_int32), ("chunk_pages", ctypes.c_int32),
+                ("demotion", ctypes.c_int32)]
 
 
 class Int4Pool(ctypes.Structure):
@@ -139,9 +140,13 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def make_config(num_q_heads, num_kv_heads, num_sinks, num_recent, chunk_pages=0) -> Config:
+DEMOTION = {"A": 0, "B": 1}  # kv4_config.demotion
+
+
+def make_config(num_q_heads, num_kv_heads, num_sinks, num_recent, chunk_pages=0,
+                demotion="A") -> Config:
     return Config(num_q_heads, num_kv_heads, HEAD_DIM, PAGE, GROUP, num_sinks, num_recent,
-                  chunk_pages)
+                  chunk_pages, DEMOTION[demotion])
 
 
 @dataclasses.dataclass

@@ -23,14 +23,16 @@ from .workload import Workload, make_paging, queries, seq_kv
 class DecodeSession:
     def __init__(self, wl: Workload, layer: int = 0, steps: int = 1, device="cuda",
                  chunk_pages: int = 0, keep_streams=(), build: bool = True,
-                 max_rows_per_call: int = 1 << 20, workspace: torch.Tensor | None = None):
+                 max_rows_per_call: int = 1 << 20, workspace: torch.Tensor | None = None,
+                 demotion: str = "A"):
         self.wl = wl
         self.layer = layer
         self.steps = steps
         self.device = torch.device(device)
         self.paging = make_paging(wl, extra_tokens=steps)
+        self.demotion = demotion
         self.cfg = kv4.make_config(wl.num_q_heads, wl.num_kv_heads, wl.num_sinks,
-                                   wl.num_recent, chunk_pages)
+                                   wl.num_recent, chunk_pages, demotion)
         self.cache = self._allocate_cache()
         B = wl.num_seqs
         self.L0 = wl.seq_lens.astype(np.int64)  # lengths after step 0's append

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(kv4):
 
 def test_status_strings_and_version(kv4):
     lib = kv4._lib
-    assert lib.kv4_version() == 200
+    assert lib.kv4_version() == 300
     assert lib.kv4_status_string(0) == b"ok"
     assert b"144" in lib.kv4_status_string(-3)
     assert lib.kv4_status_string(-99) == b"unknown status"
@@ -53,8 +53,12 @@ def test_status_strings_and_version(kv4):
 
 def _cfg(kv4, **kw):
     d = dict(num_q_heads=32, num_kv_heads=8, num_sinks=16, num_recent=128, chunk_pages=0)
+    raw_demotion = kw.pop("demotion", None)  # an int: written to the struct as is
     d.update(kw)
-    return kv4.make_config(**d)
+    c = kv4.make_config(**d)
+    if raw_demotion is not None:
+        c.demotion = raw_demotion
+    return c
 
 
 def test_workspace_size_host_only(kv4):
@@ -75,6 +79,8 @@ def test_workspace_size_host_only(kv4):
     (dict(num_q_heads=30), -2),
     (dict(num_q_heads=128, num_kv_heads=8), -2),
     (dict(chunk_pages=65), -2),
+    (dict(demotion=2), -1),
+    (dict(demotion=-1), -1),
     (dict(num_sinks=-1), -1),
 ])
 def test_config_rejected_before_launch(kv4, kw, status):

@@ -41,7 +41,8 @@ def oracle_out(sess, b, step=0):
     k, v = sess.streams[b]
     L = int(sess.L0[b]) + step
     q = sess.q[step, b].float().cpu().numpy()
-    return O.decode_reference(q, k[:L], v[:L], sess.wl.num_sinks, sess.wl.num_recent)
+    return O.decode_reference(q, k[:L], v[:L], sess.wl.num_sinks, sess.wl.num_recent,
+                              getattr(sess, "demotion", "A"))
 
 
 def run_attention(sess, step=0):
@@ -80,7 +81,7 @@ def check_cache(sess, seqs):
     for b in seqs:
         k, v = sess.streams[b]
         L = int(sess.L0[b])
-        rec = O.token_records(k[:L], v[:L])
+        rec = O.token_records(k[:L], v[:L], getattr(sess, "demotion", "A"))
         pages = O.expected_pages(rec, L, sess.paging.page_table[b])
         for pid, (ekc, ekp, evc, evp) in pages.items():
             assert np.array_equal(kc[pid], ekc), (b, pid)
@@ -151,6 +152,28 @@ def test_edge_cases(name, lens, Hq, Hkv, S, R, C):
     check_cache(sess, range(len(lens)))
     check_attention(sess, range(len(lens)))
     sess.check_err()
+
+
+@pytest.mark.parametrize("name,lens,S,R,C", [
+    ("tiny-like", [37, 150, 300, 511], 4, 32, 0),
+    ("pure-int4", [1, 17, 200], 0, 0, 0),
+    ("odd-S-R-chunk3", [23, 64, 511, 700], 7, 13, 3),
+], ids=["tiny-like", "pure-int4", "odd-S-R-chunk3"])
+def test_demotion_reading_b(name, lens, S, R, C):
+    """INT4 copies quantised from the INT8 copy: pages bit-exact against the oracle's
+    reading B, attention within the tolerance, over several decode steps."""
+    _, session, W = _mods()
+    wl = W.custom_workload(lens, num_sinks=S, num_recent=R, seed=17, outlier_channels=4,
+                           outlier_scale=8.0)
+    sess = session.DecodeSession(wl, steps=3, keep_streams=range(len(lens)), chunk_pages=C,
+                                 demotion="B")
+    for s in range(3):
+        sess.append_step(s)
+        torch.cuda.synchronize()
+        check_attention(sess, range(len(lens)), step=s)
+    sess.check_err()
+    sess.L0 = sess.L0 + 2
+    check_cache(sess, range(len(lens)))
 
 
 def test_shared_prefix_groups():
