@@ -187,6 +187,27 @@ def test_shared_prefix_groups():
     sess.check_err()
 
 
+@pytest.mark.parametrize("C", [0, 4])
+def test_pairs_sharing_prompt_pages(C):
+    """Shared-prompt batches: neighbouring sequences whose page tables map their leading
+    pages to the same physical pages, members whose recent window starts inside the
+    shared prompt, neighbours from different prompt groups, an odd batch size, and
+    decode steps on top."""
+    _, session, W = _mods()
+    lens = [900, 1000, 300, 700, 650, 180, 420, 2000, 1200]
+    # every sequence is longer than its prompt (the prompt's recent ring is forked)
+    wl = W.custom_workload(lens, num_sinks=16, num_recent=128, prompt_len=160, group_seqs=3,
+                           seed=23, outlier_channels=3, outlier_scale=10.0)
+    sess = session.DecodeSession(wl, steps=2, keep_streams=range(len(lens)), chunk_pages=C)
+    pt = sess.paging.page_table
+    assert (pt[0, :10] == pt[1, :10]).all() and (pt[2, 1] != pt[3, 1])
+    for s in range(2):
+        sess.append_step(s)
+        torch.cuda.synchronize()
+        check_attention(sess, range(len(lens)), step=s)
+    sess.check_err()
+
+
 def test_heavy_tailed_values():
     _, _, W = _mods()
     wl = W.custom_workload([300, 901], num_q_heads=32, num_kv_heads=8, num_sinks=16,
