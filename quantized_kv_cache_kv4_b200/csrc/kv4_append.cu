@@ -14,7 +14,8 @@
 // One warp per (new token, kv head); lane i owns dims 4i..4i+3, so an INT4 group of 32
 // dims is 8 lanes and its min/max is a 3-step shuffle reduction. The code decisions are
 // taken in IEEE fp32 (__fsub_rn / __fdiv_rn / rintf = nearest-even) so they are unique
-// and reproducible bit for bit.
+// and reproducible bit for bit; the quotients of the code decisions go through
+// rint_quotient (a reciprocal multiply, with the IEEE division near half-integers).
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 
@@ -86,9 +87,10 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       s8h = f16_sat(__fdiv_rn(amax, 127.0f));
       s8 = __half2float(s8h);
+      const float r8 = s8 == 0.0f ? 0.0f : __frcp_rn(s8);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float qv = s8 == 0.0f ? 0.0f : rintf(__fdiv_rn(x[i], s8));
+        const float qv = s8 == 0.0f ? 0.0f : rint_quotient(x[i], s8, r8);
         q8[i] = fminf(fmaxf(qv, -127.0f), 127.0f);
       }
     }
@@ -109,10 +111,11 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
     const __half scale_h = f16_sat(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
     const float minf = __half2float(min_h);
     const float sf = __half2float(scale_h);
+    const float rf = sf == 0.0f ? 0.0f : __frcp_rn(sf);
     uint32_t code4[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float q = sf == 0.0f ? 0.0f : rintf(__fdiv_rn(__fsub_rn(x[i], minf), sf));
+      float q = sf == 0.0f ? 0.0f : rint_quotient(__fsub_rn(x[i], minf), sf, rf);
       code4[i] = static_cast<uint32_t>(fminf(fmaxf(q, 0.0f), 15.0f));
     }
     if (page_ok) {

@@ -270,6 +270,19 @@ __device__ __forceinline__ void locate_new_token(const int32_t *__restrict__ seq
   pos = (i >= 0 && i < n) ? L - n + i : -1;
 }
 
+// rint(RN(a / b)) -- the nearest integer (ties to even) to the fp32 quotient -- for
+// quotients below 2^8 in magnitude, without an IEEE division in the common case.
+// qa = RN(a * RN(1/b)) is within 2^-22 |a/b| + ulp/2 of a/b, and RN(a/b) within ulp/2,
+// so for |a/b| < 256 the two differ by less than 2^-14. Their nearest integers can
+// differ only when qa lies within that distance of a half-integer; such rare lanes
+// take the IEEE division. rcp_b is RN(1/b), computed once per scale. b > 0.
+__device__ __forceinline__ float rint_quotient(float a, float b, float rcp_b) {
+  const float qa = a * rcp_b;
+  const float c = rintf(qa);
+  if (fabsf(qa - c) > 0.5f - 0x1p-13f) return rintf(__fdiv_rn(a, b));
+  return c;
+}
+
 __device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {
   if (flag) atomicOr(reinterpret_cast<unsigned int *>(flag), bit);
 }
