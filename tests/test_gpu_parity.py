@@ -208,6 +208,41 @@ def test_pairs_sharing_prompt_pages(C):
     sess.check_err()
 
 
+def test_code_decisions_at_exact_ties():
+    """Inputs whose code quotients are exact half-integers: INT4 positions on the grid
+    x = j/4 with group min 0 and max 7.5 (scale exactly 0.5, so (x - min)/scale = j/2),
+    protected positions on x = (2k+1)/8 with max|x| = 31.75 (INT8 scale exactly 0.25, so
+    x/scale = k + 1/2). Every tie must round to even, bit for bit with the oracle."""
+    kv4, session, W = _mods()
+    L, H = 64, 2
+    wl = W.custom_workload([L], num_q_heads=8, num_kv_heads=H, num_sinks=4, num_recent=16,
+                           seed=5)
+    sess = session.DecodeSession(wl, steps=1, build=False)
+    rng = np.random.default_rng(31)
+    streams = []
+    for _ in range(2):  # K, V
+        x = rng.integers(0, 31, (L, H, 128)).astype(np.float32) * 0.25
+        g = x.reshape(L, H, 4, 32)
+        g[..., 0] = 0.0
+        g[..., 1] = 7.5
+        prot = [t for t in range(L) if t < 4 or t >= L - 16]
+        y = (2 * rng.integers(-127, 127, (len(prot), H, 128)) + 1).astype(np.float32) / 8
+        y[:, :, 5] = 31.75
+        x[prot] = y
+        streams.append(x)
+    k, v = streams
+    sess.streams[0] = (k, v)
+    dev = torch.device("cuda")
+    to = lambda a: torch.from_numpy(a).to(torch.bfloat16).to(dev)
+    assert np.array_equal(to(k).float().cpu().numpy(), k)  # exact in bf16
+    batch = sess.batch(torch.tensor([L], dtype=torch.int32, device=dev))
+    sess.append(batch, to(k), to(v), torch.tensor([0, L], dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    sess.check_err()
+    check_cache(sess, [0])
+    check_attention(sess, [0])
+
+
 def test_heavy_tailed_values():
     _, _, W = _mods()
     wl = W.custom_workload([300, 901], num_q_heads=32, num_kv_heads=8, num_sinks=16,
