@@ -11,17 +11,22 @@
 // token's INT8 copy (code * scale) instead of its bf16 values, which is what demotion out
 // of the recent window would write; the attention reads the same regions either way.
 //
-// One warp per (new token, kv head); lane i owns dims 4i..4i+3, so an INT4 group of 32
-// dims is 8 lanes and its min/max is a 3-step shuffle reduction. The code decisions are
-// taken in IEEE fp32 (__fsub_rn / __fdiv_rn / rintf = nearest-even) so they are unique
-// and reproducible bit for bit; the quotients of the code decisions go through
-// rint_quotient (a reciprocal multiply, with the IEEE division near half-integers).
+// Two kernels, the same arithmetic:
+//   append_kernel       one warp per (new token, kv head); lane i owns dims 4i..4i+3, so an
+//                       INT4 group of 32 dims is 8 lanes and its min/max a 3-step shuffle
+//                       reduction. Used for one token per sequence (decode steps), where
+//                       the launch, not the arithmetic, sets the time.
+//   append_rows_kernel  bulk appends (CSR rows, e.g. prefill of prompts): one thread per
+//                       (new token, kv head), a warp = 32 consecutive rows of one head.
+//                       No shuffles; consecutive rows are consecutive page slots, so each
+//                       16-byte code and parameter store of the warp lands in contiguous
+//                       256-byte runs of a page block (full sectors).
+// The code decisions are taken in IEEE fp32 (subtraction, division, nearest-even
+// rounding) so they are unique and reproducible bit for bit; the quotients go through a
+// reciprocal multiply, with the IEEE division only near half-integers.
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 
-#ifndef KV4_APPEND_ROWS
-#define KV4_APPEND_ROWS 4  // new-token rows per warp in bulk appends
-#endif
 
 namespace kv4 {
 
@@ -166,9 +171,8 @@ __device__ __forceinline__ int find_seq_warp(const int32_t *__restrict__ indptr,
   return lo;
 }
 
-// One warp per (block of T consecutive new-token rows, kv head); the loads of all T rows
-// are issued before the first is quantised. T = 1 for decode steps (one row per sequence).
-template <int T>
+// One warp per (new token, kv head): the token's 256 bytes of K and of V are one
+// coalesced load per warp.
 __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t *__restrict__ k_new,
                                                      const uint16_t *__restrict__ v_new,
                                                      const int32_t *__restrict__ new_indptr,
@@ -176,43 +180,331 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int H = c.num_kv_heads;
-  const int blocks = (total_new + T - 1) / T;
-  if (warp >= blocks * H) return;
+  if (warp >= total_new * H) return;
   const int h = warp % H;
-  const int r0 = (warp / H) * T;
-  uint2 kr[T], vr[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const int row = r0 + t;
-    if (row < total_new) {
-      const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim + 4 * lane;
-      kr[t] = *reinterpret_cast<const uint2 *>(k_new + rowoff);
-      vr[t] = *reinterpret_cast<const uint2 *>(v_new + rowoff);
-    }
+  const int row = warp / H;
+  const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim + 4 * lane;
+  const uint2 kr = *reinterpret_cast<const uint2 *>(k_new + rowoff);
+  const uint2 vr = *reinterpret_cast<const uint2 *>(v_new + rowoff);
+  int b, pos, L;
+  if (new_indptr == nullptr) {
+    b = row;
+    L = c.seq_lens[b];
+    pos = L - 1;
+  } else {
+    b = find_seq_warp(new_indptr, c.num_seqs, row, lane);
+    const int n = new_indptr[b + 1] - new_indptr[b];
+    const int i = row - new_indptr[b];
+    L = c.seq_lens[b];
+    pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
   }
-  int b = new_indptr ? find_seq_warp(new_indptr, c.num_seqs, r0, lane) : r0;
+  if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
+    if (lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
+    return;
+  }
+  append_token(c, h, b, pos, L, kr, vr, lane, err);
+}
+
+// ---------------------------------------------------------------------------
+// bulk appends: one thread per (new token, kv head)
+// ---------------------------------------------------------------------------
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+constexpr float kTieBand = 0.5f - 0x1p-13f;
+
+// Nearest-even integer of qa clamped to [lo, hi] (integer bounds, |lo|, |hi| < 2^22):
+// y = clamp(qa) + 1.5*2^23 is exact up to the rounding to an integer, which the add
+// performs in round-to-nearest-even, so y's low mantissa bits hold the result (as
+// y_bits - 0x4B400000). Clamping before rounding gives the same integer as rounding
+// before clamping, the bounds being integers. `near` is raised when the clamped
+// quotient lies within 2^-13 of a half-integer, where the rounding of the reciprocal
+// product can differ from that of the IEEE quotient (see rint_quotient).
+__device__ __forceinline__ uint32_t round_clamped(float qa, float lo, float hi, bool &near) {
+  const float qc = fminf(fmaxf(qa, lo), hi);
+  const float y = __fadd_rn(qc, kRoundMagic);
+  near |= fabsf(__fsub_rn(qc, __fsub_rn(y, kRoundMagic))) > kTieBand;
+  return __float_as_uint(y);
+}
+
+// The same integer through the IEEE quotient, for the rare elements near a tie.
+__device__ __forceinline__ uint32_t round_clamped_exact(float a, float b, float lo, float hi) {
+  const float q = b == 0.0f ? 0.0f : rintf(__fdiv_rn(a, b));
+  return __float_as_uint(__fadd_rn(fminf(fmaxf(q, lo), hi), kRoundMagic));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ __nv_bfloat162 bf2(uint32_t w) {
+  return *reinterpret_cast<__nv_bfloat162 *>(&w);
+}
+
+// Byte 0 of each of four words, packed into one word (byte 0 = a's).
+__device__ __forceinline__ uint32_t low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Where one row's INT4 record and (when protected) INT8 copy go.
+struct RowDst {
+  uint8_t *codes;    // the (page, head) code block: [4 groups][16 slots][16 B]
+  uint16_t *params;  // the slot's [4 groups][scale, min]
+  int slot;
+  int8_t *side;      // INT8 tile (nullptr: not protected)
+  uint16_t *side_scale;
+  int side_slot;
+};
+
+// Staging of the rows in shared memory: per thread its K row (256 B), 16 B of padding,
+// its V row. The thread stride of 528 B (132 words = 4 mod 32) makes the 16-byte reads of
+// 8 consecutive threads fall in distinct banks.
+constexpr int kRowsThreads = 128;
+constexpr int kRowStageV = 272;
+constexpr int kRowStageStride = 528;
+constexpr int kRowsSmem = kRowsThreads * kRowStageStride;
+
+// The 16 words (dims 32g..32g+31, two per word) of group g of a staged row.
+__device__ __forceinline__ void group_words(const uint8_t *row, int g, uint32_t (&w)[16]) {
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const int row = r0 + t;
-    if (row >= total_new) break;
-    int pos, L;
-    if (new_indptr == nullptr) {
-      b = row;
-      L = c.seq_lens[b];
-      pos = L - 1;
-    } else {
-      while (b + 1 < c.num_seqs && new_indptr[b + 1] <= row) ++b;  // next sequence's rows
-      const int n = new_indptr[b + 1] - new_indptr[b];
-      const int i = row - new_indptr[b];
-      L = c.seq_lens[b];
-      pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(row + 64 * g + 16 * i);
+    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+}
+
+// INT8 codes of one group (words w), packed 4 per word: dim 4j+i of the group in byte i
+// of c8[j].
+__device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, float r8,
+                                           uint32_t (&c8)[8]) {
+  bool near = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    c8[j] = low_bytes(round_clamped(bf16_lo(w[2 * j]) * r8, -127.f, 127.f, near),
+                      round_clamped(bf16_hi(w[2 * j]) * r8, -127.f, 127.f, near),
+                      round_clamped(bf16_lo(w[2 * j + 1]) * r8, -127.f, 127.f, near),
+                      round_clamped(bf16_hi(w[2 * j + 1]) * r8, -127.f, 127.f, near));
+  if (near) {  // rare: some quotient within 2^-13 of a half-integer
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      c8[j] = low_bytes(round_clamped_exact(bf16_lo(w[2 * j]), s8, -127.f, 127.f),
+                        round_clamped_exact(bf16_hi(w[2 * j]), s8, -127.f, 127.f),
+                        round_clamped_exact(bf16_lo(w[2 * j + 1]), s8, -127.f, 127.f),
+                        round_clamped_exact(bf16_hi(w[2 * j + 1]), s8, -127.f, 127.f));
+  }
+}
+
+// Quantise one staged row (one new token and kv head, 128 bf16 values) into its INT4
+// record and, when protected, its INT8 copy. from8: demotion reading B (the INT4 copy
+// quantised from the INT8 copy). The group loop is not unrolled: the code stays small
+// enough for the instruction cache.
+__device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d, bool from8) {
+  const bool need8 = d.side != nullptr || from8;
+  float s8 = 0.f, r8 = 0.f;
+  uint16_t s8_bits = 0;
+  if (need8) {  // symmetric INT8: amax over the 128 dims (|x| of bf16 = clear the sign bit)
+    __nv_bfloat162 m2 = bf2(0u);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * i);
+      m2 = __hmax2(m2, bf2(v.x & 0x7FFF7FFFu));
+      m2 = __hmax2(m2, bf2(v.y & 0x7FFF7FFFu));
+      m2 = __hmax2(m2, bf2(v.z & 0x7FFF7FFFu));
+      m2 = __hmax2(m2, bf2(v.w & 0x7FFF7FFFu));
     }
+    const float amax = fmaxf(__low2float(m2), __high2float(m2));
+    const __half s8h = f16_sat(__fdiv_rn(amax, 127.0f));
+    s8_bits = __half_as_ushort(s8h);
+    s8 = __half2float(s8h);
+    r8 = s8 == 0.0f ? 0.0f : __frcp_rn(s8);
+  }
+  uint32_t pv[4];
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    uint32_t w[16];
+    group_words(row, g, w);
+    uint32_t c8[8];
+    if (need8) {
+      int8_group(w, s8, r8, c8);
+      if (d.side != nullptr) {  // strips 2g, 2g+1 (16 dims each) of the INT8 tile
+        int8_t *dst = d.side + 2 * g * (kPage * 16) + d.side_slot * 16;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(c8[0], c8[1], c8[2], c8[3]);
+        *reinterpret_cast<uint4 *>(dst + kPage * 16) = make_uint4(c8[4], c8[5], c8[6], c8[7]);
+      }
+    }
+    // ---- INT4 group: min/max, fp16 scale and min, codes ----
+    auto xval = [&](int k) {  // dim 32g+k of the values the INT4 copy is quantised from
+      if (from8) {  // INT8 code * fp16 scale: exact in fp32
+        const int code = static_cast<int8_t>(__byte_perm(c8[k >> 2], 0u, k & 3));
+        return static_cast<float>(code) * s8;
+      }
+      return (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
+    };
+    float mn, mx;
+    if (from8) {
+      mn = mx = xval(0);
+#pragma unroll
+      for (int k = 1; k < 32; ++k) {
+        mn = fminf(mn, xval(k));
+        mx = fmaxf(mx, xval(k));
+      }
+    } else {  // bf16 min/max are exact: pairwise on bf16x2, then the two halves
+      __nv_bfloat162 lo2 = bf2(w[0]), hi2 = lo2;
+#pragma unroll
+      for (int i = 1; i < 16; ++i) {
+        lo2 = __hmin2(lo2, bf2(w[i]));
+        hi2 = __hmax2(hi2, bf2(w[i]));
+      }
+      mn = fminf(__low2float(lo2), __high2float(lo2));
+      mx = fmaxf(__low2float(hi2), __high2float(hi2));
+    }
+    const __half min_h = f16_sat(mn);
+    const __half scale_h = f16_sat(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+    const float minf = __half2float(min_h);
+    const float sf = __half2float(scale_h);
+    const float rf = sf == 0.0f ? 0.0f : __frcp_rn(sf);  // scale 0: every code 0
+    // byte i of the group's 16 = code(2i) | code(2i+1) << 4. A rounded y's low nibble is
+    // the code and its next 4 bits are zero, so y_even + (y_odd << 4) has the byte in
+    // its low 8 bits.
+    uint32_t words[4];
+    bool near = false;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t pb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int k = 8 * j + 2 * i;
+        pb[i] = round_clamped(__fsub_rn(xval(k), minf) * rf, 0.f, 15.f, near) +
+                (round_clamped(__fsub_rn(xval(k + 1), minf) * rf, 0.f, 15.f, near) << 4);
+      }
+      words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
+    }
+    if (near) {  // rare: redo the group through the IEEE quotients
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t pb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = 8 * j + 2 * i;
+          pb[i] = round_clamped_exact(__fsub_rn(xval(k), minf), sf, 0.f, 15.f) +
+                  (round_clamped_exact(__fsub_rn(xval(k + 1), minf), sf, 0.f, 15.f) << 4);
+        }
+        words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
+      }
+    }
+    if (d.codes != nullptr)
+      *reinterpret_cast<uint4 *>(d.codes + g * (kPage * 16) + d.slot * 16) =
+          make_uint4(words[0], words[1], words[2], words[3]);
+    pv[g] = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
+            (static_cast<uint32_t>(__half_as_ushort(min_h)) << 16);
+  }
+  if (d.codes != nullptr)
+    *reinterpret_cast<uint4 *>(d.params) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+  if (d.side != nullptr) *d.side_scale = s8_bits;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// A warp = 32 consecutive CSR rows (lane = row) of one kv head; consecutive warps are
+// the heads of the same rows, so the rows' lookups hit the same L1 lines. Each thread
+// first stages its row's K and V (512 B) into shared memory with asynchronous copies,
+// then finds where the row goes while they land.
+__global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
+                                                         const uint16_t *__restrict__ k_new,
+                                                         const uint16_t *__restrict__ v_new,
+                                                         const int32_t *__restrict__ new_indptr,
+                                                         int32_t total_new, int32_t *err) {
+  extern __shared__ __align__(16) uint8_t rows_smem[];
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int H = c.num_kv_heads;
+  const int tiles = (total_new + 31) / 32;
+  if (warp >= tiles * H) return;  // whole warps
+  const int h = warp % H;
+  const int r0 = (warp / H) * 32;
+  const int row = r0 + lane;
+  bool live = row < total_new;
+
+  uint8_t *stage = rows_smem + threadIdx.x * kRowStageStride;
+  if (live) {
+    const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim;
+    const uint8_t *ks = reinterpret_cast<const uint8_t *>(k_new + rowoff);
+    const uint8_t *vs = reinterpret_cast<const uint8_t *>(v_new + rowoff);
+    const uint32_t st = static_cast<uint32_t>(__cvta_generic_to_shared(stage));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cp_async16(st + 16 * i, ks + 16 * i);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cp_async16(st + kRowStageV + 16 * i, vs + 16 * i);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  // the row's sequence: warp searches for the tile's first and last rows, then a
+  // per-lane binary search between them
+  const int b_first = find_seq_warp(new_indptr, c.num_seqs, r0, lane);
+  const int b_last = find_seq_warp(new_indptr, c.num_seqs, min(r0 + 31, total_new - 1), lane);
+  int lo = b_first, hi = b_last;  // largest b with indptr[b] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (new_indptr[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  const int b = lo;
+  int pos = -1, L = 0;
+  if (live) {
+    const int n = new_indptr[b + 1] - new_indptr[b];
+    const int i = row - new_indptr[b];
+    L = c.seq_lens[b];
+    pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
     if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
-      if (lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
-      continue;
+      set_err(err, KV4_DEVERR_SEQ_LEN);
+      live = false;
     }
-    append_token(c, h, b, pos, L, kr[t], vr[t], lane, err);
   }
+  RowDst dk{}, dv{};
+  if (live) {
+    const int page = c.page_table[static_cast<size_t>(b) * c.max_pages + pos / kPage];
+    if (page >= 0 && page < c.num_pages) {
+      const size_t blk = static_cast<size_t>(page) * H + h;
+      dk.codes = c.k_codes + blk * 4 * (kPage * 16);
+      dv.codes = c.v_codes + blk * 4 * (kPage * 16);
+      dk.params = c.k_params + (blk * kPage + pos % kPage) * 8;
+      dv.params = c.v_params + (blk * kPage + pos % kPage) * 8;
+    } else {
+      set_err(err, KV4_DEVERR_PAGE_ID);
+    }
+    dk.slot = dv.slot = pos % kPage;
+    const int S = c.num_sinks, R = c.num_recent;
+    if (pos < S) {
+      const int set = c.sink_idx ? c.sink_idx[b] : b;
+      if (set >= 0 && set < c.num_sink_sets) {
+        const size_t sh = static_cast<size_t>(set) * H + h;
+        const size_t tile = (sh * c.sink_tiles + pos / kPage) * kInt8CodeBytes;
+        const size_t sidx = sh * c.sink_tiles * kPage + pos;
+        dk.side = c.sink_k + tile; dk.side_scale = c.sink_ks + sidx;
+        dv.side = c.sink_v + tile; dv.side_scale = c.sink_vs + sidx;
+        dk.side_slot = dv.side_slot = pos % kPage;
+      } else {
+        set_err(err, KV4_DEVERR_SIDE_IDX);
+      }
+    } else if (R > 0 && pos >= L - R) {
+      const int ring = c.ring_idx ? c.ring_idx[b] : b;
+      if (ring >= 0 && ring < c.num_rings) {
+        const int rs = pos % R;
+        const size_t rh = static_cast<size_t>(ring) * H + h;
+        const size_t tile = (rh * c.ring_tiles + rs / kPage) * kInt8CodeBytes;
+        const size_t sidx = rh * c.ring_tiles * kPage + rs;
+        dk.side = c.ring_k + tile; dk.side_scale = c.ring_ks + sidx;
+        dv.side = c.ring_v + tile; dv.side_scale = c.ring_vs + sidx;
+        dk.side_slot = dv.side_slot = rs % kPage;
+      } else {
+        set_err(err, KV4_DEVERR_SIDE_IDX);
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's own copies
+  if (!live) return;
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which)
+    quantize_row(stage + which * kRowStageV, which == 0 ? dk : dv, c.int4_from_int8);
 }
 
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
@@ -220,16 +512,27 @@ cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint1
                           cudaStream_t s) {
   if (total_new == 0) return cudaSuccess;
   const int threads = 256;
-  // bulk appends (prefill): KV4_APPEND_ROWS rows per warp; decode-sized appends: one
-  constexpr int TB = KV4_APPEND_ROWS;
-  const bool bulk = new_indptr != nullptr && total_new >= TB * 148 * 64;
-  const int T = bulk ? TB : 1;
-  const long long warps = static_cast<long long>((total_new + T - 1) / T) * c.num_kv_heads;
-  const unsigned blocks = static_cast<unsigned>((warps * 32 + threads - 1) / threads);
-  if (bulk)
-    append_kernel<TB><<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
-  else
-    append_kernel<1><<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
+  if (new_indptr != nullptr) {  // CSR rows: one thread per (row, kv head)
+    static int configured_device = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev != configured_device) {
+      e = cudaFuncSetAttribute(append_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kRowsSmem);
+      if (e != cudaSuccess) return e;
+      configured_device = dev;
+    }
+    const long long warps = static_cast<long long>((total_new + 31) / 32) * c.num_kv_heads;
+    const unsigned blocks =
+        static_cast<unsigned>((warps * 32 + kRowsThreads - 1) / kRowsThreads);
+    append_rows_kernel<<<blocks, kRowsThreads, kRowsSmem, s>>>(c, k_new, v_new, new_indptr,
+                                                               total_new, err_flag);
+  } else {  // one token per sequence: one warp per (token, kv head)
+    const long long warps = static_cast<long long>(total_new) * c.num_kv_heads;
+    const unsigned blocks = static_cast<unsigned>((warps * 32 + threads - 1) / threads);
+    append_kernel<<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
+  }
   return cudaGetLastError();
 }
 
