@@ -22,8 +22,9 @@
 //                       16-byte code and parameter store of the warp lands in contiguous
 //                       256-byte runs of a page block (full sectors).
 // The code decisions are taken in IEEE fp32 (subtraction, division, nearest-even
-// rounding) so they are unique and reproducible bit for bit; the quotients go through a
-// reciprocal multiply, with the IEEE division only near half-integers.
+// rounding) so they are unique and reproducible bit for bit; the correctly rounded
+// quotients come from a reciprocal multiply and one fma correction (quotient_rn), exact
+// for the fp16 scales.
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
 
@@ -90,12 +91,12 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      s8h = f16_sat(__fdiv_rn(amax, 127.0f));
+      s8h = f16_sat(quotient_rn(amax, 127.0f, kRcp127));
       s8 = __half2float(s8h);
       const float r8 = s8 == 0.0f ? 0.0f : __frcp_rn(s8);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float qv = s8 == 0.0f ? 0.0f : rint_quotient(x[i], s8, r8);
+        const float qv = rintf(quotient_rn(x[i], s8, r8));  // r8 = 0 when s8 = 0: 0
         q8[i] = fminf(fmaxf(qv, -127.0f), 127.0f);
       }
     }
@@ -113,14 +114,14 @@ __device__ __forceinline__ void append_token(const CacheView &c, int h, int b, i
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
     const __half min_h = f16_sat(mn);
-    const __half scale_h = f16_sat(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+    const __half scale_h = f16_sat(quotient_rn(__fsub_rn(mx, mn), 15.0f, kRcp15));
     const float minf = __half2float(min_h);
     const float sf = __half2float(scale_h);
     const float rf = sf == 0.0f ? 0.0f : __frcp_rn(sf);
     uint32_t code4[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float q = sf == 0.0f ? 0.0f : rint_quotient(__fsub_rn(x[i], minf), sf, rf);
+      float q = rintf(quotient_rn(__fsub_rn(x[i], minf), sf, rf));  // rf = 0 when sf = 0: 0
       code4[i] = static_cast<uint32_t>(fminf(fmaxf(q, 0.0f), 15.0f));
     }
     if (page_ok) {
@@ -208,28 +209,18 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t
 // ---------------------------------------------------------------------------
 // bulk appends: one thread per (new token, kv head)
 // ---------------------------------------------------------------------------
+// y = v + 1.5*2^23 (|v| < 2^22) is rounded by the add to an integer in round-to-nearest-
+// even, which y's low mantissa bits then hold: y_bits - 0x4B400000 (two's complement for
+// negative integers, so the low byte of y_bits is an int8 code and the low nibble an
+// INT4 code).
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr uint32_t kRoundMagicBits = 0x4B400000u;
-constexpr float kTieBand = 0.5f - 0x1p-13f;
 
-// Nearest-even integer of qa clamped to [lo, hi] (integer bounds, |lo|, |hi| < 2^22):
-// y = clamp(qa) + 1.5*2^23 is exact up to the rounding to an integer, which the add
-// performs in round-to-nearest-even, so y's low mantissa bits hold the result (as
-// y_bits - 0x4B400000). Clamping before rounding gives the same integer as rounding
-// before clamping, the bounds being integers. `near` is raised when the clamped
-// quotient lies within 2^-13 of a half-integer, where the rounding of the reciprocal
-// product can differ from that of the IEEE quotient (see rint_quotient).
-__device__ __forceinline__ uint32_t round_clamped(float qa, float lo, float hi, bool &near) {
-  const float qc = fminf(fmaxf(qa, lo), hi);
-  const float y = __fadd_rn(qc, kRoundMagic);
-  near |= fabsf(__fsub_rn(qc, __fsub_rn(y, kRoundMagic))) > kTieBand;
-  return __float_as_uint(y);
-}
-
-// The same integer through the IEEE quotient, for the rare elements near a tie.
-__device__ __forceinline__ uint32_t round_clamped_exact(float a, float b, float lo, float hi) {
-  const float q = b == 0.0f ? 0.0f : rintf(__fdiv_rn(a, b));
-  return __float_as_uint(__fadd_rn(fminf(fmaxf(q, lo), hi), kRoundMagic));
+// rint(clamp(RN(a / b), lo, hi)) as y = result + 1.5*2^23 (see kRoundMagic); the integer
+// bounds make clamping before rounding equal to rounding before clamping.
+__device__ __forceinline__ uint32_t round_clamped(float a, float b, float y_rcp, float lo,
+                                                  float hi) {
+  const float q = fminf(fmaxf(quotient_rn(a, b, y_rcp), lo), hi);
+  return __float_as_uint(__fadd_rn(q, kRoundMagic));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -271,35 +262,95 @@ __device__ __forceinline__ void group_words(const uint8_t *row, int g, uint32_t 
   }
 }
 
-// INT8 codes of one group (words w), packed 4 per word: dim 4j+i of the group in byte i
-// of c8[j].
-__device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, float r8,
-                                           uint32_t (&c8)[8]) {
-  bool near = false;
+// ---- two fp32 lanes per instruction (sm_100 f32x2 arithmetic; each lane rounds to
+// nearest-even exactly as the scalar operation does) ----
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  return (static_cast<f32x2>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float lo_of(f32x2 v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_of(f32x2 v) {
+  return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// quotient_rn on a pair (nb = -b, y = RN(1/b) in both lanes), rounded to integers as
+// y = RN(a/b) + 1.5*2^23: callers know every quotient lies where no clamp is needed.
+__device__ __forceinline__ f32x2 round_quotient_pair(f32x2 a, f32x2 nb, f32x2 y) {
+  const f32x2 q0 = mul2(a, y);
+  const f32x2 q = fma2(fma2(q0, nb, a), y, q0);
+  return add2(q, pack2(kRoundMagic, kRoundMagic));
+}
+
+// INT8 codes of one group (words w: dims 2i, 2i+1 in word i), packed 4 per word (dim
+// 4j+i of the group in byte i of c8[j]); with FROM8 also the codes as floats (x8).
+// fast: RN(amax / s8) < 127.5, so every code lies in [-127, 127] without the clamp.
+template <bool FROM8>
+__device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, float r8, bool fast,
+                                           uint32_t (&c8)[8], float (&x8)[32]) {
+  if (fast) {
+    const f32x2 nb = pack2(-s8, -s8), yr = pack2(r8, r8);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    c8[j] = low_bytes(round_clamped(bf16_lo(w[2 * j]) * r8, -127.f, 127.f, near),
-                      round_clamped(bf16_hi(w[2 * j]) * r8, -127.f, 127.f, near),
-                      round_clamped(bf16_lo(w[2 * j + 1]) * r8, -127.f, 127.f, near),
-                      round_clamped(bf16_hi(w[2 * j + 1]) * r8, -127.f, 127.f, near));
-  if (near) {  // rare: some quotient within 2^-13 of a half-integer
+    for (int j = 0; j < 8; ++j) {
+      const f32x2 y0 =
+          round_quotient_pair(pack2(bf16_lo(w[2 * j]), bf16_hi(w[2 * j])), nb, yr);
+      const f32x2 y1 =
+          round_quotient_pair(pack2(bf16_lo(w[2 * j + 1]), bf16_hi(w[2 * j + 1])), nb, yr);
+      c8[j] = low_bytes(static_cast<uint32_t>(y0), static_cast<uint32_t>(y0 >> 32),
+                        static_cast<uint32_t>(y1), static_cast<uint32_t>(y1 >> 32));
+      if (FROM8) {
+        x8[4 * j] = lo_of(y0) - kRoundMagic;
+        x8[4 * j + 1] = hi_of(y0) - kRoundMagic;
+        x8[4 * j + 2] = lo_of(y1) - kRoundMagic;
+        x8[4 * j + 3] = hi_of(y1) - kRoundMagic;
+      }
+    }
+  } else {  // a saturated fp16 scale: clamp every code
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      c8[j] = low_bytes(round_clamped_exact(bf16_lo(w[2 * j]), s8, -127.f, 127.f),
-                        round_clamped_exact(bf16_hi(w[2 * j]), s8, -127.f, 127.f),
-                        round_clamped_exact(bf16_lo(w[2 * j + 1]), s8, -127.f, 127.f),
-                        round_clamped_exact(bf16_hi(w[2 * j + 1]), s8, -127.f, 127.f));
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t y[4] = {round_clamped(bf16_lo(w[2 * j]), s8, r8, -127.f, 127.f),
+                             round_clamped(bf16_hi(w[2 * j]), s8, r8, -127.f, 127.f),
+                             round_clamped(bf16_lo(w[2 * j + 1]), s8, r8, -127.f, 127.f),
+                             round_clamped(bf16_hi(w[2 * j + 1]), s8, r8, -127.f, 127.f)};
+      c8[j] = low_bytes(y[0], y[1], y[2], y[3]);
+      if (FROM8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x8[4 * j + i] = __uint_as_float(y[i]) - kRoundMagic;
+      }
+    }
   }
 }
 
 // Quantise one staged row (one new token and kv head, 128 bf16 values) into its INT4
-// record and, when protected, its INT8 copy. from8: demotion reading B (the INT4 copy
+// record and, when protected, its INT8 copy. FROM8: demotion reading B (the INT4 copy
 // quantised from the INT8 copy). The group loop is not unrolled: the code stays small
 // enough for the instruction cache.
-__device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d, bool from8) {
-  const bool need8 = d.side != nullptr || from8;
+template <bool FROM8>
+__device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d) {
+  const bool need8 = FROM8 || d.side != nullptr;
   float s8 = 0.f, r8 = 0.f;
   uint16_t s8_bits = 0;
+  bool fast8 = false;
   if (need8) {  // symmetric INT8: amax over the 128 dims (|x| of bf16 = clear the sign bit)
     __nv_bfloat162 m2 = bf2(0u);
 #pragma unroll
@@ -311,10 +362,11 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d
       m2 = __hmax2(m2, bf2(v.w & 0x7FFF7FFFu));
     }
     const float amax = fmaxf(__low2float(m2), __high2float(m2));
-    const __half s8h = f16_sat(__fdiv_rn(amax, 127.0f));
+    const __half s8h = f16_sat(quotient_rn(amax, 127.0f, kRcp127));
     s8_bits = __half_as_ushort(s8h);
     s8 = __half2float(s8h);
     r8 = s8 == 0.0f ? 0.0f : __frcp_rn(s8);
+    fast8 = quotient_rn(amax, s8, r8) < 127.5f;  // |x| <= amax: every quotient below it
   }
   uint32_t pv[4];
 #pragma unroll 1
@@ -322,8 +374,9 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d
     uint32_t w[16];
     group_words(row, g, w);
     uint32_t c8[8];
+    float x8[32];  // FROM8: the group's INT8 codes; the INT4 copy is quantised from x8 * s8
     if (need8) {
-      int8_group(w, s8, r8, c8);
+      int8_group<FROM8>(w, s8, r8, fast8, c8, x8);
       if (d.side != nullptr) {  // strips 2g, 2g+1 (16 dims each) of the INT8 tile
         int8_t *dst = d.side + 2 * g * (kPage * 16) + d.side_slot * 16;
         *reinterpret_cast<uint4 *>(dst) = make_uint4(c8[0], c8[1], c8[2], c8[3]);
@@ -332,14 +385,11 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d
     }
     // ---- INT4 group: min/max, fp16 scale and min, codes ----
     auto xval = [&](int k) {  // dim 32g+k of the values the INT4 copy is quantised from
-      if (from8) {  // INT8 code * fp16 scale: exact in fp32
-        const int code = static_cast<int8_t>(__byte_perm(c8[k >> 2], 0u, k & 3));
-        return static_cast<float>(code) * s8;
-      }
+      if (FROM8) return x8[k] * s8;  // INT8 code * fp16 scale: exact in fp32
       return (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
     };
     float mn, mx;
-    if (from8) {
+    if (FROM8) {
       mn = mx = xval(0);
 #pragma unroll
       for (int k = 1; k < 32; ++k) {
@@ -357,35 +407,40 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d
       mx = fmaxf(__low2float(hi2), __high2float(hi2));
     }
     const __half min_h = f16_sat(mn);
-    const __half scale_h = f16_sat(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+    const __half scale_h = f16_sat(quotient_rn(__fsub_rn(mx, mn), 15.0f, kRcp15));
     const float minf = __half2float(min_h);
     const float sf = __half2float(scale_h);
-    const float rf = sf == 0.0f ? 0.0f : __frcp_rn(sf);  // scale 0: every code 0
+    const float rf = sf == 0.0f ? 0.0f : __frcp_rn(sf);  // scale 0: every quotient 0
+    // RN(RN(x - min) / scale) is monotone in x, so the group's quotients lie between
+    // those of mn and mx; within [-1/2, 15.5) they round into [0, 15] without the clamp
+    const bool fast = quotient_rn(__fsub_rn(mn, minf), sf, rf) >= -0.5f &&
+                      quotient_rn(__fsub_rn(mx, minf), sf, rf) < 15.5f;
     // byte i of the group's 16 = code(2i) | code(2i+1) << 4. A rounded y's low nibble is
     // the code and its next 4 bits are zero, so y_even + (y_odd << 4) has the byte in
     // its low 8 bits.
     uint32_t words[4];
-    bool near = false;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t pb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int k = 8 * j + 2 * i;
-        pb[i] = round_clamped(__fsub_rn(xval(k), minf) * rf, 0.f, 15.f, near) +
-                (round_clamped(__fsub_rn(xval(k + 1), minf) * rf, 0.f, 15.f, near) << 4);
-      }
-      words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
-    }
-    if (near) {  // rare: redo the group through the IEEE quotients
+    if (fast) {
+      const f32x2 m2 = pack2(minf, minf), nb = pack2(-sf, -sf), yr = pack2(rf, rf);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t pb[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int k = 8 * j + 2 * i;
-          pb[i] = round_clamped_exact(__fsub_rn(xval(k), minf), sf, 0.f, 15.f) +
-                  (round_clamped_exact(__fsub_rn(xval(k + 1), minf), sf, 0.f, 15.f) << 4);
+          const f32x2 y = round_quotient_pair(sub2(pack2(xval(k), xval(k + 1)), m2), nb, yr);
+          pb[i] = static_cast<uint32_t>(y) + (static_cast<uint32_t>(y >> 32) << 4);
+        }
+        words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
+      }
+    } else {  // a min far from the group (|min| >> range) or a saturated scale: clamp
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t pb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = 8 * j + 2 * i;
+          pb[i] = round_clamped(__fsub_rn(xval(k), minf), sf, rf, 0.f, 15.f) +
+                  (round_clamped(__fsub_rn(xval(k + 1), minf), sf, rf, 0.f, 15.f) << 4);
         }
         words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
       }
@@ -409,6 +464,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 // the heads of the same rows, so the rows' lookups hit the same L1 lines. Each thread
 // first stages its row's K and V (512 B) into shared memory with asynchronous copies,
 // then finds where the row goes while they land.
+template <bool FROM8>
 __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
                                                          const uint16_t *__restrict__ k_new,
                                                          const uint16_t *__restrict__ v_new,
@@ -504,7 +560,7 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
   if (!live) return;
 #pragma unroll 1
   for (int which = 0; which < 2; ++which)
-    quantize_row(stage + which * kRowStageV, which == 0 ? dk : dv, c.int4_from_int8);
+    quantize_row<FROM8>(stage + which * kRowStageV, which == 0 ? dk : dv);
 }
 
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
@@ -518,16 +574,23 @@ cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint1
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev != configured_device) {
-      e = cudaFuncSetAttribute(append_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kRowsSmem);
+      e = cudaFuncSetAttribute(append_rows_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(append_rows_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
       if (e != cudaSuccess) return e;
       configured_device = dev;
     }
     const long long warps = static_cast<long long>((total_new + 31) / 32) * c.num_kv_heads;
     const unsigned blocks =
         static_cast<unsigned>((warps * 32 + kRowsThreads - 1) / kRowsThreads);
-    append_rows_kernel<<<blocks, kRowsThreads, kRowsSmem, s>>>(c, k_new, v_new, new_indptr,
-                                                               total_new, err_flag);
+    if (c.int4_from_int8)
+      append_rows_kernel<true><<<blocks, kRowsThreads, kRowsSmem, s>>>(c, k_new, v_new, new_indptr,
+                                                                       total_new, err_flag);
+    else
+      append_rows_kernel<false><<<blocks, kRowsThreads, kRowsSmem, s>>>(c, k_new, v_new, new_indptr,
+                                                                        total_new, err_flag);
   } else {  // one token per sequence: one warp per (token, kv head)
     const long long warps = static_cast<long long>(total_new) * c.num_kv_heads;
     const unsigned blocks = static_cast<unsigned>((warps * 32 + threads - 1) / threads);

@@ -75,13 +75,13 @@ __global__ void __launch_bounds__(256) baseline_append_kernel(CacheView c,
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      const __half s8h = f16_sat(__fdiv_rn(amax, 127.0f));
+      const __half s8h = f16_sat(quotient_rn(amax, 127.0f, kRcp127));
       const float s8 = __half2float(s8h);
       const float r8 = s8 == 0.0f ? 0.0f : __frcp_rn(s8);
       uint32_t word = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float qv = s8 == 0.0f ? 0.0f : rint_quotient(x[i], s8, r8);
+        float qv = rintf(quotient_rn(x[i], s8, r8));  // r8 = 0 when s8 = 0: 0
         qv = fminf(fmaxf(qv, -127.0f), 127.0f);
         word |= (static_cast<uint32_t>(static_cast<int32_t>(qv)) & 0xFFu) << (8 * i);
       }

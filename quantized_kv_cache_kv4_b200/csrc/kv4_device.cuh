@@ -270,18 +270,26 @@ __device__ __forceinline__ void locate_new_token(const int32_t *__restrict__ seq
   pos = (i >= 0 && i < n) ? L - n + i : -1;
 }
 
-// rint(RN(a / b)) -- the nearest integer (ties to even) to the fp32 quotient -- for
-// quotients below 2^8 in magnitude, without an IEEE division in the common case.
-// qa = RN(a * RN(1/b)) is within 2^-22 |a/b| + ulp/2 of a/b, and RN(a/b) within ulp/2,
-// so for |a/b| < 256 the two differ by less than 2^-14. Their nearest integers can
-// differ only when qa lies within that distance of a half-integer; such rare lanes
-// take the IEEE division. rcp_b is RN(1/b), computed once per scale. b > 0.
-__device__ __forceinline__ float rint_quotient(float a, float b, float rcp_b) {
-  const float qa = a * rcp_b;
-  const float c = rintf(qa);
-  if (fabsf(qa - c) > 0.5f - 0x1p-13f) return rintf(__fdiv_rn(a, b));
-  return c;
+// RN(a / b), the IEEE binary32 quotient, without a division, for a divisor b with at most
+// 11 significant bits (an fp16 value, or the constants 15 and 127) and y = RN(1/b):
+//   q0 = RN(a*y) lies within 2 ulp(a/b) of a/b (|b*y - 1| <= 2^-24);
+//   r = a - q0*b is exact (a multiple of 2^(e_q + e_b - 34) below 2^14 of those units),
+//   so the fma returns it exactly;
+//   q0 + r*y = a/b + (a/b - q0)(b*y - 1) = a/b + delta with |delta| <= 2^-23 ulp(a/b),
+//   and RN(q0 + r*y) is taken by the second fma in one rounding.
+// RN(a/b + delta) = RN(a/b) unless a rounding midpoint lies between a/b and a/b + delta.
+// a - m*b is a multiple of 2^(e_q + e_b - 34) for every midpoint m at a/b's exponent
+// (b has <= 11 bits, m <= 25), so a nonzero distance |a/b - m| is at least 2^-12 ulp(a/b);
+// and a/b = m exactly would need 25 significant bits in a. Hence the result is RN(a/b)
+// (a/b and a in the normal range; tiny quotients only decide codes that are 0 either way).
+// b = 0 with y = 0 gives 0.
+__device__ __forceinline__ float quotient_rn(float a, float b, float y) {
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-q0, b, a);
+  return __fmaf_rn(r, y, q0);
 }
+constexpr float kRcp15 = 1.0f / 15.0f;    // RN(1/15), folded by the compiler in binary32
+constexpr float kRcp127 = 1.0f / 127.0f;  // RN(1/127)
 
 __device__ __forceinline__ void set_err(int32_t *flag, uint32_t bit) {
   if (flag) atomicOr(reinterpret_cast<unsigned int *>(flag), bit);
