@@ -245,12 +245,12 @@ struct RowDst {
   int side_slot;
 };
 
-// Staging of the rows in shared memory: per thread its K row (256 B), 16 B of padding,
-// its V row. The thread stride of 528 B (132 words = 4 mod 32) makes the 16-byte reads of
-// 8 consecutive threads fall in distinct banks.
+// Staging of the rows in shared memory: per thread one row (256 B: its K row, then its V
+// row) and 16 B of padding. The thread stride of 272 B (68 words = 4 mod 32) makes the
+// 16-byte reads of 8 consecutive threads fall in distinct banks; 34 KB per block of 128
+// threads lets 6 blocks (24 warps) share an SM.
 constexpr int kRowsThreads = 128;
-constexpr int kRowStageV = 272;
-constexpr int kRowStageStride = 528;
+constexpr int kRowStageStride = 272;
 constexpr int kRowsSmem = kRowsThreads * kRowStageStride;
 
 // The 16 words (dims 32g..32g+31, two per word) of group g of a staged row.
@@ -341,12 +341,18 @@ __device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, fl
   }
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
 // Quantise one staged row (one new token and kv head, 128 bf16 values) into its INT4
 // record and, when protected, its INT8 copy. FROM8: demotion reading B (the INT4 copy
 // quantised from the INT8 copy). The group loop is not unrolled: the code stays small
-// enough for the instruction cache.
+// enough for the instruction cache. next (or nullptr): the global row staged into this
+// slot next; each of its groups is requested as soon as this row's group has been used.
 template <bool FROM8>
-__device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d) {
+__device__ __forceinline__ void quantize_row(uint8_t *row, const RowDst &d,
+                                             const uint8_t *next) {
   const bool need8 = FROM8 || d.side != nullptr;
   float s8 = 0.f, r8 = 0.f;
   uint16_t s8_bits = 0;
@@ -450,20 +456,23 @@ __device__ __forceinline__ void quantize_row(const uint8_t *row, const RowDst &d
           make_uint4(words[0], words[1], words[2], words[3]);
     pv[g] = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
             (static_cast<uint32_t>(__half_as_ushort(min_h)) << 16);
+    if (next != nullptr) {  // group g of this slot is consumed: fetch the next row's
+      const uint32_t st = static_cast<uint32_t>(__cvta_generic_to_shared(row + 64 * g));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cp_async16(st + 16 * i, next + 64 * g + 16 * i);
+    }
   }
   if (d.codes != nullptr)
     *reinterpret_cast<uint4 *>(d.params) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
   if (d.side != nullptr) *d.side_scale = s8_bits;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 
 // A warp = 32 consecutive CSR rows (lane = row) of one kv head; consecutive warps are
 // the heads of the same rows, so the rows' lookups hit the same L1 lines. Each thread
-// first stages its row's K and V (512 B) into shared memory with asynchronous copies,
-// then finds where the row goes while they land.
+// first stages its row's K (256 B) into shared memory with asynchronous copies and
+// prefetches its V into L2, then finds where the row goes while they land; V is staged
+// into the same slot once K is quantised.
 template <bool FROM8>
 __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
                                                          const uint16_t *__restrict__ k_new,
@@ -482,34 +491,63 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
   bool live = row < total_new;
 
   uint8_t *stage = rows_smem + threadIdx.x * kRowStageStride;
+  const size_t rowoff = (static_cast<size_t>(live ? row : r0) * H + h) * kHeadDim;
   if (live) {
-    const size_t rowoff = (static_cast<size_t>(row) * H + h) * kHeadDim;
     const uint8_t *ks = reinterpret_cast<const uint8_t *>(k_new + rowoff);
     const uint8_t *vs = reinterpret_cast<const uint8_t *>(v_new + rowoff);
     const uint32_t st = static_cast<uint32_t>(__cvta_generic_to_shared(stage));
 #pragma unroll
     for (int i = 0; i < 16; ++i) cp_async16(st + 16 * i, ks + 16 * i);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) cp_async16(st + kRowStageV + 16 * i, vs + 16 * i);
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(vs));  // V is staged after K is done
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(vs + 128));
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 
-  // the row's sequence: warp searches for the tile's first and last rows, then a
-  // per-lane binary search between them
-  const int b_first = find_seq_warp(new_indptr, c.num_seqs, r0, lane);
-  const int b_last = find_seq_warp(new_indptr, c.num_seqs, min(r0 + 31, total_new - 1), lane);
-  int lo = b_first, hi = b_last;  // largest b with indptr[b] <= row
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (new_indptr[mid] <= row) lo = mid; else hi = mid - 1;
-  }
-  const int b = lo;
-  int pos = -1, L = 0;
-  if (live) {
-    const int n = new_indptr[b + 1] - new_indptr[b];
-    const int i = row - new_indptr[b];
+  // the row's sequence: the warp finds the first row's sequence b0, then reads the CSR
+  // offsets, lengths and side-set indices of sequences b0 .. b0+31 in one round, and each
+  // lane picks its own sequence from them by a shuffle search (largest j with
+  // indptr[b0 + j] <= row)
+  const int B = c.num_seqs;
+  const int b0 = find_seq_warp(new_indptr, B, r0, lane);
+  const int wb = min(b0 + lane, B);
+  const int w_off = new_indptr[wb];
+  const int w_end = new_indptr[min(b0 + 32, B)];
+  const bool w_ok = b0 + lane < B;
+  const int w_len = w_ok ? c.seq_lens[wb] : 0;
+  const int w_sink = (w_ok && c.sink_idx) ? c.sink_idx[wb] : wb;
+  const int w_ring = (w_ok && c.ring_idx) ? c.ring_idx[wb] : wb;
+  int j = 0;
+#pragma unroll
+  for (int step = 16; step; step >>= 1)
+    if (__shfl_sync(0xffffffffu, w_off, j + step) <= row) j += step;
+  // every lane takes part in every shuffle (none sits inside a conditional expression)
+  const int off_b = __shfl_sync(0xffffffffu, w_off, j);
+  const int off_after = __shfl_sync(0xffffffffu, w_off, min(j + 1, 31));
+  const int off_next = j == 31 ? w_end : off_after;
+  int b = b0 + j;
+  int L = __shfl_sync(0xffffffffu, w_len, j);
+  int sink_set = __shfl_sync(0xffffffffu, w_sink, j);
+  int ring_id = __shfl_sync(0xffffffffu, w_ring, j);
+  int n = off_next - off_b, first = off_b;
+  if (live && j == 31 && w_end <= row && b0 + 32 < B) {
+    // rare: the row's sequence lies beyond the window (more than 32 sequences start in
+    // these 32 rows, i.e. empty ones): per-lane binary search
+    int lo = b0 + 32, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (new_indptr[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    first = new_indptr[b];
+    n = new_indptr[b + 1] - first;
     L = c.seq_lens[b];
-    pos = (i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges are rejected
+    sink_set = c.sink_idx ? c.sink_idx[b] : b;
+    ring_id = c.ring_idx ? c.ring_idx[b] : b;
+  }
+  int pos = -1;
+  if (live) {
+    const int i = row - first;
+    pos = (b < B && i >= 0 && i < n) ? L - n + i : -1;  // rows outside the CSR ranges
     if (pos < 0 || pos >= L || L > c.max_pages * kPage) {
       set_err(err, KV4_DEVERR_SEQ_LEN);
       live = false;
@@ -530,7 +568,7 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
     dk.slot = dv.slot = pos % kPage;
     const int S = c.num_sinks, R = c.num_recent;
     if (pos < S) {
-      const int set = c.sink_idx ? c.sink_idx[b] : b;
+      const int set = sink_set;
       if (set >= 0 && set < c.num_sink_sets) {
         const size_t sh = static_cast<size_t>(set) * H + h;
         const size_t tile = (sh * c.sink_tiles + pos / kPage) * kInt8CodeBytes;
@@ -542,7 +580,7 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
         set_err(err, KV4_DEVERR_SIDE_IDX);
       }
     } else if (R > 0 && pos >= L - R) {
-      const int ring = c.ring_idx ? c.ring_idx[b] : b;
+      const int ring = ring_id;
       if (ring >= 0 && ring < c.num_rings) {
         const int rs = pos % R;
         const size_t rh = static_cast<size_t>(ring) * H + h;
@@ -558,9 +596,10 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's own copies
   if (!live) return;
-#pragma unroll 1
-  for (int which = 0; which < 2; ++which)
-    quantize_row<FROM8>(stage + which * kRowStageV, which == 0 ? dk : dv);
+  quantize_row<FROM8>(stage, dk, reinterpret_cast<const uint8_t *>(v_new + rowoff));
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  quantize_row<FROM8>(stage, dv, nullptr);
 }
 
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,

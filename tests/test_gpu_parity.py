@@ -243,6 +243,41 @@ def test_code_decisions_at_exact_ties():
     check_attention(sess, [0])
 
 
+def test_bulk_append_across_empty_sequences():
+    """One CSR append whose 32-row tiles start more than 32 sequences (runs of empty
+    sequences between ones with rows), plus single-row and page-straddling sequences:
+    every written page and side copy bit-exact with the oracle."""
+    kv4, session, W = _mods()
+    counts = np.zeros(96, dtype=np.int64)
+    counts[0] = 5
+    counts[41] = 50      # 40 empty sequences after the first one's 5 rows
+    counts[42:75:3] = 1  # single rows with empty neighbours
+    counts[80] = 37
+    counts[95] = 70
+    wl = W.custom_workload(np.maximum(counts, 1), num_q_heads=8, num_kv_heads=2, num_sinks=4,
+                           num_recent=32, seed=23)
+    sess = session.DecodeSession(wl, steps=1, build=False)
+    dev = torch.device("cuda")
+    ks, vs = [], []
+    rng = np.random.default_rng(5)
+    for b in range(wl.num_seqs):
+        k = rng.standard_normal((int(counts[b]), 2, 128)).astype(np.float32)
+        v = rng.standard_normal((int(counts[b]), 2, 128)).astype(np.float32)
+        k = torch.from_numpy(k).to(torch.bfloat16)
+        v = torch.from_numpy(v).to(torch.bfloat16)
+        ks.append(k); vs.append(v)
+        sess.streams[b] = (k.float().numpy(), v.float().numpy())
+    indptr = np.zeros(wl.num_seqs + 1, dtype=np.int32)
+    indptr[1:] = np.cumsum(counts)
+    lens = torch.as_tensor(counts.astype(np.int32), device=dev)
+    sess.append(sess.batch(lens), torch.cat(ks).to(dev), torch.cat(vs).to(dev),
+                torch.as_tensor(indptr, device=dev))
+    torch.cuda.synchronize()
+    sess.check_err()
+    sess.L0 = counts
+    check_cache(sess, [b for b in range(wl.num_seqs) if counts[b] > 0])
+
+
 def test_heavy_tailed_values():
     _, _, W = _mods()
     wl = W.custom_workload([300, 901], num_q_heads=32, num_kv_heads=8, num_sinks=16,
