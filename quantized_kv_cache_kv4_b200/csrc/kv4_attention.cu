@@ -153,17 +153,30 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     return sp;
   };
 
-  // pass 1: totals over every sequence
+  // pass 1: totals over every sequence. A batch of at most kPlanThreads sequences is
+  // one block-wide pass, whose exclusive offsets and key ranks are kept for pass 2.
+  const bool single = B <= kPlanThreads;
   int tot[kScanN] = {0, 0, 0, 0, 0};
+  SeqPlan keep{};
+  int keep_off[kScanN] = {0, 0, 0, 0, 0};
+  int keep_rank = 0;
   if (threadIdx.x < 32) key_tot[threadIdx.x] = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
     SeqPlan sp = plan_of(base + threadIdx.x);
-    int t[kScanN];
-    block_scan_n(sp.n, t, warp_sums);
+    int off[kScanN], t[kScanN];
+#pragma unroll
+    for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
+    block_scan_n(off, t, warp_sums);
 #pragma unroll
     for (int i = 0; i < kScanN; ++i) tot[i] += t[i];
-    key_rank(sp.key, key_cnt, key_chunk);
+    const int krank = key_rank(sp.key, key_cnt, key_chunk);
     if (threadIdx.x < 32) key_tot[threadIdx.x] += key_chunk[threadIdx.x];
+    if (single) {
+      keep = sp;
+#pragma unroll
+      for (int i = 0; i < kScanN; ++i) keep_off[i] = off[i];
+      keep_rank = krank;
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {  // first rank of every key: exclusive scan over the keys
@@ -180,28 +193,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
   // pass 2: offsets up to this CTA's slice; entries of the slice (every unit empty if
   // the workspace is too small)
   // class bases: full chunks at 0, then long partial chunks, protected sets, short chunks
-  int run[kScanN] = {0, 0, tot[1], tot[1] + tot[2], tot[1] + tot[2] + tot[3]};
-  for (int base = 0; base < my_hi; base += kPlanThreads) {
-    const int b = base + threadIdx.x;
-    SeqPlan sp = fits ? plan_of(b) : SeqPlan{};
-    int off[kScanN], t[kScanN];
-#pragma unroll
-    for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
-    block_scan_n(off, t, warp_sums);
-#pragma unroll
-    for (int i = 0; i < kScanN; ++i) {
-      off[i] += run[i];
-      run[i] += t[i];
-    }
-    const int krank = key_rank(sp.key, key_cnt, key_chunk);
-    const int short_rank = sp.key >= 0 ? key_run[sp.key] + krank : 0;
-    __syncthreads();
-    if (threadIdx.x < 32) key_run[threadIdx.x] += key_chunk[threadIdx.x];
-    __syncthreads();
-    if (b < my_lo || b >= my_hi) continue;
+  const int class_base[kScanN] = {0, 0, tot[1], tot[1] + tot[2], tot[1] + tot[2] + tot[3]};
+  auto write_seq = [&](int b, const SeqPlan &sp, const int (&off)[kScanN], int short_rank) {
     const int pairs = sp.n[0];
     for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * off[0] + h * pairs;
-    if (pairs == 0) continue;
+    if (pairs == 0) return;
     const Regions &g = sp.g;
     int ef = off[1], el = off[2], epr = off[3];
     const int es = tot[1] + tot[2] + tot[3] + short_rank * nslots;
@@ -215,6 +211,39 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
       int e = sp.last_long ? el : es;
       for (int s = 0; s < nslots; ++s)
         w.entries[e++] = make_int4(b, g.has_prot + sp.nfull, s * hpw, min(hpw, H - s * hpw));
+    }
+  };
+  if (single) {  // the kept pass-1 offsets are final
+    const int b = threadIdx.x;
+    if (b >= my_lo && b < my_hi) {
+      int off[kScanN];
+      SeqPlan sp = fits ? keep : SeqPlan{};
+#pragma unroll
+      for (int i = 0; i < kScanN; ++i) off[i] = (fits ? keep_off[i] : 0) + class_base[i];
+      write_seq(b, sp, off, sp.key >= 0 ? key_run[sp.key] + keep_rank : 0);
+    }
+  } else {
+    int run[kScanN];
+#pragma unroll
+    for (int i = 0; i < kScanN; ++i) run[i] = class_base[i];
+    for (int base = 0; base < my_hi; base += kPlanThreads) {
+      const int b = base + threadIdx.x;
+      SeqPlan sp = fits ? plan_of(b) : SeqPlan{};
+      int off[kScanN], t[kScanN];
+#pragma unroll
+      for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
+      block_scan_n(off, t, warp_sums);
+#pragma unroll
+      for (int i = 0; i < kScanN; ++i) {
+        off[i] += run[i];
+        run[i] += t[i];
+      }
+      const int krank = key_rank(sp.key, key_cnt, key_chunk);
+      const int short_rank = sp.key >= 0 ? key_run[sp.key] + krank : 0;
+      __syncthreads();
+      if (threadIdx.x < 32) key_run[threadIdx.x] += key_chunk[threadIdx.x];
+      __syncthreads();
+      if (b >= my_lo && b < my_hi) write_seq(b, sp, off, short_rank);
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
