@@ -22,7 +22,8 @@ from .workload import Workload, make_paging, queries, seq_kv
 
 class DecodeSession:
     def __init__(self, wl: Workload, layer: int = 0, steps: int = 1, device="cuda",
-                 chunk_pages: int = 0, keep_streams=(), build: bool = True,
+                 chunk_pages: int = 0, keep_streams=(), keep_bits: bool = False,
+                 build: bool = True,
                  max_rows_per_call: int = 1 << 20, workspace: torch.Tensor | None = None,
                  demotion: str = "A"):
         self.wl = wl
@@ -45,7 +46,10 @@ class DecodeSession:
             (self.L0[None, :] + np.arange(steps)[:, None]).astype(np.int32), device=dev)
         self.max_len = int(self.L0.max()) + steps
         self.keep = set(int(b) for b in keep_streams)
-        self.streams = {}  # b -> (k, v) full bf16 streams kept on the host for the oracle
+        # b -> (k, v) full bf16 streams kept on the host for the oracle: float32 values,
+        # or (keep_bits) the bf16 bit patterns as uint16 (half the host memory)
+        self.streams = {}
+        self.keep_bits = keep_bits
         self.step_k = torch.empty((steps, B, wl.num_kv_heads, wl.head_dim), dtype=torch.bfloat16,
                                   device=dev)
         self.step_v = torch.empty_like(self.step_k)
@@ -100,7 +104,11 @@ class DecodeSession:
         end = int(self.L0[b]) + self.steps
         k, v = seq_kv(self.wl, b, end, self.layer, self.device)
         if b in self.keep:
-            self.streams[b] = (k.float().cpu().numpy(), v.float().cpu().numpy())
+            if self.keep_bits:
+                self.streams[b] = (k.view(torch.int16).cpu().numpy().view(np.uint16),
+                                   v.view(torch.int16).cpu().numpy().view(np.uint16))
+            else:
+                self.streams[b] = (k.float().cpu().numpy(), v.float().cpu().numpy())
         return k, v
 
     # ------------------------------------------------------------------ build
