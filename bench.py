@@ -531,7 +531,7 @@ def run_gpu(args, rank, world, local_rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kv4", choices=["kv4", "reference"])
     ap.add_argument("--workload", default="rollout")
