@@ -262,44 +262,12 @@ __device__ __forceinline__ void group_words(const uint8_t *row, int g, uint32_t 
   }
 }
 
-// ---- two fp32 lanes per instruction (sm_100 f32x2 arithmetic; each lane rounds to
-// nearest-even exactly as the scalar operation does) ----
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
-  return (static_cast<f32x2>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
-}
-__device__ __forceinline__ float lo_of(f32x2 v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float hi_of(f32x2 v) {
-  return __uint_as_float(static_cast<uint32_t>(v >> 32));
-}
-__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-  f32x2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
 // quotient_rn on a pair (nb = -b, y = RN(1/b) in both lanes), rounded to integers as
 // y = RN(a/b) + 1.5*2^23: callers know every quotient lies where no clamp is needed.
-__device__ __forceinline__ f32x2 round_quotient_pair(f32x2 a, f32x2 nb, f32x2 y) {
-  const f32x2 q0 = mul2(a, y);
-  const f32x2 q = fma2(fma2(q0, nb, a), y, q0);
-  return add2(q, pack2(kRoundMagic, kRoundMagic));
+__device__ __forceinline__ float2 round_quotient_pair(float2 a, float2 nb, float2 y) {
+  const float2 q0 = fmul2(a, y);
+  const float2 q = ffma2(ffma2(q0, nb, a), y, q0);
+  return fadd2(q, make_float2(kRoundMagic, kRoundMagic));
 }
 
 // INT8 codes of one group (words w: dims 2i, 2i+1 in word i), packed 4 per word (dim
@@ -309,20 +277,20 @@ template <bool FROM8>
 __device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, float r8, bool fast,
                                            uint32_t (&c8)[8], float (&x8)[32]) {
   if (fast) {
-    const f32x2 nb = pack2(-s8, -s8), yr = pack2(r8, r8);
+    const float2 nb = make_float2(-s8, -s8), yr = make_float2(r8, r8);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const f32x2 y0 =
-          round_quotient_pair(pack2(bf16_lo(w[2 * j]), bf16_hi(w[2 * j])), nb, yr);
-      const f32x2 y1 =
-          round_quotient_pair(pack2(bf16_lo(w[2 * j + 1]), bf16_hi(w[2 * j + 1])), nb, yr);
-      c8[j] = low_bytes(static_cast<uint32_t>(y0), static_cast<uint32_t>(y0 >> 32),
-                        static_cast<uint32_t>(y1), static_cast<uint32_t>(y1 >> 32));
+      const float2 y0 =
+          round_quotient_pair(make_float2(bf16_lo(w[2 * j]), bf16_hi(w[2 * j])), nb, yr);
+      const float2 y1 = round_quotient_pair(
+          make_float2(bf16_lo(w[2 * j + 1]), bf16_hi(w[2 * j + 1])), nb, yr);
+      c8[j] = low_bytes(__float_as_uint(y0.x), __float_as_uint(y0.y), __float_as_uint(y1.x),
+                        __float_as_uint(y1.y));
       if (FROM8) {
-        x8[4 * j] = lo_of(y0) - kRoundMagic;
-        x8[4 * j + 1] = hi_of(y0) - kRoundMagic;
-        x8[4 * j + 2] = lo_of(y1) - kRoundMagic;
-        x8[4 * j + 3] = hi_of(y1) - kRoundMagic;
+        x8[4 * j] = y0.x - kRoundMagic;
+        x8[4 * j + 1] = y0.y - kRoundMagic;
+        x8[4 * j + 2] = y1.x - kRoundMagic;
+        x8[4 * j + 3] = y1.y - kRoundMagic;
       }
     }
   } else {  // a saturated fp16 scale: clamp every code
@@ -426,15 +394,17 @@ __device__ __forceinline__ void quantize_row(uint8_t *row, const RowDst &d,
     // its low 8 bits.
     uint32_t words[4];
     if (fast) {
-      const f32x2 m2 = pack2(minf, minf), nb = pack2(-sf, -sf), yr = pack2(rf, rf);
+      const float2 m2 = make_float2(minf, minf), nb = make_float2(-sf, -sf);
+      const float2 yr = make_float2(rf, rf);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t pb[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int k = 8 * j + 2 * i;
-          const f32x2 y = round_quotient_pair(sub2(pack2(xval(k), xval(k + 1)), m2), nb, yr);
-          pb[i] = static_cast<uint32_t>(y) + (static_cast<uint32_t>(y >> 32) << 4);
+          const float2 y =
+              round_quotient_pair(fsub2(make_float2(xval(k), xval(k + 1)), m2), nb, yr);
+          pb[i] = __float_as_uint(y.x) + (__float_as_uint(y.y) << 4);
         }
         words[j] = low_bytes(pb[0], pb[1], pb[2], pb[3]);
       }

@@ -192,8 +192,29 @@ __device__ __forceinline__ void nib_pairs_v_sub(uint32_t x, uint32_t (&p)[4]) {
 }
 
 // ---------------------------------------------------------------------------
-// packed fp32 pairs (sm_100 f32x2 FMA pipe operations)
+// packed fp32 pairs (sm_100 f32x2 FMA pipe operations; each lane rounds to nearest-even
+// exactly as the scalar operation does)
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   float2 r;
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
