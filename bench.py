@@ -1,9 +1,10 @@
 """Benchmark: batched decode steps of paged INT4 + INT8-protected attention on B200.
 
-One step = the whole hot path for one batch: kv4_quantize_append of one new token per
-sequence (INT4 page write, INT8 copy, demotion out of the recent window) followed by
-kv4_decode_attention (INT8 protected partials, split-K INT4 partials, exact regional
-merge). The workload defaults to the 1024-sequence async-rollout batch (128 groups x 8
+One step = the whole hot path for one batch: kv4_decode_step, i.e. the quantise-append
+of one new token per sequence (INT4 page write, INT8 copy, demotion out of the recent
+window) followed by the decode attention (INT8 protected partials, split-K INT4
+partials, exact regional merge), in one call per layer. The attention is also timed as
+the separate kv4_decode_attention call, for the roofline. The workload defaults to the 1024-sequence async-rollout batch (128 groups x 8
 responses sharing a 256-token prompt, lognormal response lengths with mean 1450).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl kv4|reference]
@@ -407,46 +408,37 @@ def run_gpu(args, rank, world, local_rank):
             ls.check_err()
         return ev[0].elapsed_time(ev[1]), [a.elapsed_time(b) for a, b in att]
 
+    # A timed step is one kv4_decode_step call per layer (append + attention in one call,
+    # the attention's work list built beside the append); the attention calls are also
+    # timed on their own, as the separate kv4_decode_attention call, for the roofline.
     # eager: every call launches its kernels from the host
     with ClockSampler(local_rank) as clocks_eager:
-        ms_eager, att_eager = timed(lambda i, s, li: layers[li].append_step(s),
-                                    lambda i, s, li: layers[li].attention_step(s))
-    # graphs: each step's append and attention calls captured once per layer (outside the
-    # timed region) and replayed; the same kernels on the same per-step inputs
-    g_app, g_att = [], []
-    if args.launch == "graph-step":
-        # one graph per step: the append and attention calls of every layer
-        for s in steps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for ls in layers:
-                    ls.append_step(s)
-                    ls.attention_step(s)
-            g_app.append(g)
-        with ClockSampler(local_rank) as clocks:
-            ms, _ = timed(lambda i, s, li: g_app[i].replay() if li == 0 else None,
-                          lambda i, s, li: None)
-        att_ms = att_eager  # calls inside one graph are not timed one by one
-    elif args.launch == "graph":
+        ms_eager_calls, att_eager = timed(lambda i, s, li: layers[li].append_step(s),
+                                          lambda i, s, li: layers[li].attention_step(s))
+        ms_eager, _ = timed(lambda i, s, li: layers[li].fused_step(s), lambda i, s, li: None)
+    if args.launch == "graph":
+        # graphs: every call captured once per step and layer (outside the timed region)
+        # and replayed; the same kernels on the same per-step inputs
+        g_app, g_att, g_step = [], [], []
         for s in steps:
             for ls in layers:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    ls.append_step(s)
-                g_app.append(g)
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    ls.attention_step(s)
-                g_att.append(g)
+                for gl, fn in ((g_app, ls.append_step), (g_att, ls.attention_step),
+                               (g_step, ls.fused_step)):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        fn(s)
+                    gl.append(g)
+        ms_calls, att_ms = timed(lambda i, s, li: g_app[i * nl + li].replay(),
+                                 lambda i, s, li: g_att[i * nl + li].replay())
         with ClockSampler(local_rank) as clocks:
-            ms, att_ms = timed(lambda i, s, li: g_app[i * nl + li].replay(),
-                               lambda i, s, li: g_att[i * nl + li].replay())
+            ms, _ = timed(lambda i, s, li: g_step[i * nl + li].replay(), lambda i, s, li: None)
     else:
-        clocks, ms, att_ms = clocks_eager, ms_eager, att_eager
+        clocks, ms, att_ms, ms_calls = clocks_eager, ms_eager, att_eager, ms_eager_calls
     units_local = nl * sum(units_per_step(wl, L0 + s) for s in range(W, W + K))
     ms_max, units_all = combine_ranks(ms, units_local, world, dev)
     value = units_all / (ms_max / 1000.0)
     ms_eager_max, _ = combine_ranks(ms_eager, 0, world, dev)
+    ms_calls_max, _ = combine_ranks(ms_calls, 0, world, dev)
 
     # ---- roofline of the attention call (plan + split-K attention + merge) ----
     uniq = [attention_bytes(wl, L0 + s, args.cache) for s in range(W, W + K)]
@@ -498,12 +490,15 @@ def run_gpu(args, rank, world, local_rank):
                              f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
                        "cache": args.cache,
                        "parallelism": f"dp{world} (independent replica batches)",
-                       "launch": {"graph": "cuda graph per call (each layer's append and "
-                                           "attention call of every step)",
-                                  "graph-step": "one cuda graph per step (all calls of all "
-                                                "layers); attention call times from the eager run",
+                       "step": "one kv4_decode_step call per layer (append + attention; "
+                               "the work list built on a second stream beside the append)",
+                       "launch": {"graph": "cuda graph per call, replayed (each layer's "
+                                           "call of every step)",
                                   "eager": "eager"}[args.launch]},
             "attention_ms": statistics.mean(att_ms),
+            "two_calls": {"ms_per_step": ms_calls_max / K,
+                          "note": "kv4_quantize_append and kv4_decode_attention as separate "
+                                  "calls; attention_ms and the roofline time the latter"},
             "eager": {"value": units_all / (ms_eager_max / 1000.0),
                       "ms_per_step": ms_eager_max / K,
                       "attention_ms": statistics.mean(att_eager)},
@@ -545,8 +540,8 @@ def main(argv=None):
     ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
     ap.add_argument("--prefill", action="store_true",
                     help="also time a bulk prefill (one CSR append call of ~1M rows)")
-    ap.add_argument("--launch", default="graph", choices=["graph", "graph-step", "eager"],
-                    help="timed steps replayed from CUDA graphs (default) or launched eagerly")
+    ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
+                    help="timed calls replayed from CUDA graphs (default) or launched eagerly")
     args = ap.parse_args(argv)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

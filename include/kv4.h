@@ -198,6 +198,23 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
                                 kv4_stream_t stream);
 
 /*
+ * One decode step: kv4_quantize_append of one new token per sequence (new_indptr NULL,
+ * total_new = num_seqs; k_new, v_new bf16 [num_seqs][Hkv][128]) followed by
+ * kv4_decode_attention, with the same arguments, checks, results and error flags as
+ * the two calls made in that order on `stream` (batch->seq_lens are the lengths after
+ * the append). The attention's work list depends only on the lengths, so it is built on
+ * a second stream, forked from and joined back to `stream` with events, while the
+ * append runs; the call stays asynchronous and can be captured in a CUDA graph. The
+ * second stream and the two events are created on first use, one set per host thread
+ * and device, and live until the process ends.
+ */
+kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
+                           const kv4_int8_side *side, const kv4_batch *batch,
+                           const void *k_new, const void *v_new, const void *q, void *out,
+                           float *out_f32, float *lse, void *workspace, size_t ws_bytes,
+                           int32_t *err_flag, kv4_stream_t stream);
+
+/*
  * Exact regional softmax merge (ai4snews summary, "Interpretation" para. 3) of partial
  * states. A partial record is head_dim+4 floats: acc[head_dim] (sum of e^(s-m) v),
  * m (max logit, natural-log units), l (sum of e^(s-m)), 2 unused. Record (r, j) of

@@ -171,6 +171,31 @@ kv4_status carve_workspace(const kv4_config *cfg, const kv4::CacheView &v,
   return ws_bytes < need ? KV4_ERR_WORKSPACE_TOO_SMALL : KV4_OK;
 }
 
+// The second stream and fork/join events of kv4_decode_step: one set per host thread
+// and device, created on first use and kept for the life of the process.
+struct StepStreams {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+cudaError_t step_streams(StepStreams **out) {
+  constexpr int kMaxDevices = 64;
+  thread_local StepStreams per_device[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  StepStreams &ss = per_device[dev];
+  if (ss.side == nullptr) {
+    e = cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
 kv4_status check_attention_args(const kv4_batch *batch, const void *q, const void *out,
                                 const float *out_f32, const void *workspace) {
   if (q == nullptr || out == nullptr || workspace == nullptr) return KV4_ERR_INVALID_ARG;
@@ -224,6 +249,45 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   if (st != KV4_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
+  if (e == cudaSuccess)
+    e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
+                          static_cast<uint16_t *>(out), out_f32, lse, s);
+  return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
+                           const kv4_int8_side *side, const kv4_batch *batch,
+                           const void *k_new, const void *v_new, const void *q, void *out,
+                           float *out_f32, float *lse, void *workspace, size_t ws_bytes,
+                           int32_t *err_flag, kv4_stream_t stream) {
+  kv4::CacheView v;
+  kv4_status st = make_view(cfg, pool, side, batch, &v);
+  if (st != KV4_OK) return st;
+  if (batch->num_seqs == 0) return KV4_OK;
+  if (k_new == nullptr || v_new == nullptr || misaligned16(k_new) || misaligned16(v_new))
+    return KV4_ERR_INVALID_ARG;
+  st = check_attention_args(batch, q, out, out_f32, workspace);
+  if (st != KV4_OK) return st;
+  kv4::Workspace w;
+  st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
+  if (st != KV4_OK) return st;
+  StepStreams *ss = nullptr;
+  cudaError_t e = step_streams(&ss);
+  if (e != cudaSuccess) return KV4_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // fork: the work list on the second stream while the append runs on the caller's
+  e = cudaEventRecord(ss->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->side, ss->fork, 0);
+  if (e == cudaSuccess) e = kv4::launch_plan(v, w, err_flag, ss->side);
+  if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->side);
+  if (e == cudaSuccess)
+    e = kv4::launch_append(v, static_cast<const uint16_t *>(k_new),
+                           static_cast<const uint16_t *>(v_new), nullptr, batch->num_seqs,
+                           err_flag, s);
+  // join, then the attention and the merge behind both
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
@@ -315,6 +379,6 @@ const char *kv4_status_string(kv4_status status) {
   return "unknown status";
 }
 
-int32_t kv4_version(void) { return 300; }
+int32_t kv4_version(void) { return 400; }
 
 }  // extern "C"

@@ -7,8 +7,8 @@ streams with two device buffer sets, so that the host->device copy of the next l
 call and the device->host copy of the previous one overlap the append and attention
 kernels of the current one. Every call still moves all of its inputs and its whole
 output; only the order on the copy engines changes. The kernels are the library's,
-through the session's append and attend calls (kv4.quantize_append and
-kv4.decode_attention, or the baseline calls for a comparison cache).
+through the session's step call (kv4.decode_step: the append and the attention in one
+call, or the two baseline calls for a comparison cache).
 """
 from __future__ import annotations
 
@@ -19,8 +19,8 @@ class HostStepPipeline:
     """Double-buffered host<->device decode steps over one or more layers.
 
     `layers` is a DecodeSession-like object or a list of them (one per layer, same
-    shapes); each provides `append(batch, k, v)`, `attend(batch, q, out)`, `batch(lens)`
-    and example device tensors `step_k[0]`, `step_v[0]`, `q[0]`, `step_lens[0]`, `out`.
+    shapes); each provides `step_call(batch, k, v, q, out)`, `batch(lens)` and example
+    device tensors `step_k[0]`, `step_v[0]`, `q[0]`, `step_lens[0]`, `out`.
     """
 
     def __init__(self, layers, device=None):
@@ -73,8 +73,7 @@ class HostStepPipeline:
                 if u >= 2:
                     main.wait_event(self.copied_out[j])  # call u-2's output is on the host
                 b = sess.batch(self.lens[j])
-                sess.append(b, self.k[j], self.v[j])
-                sess.attend(b, self.q[j], self.out[j])
+                sess.step_call(b, self.k[j], self.v[j], self.q[j], self.out[j])
                 self.computed[j].record(main)
                 with torch.cuda.stream(self.d2h):
                     self.d2h.wait_event(self.computed[j])

@@ -29,7 +29,7 @@ PAGE = 16
 GROUP = 32
 
 EXPORTS = ("kv4_workspace_size", "kv4_quantize_append", "kv4_decode_attention",
-           "kv4_regional_merge", "kv4_status_string", "kv4_version",
+           "kv4_decode_step", "kv4_regional_merge", "kv4_status_string", "kv4_version",
            "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes",
            "kv4_baseline_append", "kv4_baseline_workspace_size",
            "kv4_baseline_decode_attention")
@@ -90,6 +90,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kv4_decode_attention.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Int4Pool),
                                          ctypes.POINTER(Int8Side), ctypes.POINTER(Batch),
                                          P, P, P, P, P, ctypes.c_size_t, P, P]
+    lib.kv4_decode_step.restype = ctypes.c_int
+    lib.kv4_decode_step.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Int4Pool),
+                                    ctypes.POINTER(Int8Side), ctypes.POINTER(Batch),
+                                    P, P, P, P, P, P, P, ctypes.c_size_t, P, P]
     lib.kv4_regional_merge.restype = ctypes.c_int
     lib.kv4_regional_merge.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        P, P, P, P]
@@ -249,6 +253,22 @@ def decode_attention(cache: Cache, batch: BatchTensors, q: torch.Tensor, out: to
                                    _ptr(out_f32), _ptr(lse), _ptr(workspace),
                                    workspace.numel(), _ptr(err), _stream(stream))
     _check(st, "kv4_decode_attention")
+
+
+def decode_step(cache: Cache, batch: BatchTensors, k_new: torch.Tensor, v_new: torch.Tensor,
+                q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                out_f32: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                err: torch.Tensor | None = None, stream=None):
+    """One decode step: quantize_append of one token per sequence (k_new, v_new bf16
+    [B, Hkv, 128]) then decode_attention, in one library call (the attention's work list
+    is built on a second stream while the append runs). batch.lens: lengths after the
+    append."""
+    pool, side, bs = cache.pool_struct(), cache.side_struct(), batch.struct()
+    st = _lib.kv4_decode_step(ctypes.byref(cache.cfg), ctypes.byref(pool), ctypes.byref(side),
+                              ctypes.byref(bs), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out),
+                              _ptr(out_f32), _ptr(lse), _ptr(workspace), workspace.numel(),
+                              _ptr(err), _stream(stream))
+    _check(st, "kv4_decode_step")
 
 
 def decode_attention_noalloc(cache: Cache, batch: BatchTensors, q: torch.Tensor,

@@ -181,6 +181,18 @@ class DecodeSession:
         self.append_step(s, stream=kw.get("stream"))
         self.attention_step(s, **kw)
 
+    def step_call(self, batch, k, v, q, out, out_f32=None, lse=None, stream=None):
+        """One decode step (one new token per sequence) as one kv4.decode_step call:
+        append + attention, the attention's work list built beside the append."""
+        kv4.decode_step(self.cache, batch, k, v, q, out, self.workspace, out_f32, lse,
+                        self.err, stream=stream)
+
+    def fused_step(self, s: int = 0, out=None, out_f32=None, lse=None, stream=None):
+        """Step s through step_call."""
+        self.step_call(self.batch(self.step_lens[s]), self.step_k[s], self.step_v[s],
+                       self.q[s], self.out if out is None else out, out_f32, lse,
+                       stream=stream)
+
     def check_err(self):
         flag = int(self.err.item())
         if flag:
@@ -209,3 +221,8 @@ class BaselineSession(DecodeSession):
     def attend(self, batch, q, out, out_f32=None, lse=None, stream=None):
         kv4.baseline_decode_attention(self.cache, batch, q, out, self.workspace, out_f32, lse,
                                       self.err, stream=stream)
+
+    def step_call(self, batch, k, v, q, out, out_f32=None, lse=None, stream=None):
+        """The comparison caches have no fused entry point: the two calls in order."""
+        self.append(batch, k, v, None, stream=stream)
+        self.attend(batch, q, out, out_f32, lse, stream=stream)

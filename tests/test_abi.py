@@ -28,8 +28,9 @@ def declared_functions():
 
 def test_header_declares_the_calls():
     names = declared_functions()
-    for want in ("kv4_quantize_append", "kv4_decode_attention", "kv4_regional_merge",
-                 "kv4_workspace_size", "kv4_status_string", "kv4_version"):
+    for want in ("kv4_quantize_append", "kv4_decode_attention", "kv4_decode_step",
+                 "kv4_regional_merge", "kv4_workspace_size", "kv4_status_string",
+                 "kv4_version"):
         assert want in names
 
 
@@ -45,7 +46,7 @@ def test_library_exports_every_declared_symbol(kv4):
 
 def test_status_strings_and_version(kv4):
     lib = kv4._lib
-    assert lib.kv4_version() == 300
+    assert lib.kv4_version() == 400
     assert lib.kv4_status_string(0) == b"ok"
     assert b"144" in lib.kv4_status_string(-3)
     assert lib.kv4_status_string(-99) == b"unknown status"
@@ -154,6 +155,35 @@ def test_workspace_too_small_is_reported(kv4):
                                        ctypes.c_void_p(1 << 20), None, None,
                                        ctypes.c_void_p(1 << 20), need - 256, None, None)
     assert st == -4
+
+
+def test_decode_step_argument_checks(kv4):
+    """kv4_decode_step checks the append's and the attention's arguments before it
+    creates or launches anything (no device needed for these)."""
+    lib = kv4._lib
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+
+    def call(c, pool, side, batch, k, v, ws_bytes):
+        return lib.kv4_decode_step(ctypes.byref(c), ctypes.byref(pool), ctypes.byref(side),
+                                   ctypes.byref(batch), k, v, good, good, None, None, good,
+                                   ws_bytes, None, None)
+    pool = kv4.Int4Pool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
+    side = kv4.Int8Side(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1 << 20, 1 << 20, 1 << 20,
+                        1 << 20, 2)
+    batch = kv4.Batch(1 << 20, 64, 1 << 20, 1 << 20, 0, 2, 1000)
+    need = kv4.workspace_size(_cfg(kv4, chunk_pages=64), 2, 1000)
+    c = _cfg(kv4)
+    c.head_dim = 64
+    assert call(c, pool, side, batch, good, good, need) == -2
+    c = _cfg(kv4, num_sinks=100, num_recent=100)
+    assert call(c, pool, side, batch, good, good, need) == -3
+    c = _cfg(kv4)
+    assert call(c, pool, side, batch, None, good, need) == -1        # no new K
+    assert call(c, pool, side, batch, P((1 << 20) + 8), good, need) == -1  # misaligned K rows
+    assert call(c, pool, side, batch, good, good, need - 256) == -4  # workspace too small
+    empty = kv4.Batch(1 << 20, 64, 1 << 20, 1 << 20, 0, 0, 1000)
+    assert call(c, pool, side, empty, None, None, 0) == 0             # nothing to do
 
 
 def test_baseline_argument_checks(kv4):

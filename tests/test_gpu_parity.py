@@ -280,6 +280,52 @@ def test_bulk_append_across_empty_sequences():
     check_cache(sess, [b for b in range(wl.num_seqs) if counts[b] > 0])
 
 
+def test_decode_step_matches_separate_calls():
+    """kv4_decode_step (append + attention, the work list built on a second stream) gives
+    the same cache and the same outputs, bit for bit, as the two calls in order; also
+    when captured in a CUDA graph; and its outputs match the oracle."""
+    kv4, session, W = _mods()
+    wl = W.custom_workload([37, 150, 161, 600, 1, 2049], num_sinks=4, num_recent=32, seed=41)
+    keep = range(wl.num_seqs)
+    sa = session.DecodeSession(wl, steps=3, keep_streams=keep)
+    sb = session.DecodeSession(wl, steps=3, keep_streams=keep)
+    B, Hq = wl.num_seqs, wl.num_q_heads
+    dev = torch.device("cuda")
+
+    def outs():
+        return (torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev),
+                torch.empty((B, Hq, 128), dtype=torch.float32, device=dev),
+                torch.empty((B, Hq), dtype=torch.float32, device=dev))
+    for s in range(2):
+        oa, fa, la = outs()
+        ob, fb, lb = outs()
+        sa.append_step(s)
+        sa.attention_step(s, out=oa, out_f32=fa, lse=la)
+        sb.fused_step(s, out=ob, out_f32=fb, lse=lb)
+        torch.cuda.synchronize()
+        assert torch.equal(oa, ob) and torch.equal(fa, fb) and torch.equal(la, lb), s
+        if s == 0:
+            check_attention(sb, range(B), got=(ob.float().cpu().numpy(), fb.cpu().numpy(),
+                                               lb.cpu().numpy()))
+    # step 2 replayed from a captured graph
+    oa, fa, la = outs()
+    ob, fb, lb = outs()
+    sa.append_step(2)
+    sa.attention_step(2, out=oa, out_f32=fa, lse=la)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        sb.fused_step(2, out=ob, out_f32=fb, lse=lb)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(oa, ob) and torch.equal(fa, fb) and torch.equal(la, lb)
+    sa.check_err()
+    sb.check_err()
+    ca, cb = sa.cache, sb.cache
+    for name in ("k_codes", "v_codes", "k_params", "v_params", "sink_k", "sink_ks", "sink_v",
+                 "sink_vs", "ring_k", "ring_ks", "ring_v", "ring_vs"):
+        assert torch.equal(getattr(ca, name), getattr(cb, name)), name
+
+
 def test_heavy_tailed_values():
     _, _, W = _mods()
     wl = W.custom_workload([300, 901], num_q_heads=32, num_kv_heads=8, num_sinks=16,
