@@ -213,7 +213,10 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
                   demotion: str = "A"):
     """Time the oracle's decode output (quantise -> dequantise -> softmax attention; for a
     comparison cache its BF16 / KV8 reference) on consecutive sequences of the workload
-    until `budget_s` of CPU time is used. Returns (units, seconds, description, threads)."""
+    until `budget_s` of CPU time is used. For the KV4-RL cache the oracle's quantiser
+    alone (the stored records of every position: what the append writes) is timed on the
+    same sequences too. Returns (units, seconds, description, threads, quantise seconds
+    or None)."""
     import torch
     from oracle import kv4_oracle as O
     from quantized_kv_cache_kv4_b200.workload import queries, seq_kv
@@ -224,6 +227,7 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
         threads = 1
     q_all = queries(wl, 0, 0, "cpu").float().numpy()
     units, spent, seqs = 0, 0.0, []
+    quant = 0.0 if cache == "kv4" else None
     b = start_seq
     while spent < budget_s and len(seqs) < wl.num_seqs:
         bb = b % wl.num_seqs
@@ -238,6 +242,10 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
         else:
             O.decode_reference(q_all[bb], k, v, wl.num_sinks, wl.num_recent, demotion)
         spent += time.perf_counter() - t0
+        if quant is not None:
+            t0 = time.perf_counter()
+            O.token_records(k, v, demotion)
+            quant += time.perf_counter() - t0
         units += L * wl.num_kv_heads
         seqs.append(bb)
         b += 1
@@ -246,7 +254,7 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
     desc = (f"oracle {fn} (fp64 numpy: quantise every position, dequantise, "
             f"softmax attention) on {len(seqs)} sequence(s) of the workload "
             f"({units // wl.num_kv_heads} context tokens)")
-    return units, spent, desc, threads
+    return units, spent, desc, threads, quant
 
 
 def run_reference(args, rank, world):
@@ -256,7 +264,8 @@ def run_reference(args, rank, world):
     total_units, total_s, descs, threads = 0, 0.0, [], 1
     per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
-        u, t, d, threads = oracle_sample(wl, per_step_budget, start_seq=s * 3, cache=args.cache,
+        u, t, d, threads, _ = oracle_sample(wl, per_step_budget, start_seq=s * 3,
+                                            cache=args.cache,
                                          demotion=args.demotion)
         if s >= args.warmup:
             total_units += u
@@ -472,10 +481,14 @@ def run_gpu(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        u, secs, desc, threads = oracle_sample(wl, args.cpu_budget, cache=args.cache,
-                                               demotion=args.demotion)
+        u, secs, desc, threads, qsecs = oracle_sample(wl, args.cpu_budget, cache=args.cache,
+                                                      demotion=args.demotion)
         cpu = {"value": u / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": desc}
+        if qsecs:
+            cpu["quantise"] = {"value": u / qsecs, "unit": "tokens*kv_heads/s",
+                               "what": "oracle token_records (INT4 records and INT8 copies "
+                                       "of every position) on the same sample"}
 
     if rank == 0:
         ub = statistics.mean(u for u, _ in uniq)
