@@ -265,8 +265,7 @@ def run_reference(args, rank, world):
     per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
         u, t, d, threads, _ = oracle_sample(wl, per_step_budget, start_seq=s * 3,
-                                            cache=args.cache,
-                                         demotion=args.demotion)
+                                            cache=args.cache, demotion=args.demotion)
         if s >= args.warmup:
             total_units += u
             total_s += t
