@@ -208,3 +208,18 @@ def test_baseline_argument_checks(kv4):
         ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 20), None, None,
         ctypes.c_void_p(1 << 20), 256, None, None)
     assert st == -4
+
+
+def test_plain_c_program_uses_the_abi(kv4, tmp_path):
+    """tests/c_abi_check.c, compiled with gcc against the header alone and linked to the
+    library, runs the host-answered calls from C."""
+    exe = tmp_path / "c_abi_check"
+    lib_dir = os.path.dirname(kv4.LIB_PATH)
+    build = subprocess.run(
+        ["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+         os.path.join(ROOT, "tests", "c_abi_check.c"), "-L", lib_dir, "-lkv4",
+         "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
+
