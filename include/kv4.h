@@ -206,7 +206,9 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
  * a second stream, forked from and joined back to `stream` with events, while the
  * append runs; the call stays asynchronous and can be captured in a CUDA graph. The
  * second stream and the two events are created on first use, one set per host thread
- * and device, and live until the process ends.
+ * and device, and live until the process ends; a thread's first call made while the
+ * stream is being captured creates nothing and builds the work list on `stream`
+ * itself (same results, without the overlap).
  */
 kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
                            const kv4_int8_side *side, const kv4_batch *batch,

@@ -178,17 +178,22 @@ struct StepStreams {
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 
-cudaError_t step_streams(StepStreams **out) {
+// *out = this thread's set for the current device, created unless `create` is false
+// (then nullptr when it does not exist yet).
+cudaError_t step_streams(bool create, StepStreams **out) {
   constexpr int kMaxDevices = 64;
   thread_local StepStreams per_device[kMaxDevices];
+  *out = nullptr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   StepStreams &ss = per_device[dev];
-  if (ss.side == nullptr) {
-    e = cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+  if (ss.join == nullptr) {
+    if (!create) return cudaSuccess;
+    if (ss.side == nullptr) e = cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking);
+    if (e == cudaSuccess && ss.fork == nullptr)
+      e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
     if (e != cudaSuccess) return e;
   }
@@ -273,21 +278,30 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   kv4::Workspace w;
   st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
-  StepStreams *ss = nullptr;
-  cudaError_t e = step_streams(&ss);
-  if (e != cudaSuccess) return KV4_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // fork: the work list on the second stream while the append runs on the caller's
-  e = cudaEventRecord(ss->fork, s);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->side, ss->fork, 0);
-  if (e == cudaSuccess) e = kv4::launch_plan(v, w, err_flag, ss->side);
-  if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->side);
+  // The second stream and its events are not created while the caller's stream is being
+  // captured into a graph; a first call made there builds the work list on the caller's
+  // stream (same results, no overlap).
+  cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &capturing);
+  if (e != cudaSuccess) return KV4_ERR_CUDA;
+  StepStreams *ss = nullptr;
+  e = step_streams(capturing == cudaStreamCaptureStatusNone, &ss);
+  if (e != cudaSuccess) return KV4_ERR_CUDA;
+  if (ss != nullptr) {  // fork: the work list on the second stream beside the append
+    e = cudaEventRecord(ss->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->side, ss->fork, 0);
+    if (e == cudaSuccess) e = kv4::launch_plan(v, w, err_flag, ss->side);
+    if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->side);
+  } else {
+    e = kv4::launch_plan(v, w, err_flag, s);
+  }
   if (e == cudaSuccess)
     e = kv4::launch_append(v, static_cast<const uint16_t *>(k_new),
                            static_cast<const uint16_t *>(v_new), nullptr, batch->num_seqs,
                            err_flag, s);
   // join, then the attention and the merge behind both
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+  if (e == cudaSuccess && ss != nullptr) e = cudaStreamWaitEvent(s, ss->join, 0);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)

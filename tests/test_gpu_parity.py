@@ -283,12 +283,13 @@ def test_bulk_append_across_empty_sequences():
 def test_decode_step_matches_separate_calls():
     """kv4_decode_step (append + attention, the work list built on a second stream) gives
     the same cache and the same outputs, bit for bit, as the two calls in order; also
-    when captured in a CUDA graph; and its outputs match the oracle."""
+    when captured in a CUDA graph, including a new thread's first call; and its outputs
+    match the oracle."""
     kv4, session, W = _mods()
     wl = W.custom_workload([37, 150, 161, 600, 1, 2049], num_sinks=4, num_recent=32, seed=41)
     keep = range(wl.num_seqs)
-    sa = session.DecodeSession(wl, steps=3, keep_streams=keep)
-    sb = session.DecodeSession(wl, steps=3, keep_streams=keep)
+    sa = session.DecodeSession(wl, steps=4, keep_streams=keep)
+    sb = session.DecodeSession(wl, steps=4, keep_streams=keep)
     B, Hq = wl.num_seqs, wl.num_q_heads
     dev = torch.device("cuda")
 
@@ -317,6 +318,30 @@ def test_decode_step_matches_separate_calls():
         sb.fused_step(2, out=ob, out_f32=fb, lse=lb)
     g.replay()
     torch.cuda.synchronize()
+    assert torch.equal(oa, ob) and torch.equal(fa, fb) and torch.equal(la, lb)
+    # step 3: the first call of a new host thread, made while capturing (the library
+    # creates nothing then and builds the work list on the captured stream)
+    import threading
+    oa, fa, la = outs()
+    ob, fb, lb = outs()
+    sa.append_step(3)
+    sa.attention_step(3, out=oa, out_f32=fa, lse=la)
+    torch.cuda.synchronize()
+    failures = []
+
+    def capture_in_new_thread():
+        try:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                sb.fused_step(3, out=ob, out_f32=fb, lse=lb)
+            g2.replay()
+            torch.cuda.synchronize()
+        except Exception as ex:  # reported below, on the test's thread
+            failures.append(ex)
+    t = threading.Thread(target=capture_in_new_thread)
+    t.start()
+    t.join()
+    assert not failures, failures
     assert torch.equal(oa, ob) and torch.equal(fa, fb) and torch.equal(la, lb)
     sa.check_err()
     sb.check_err()
