@@ -246,12 +246,12 @@ struct RowDst {
 };
 
 // Staging of the rows in shared memory: per thread one row (256 B: its K row, then its V
-// row) and 16 B of padding. The thread stride of 272 B (68 words = 4 mod 32) makes the
-// 16-byte reads of 8 consecutive threads fall in distinct banks; 34 KB per block of 128
-// threads lets 6 blocks (24 warps) share an SM.
+// row) and 16 B of padding, then two mbarriers per warp. The thread stride of 272 B (68
+// words = 4 mod 32) makes the 16-byte reads of 8 consecutive threads fall in distinct
+// banks; 34 KB per block of 128 threads lets 6 blocks (24 warps) share an SM.
 constexpr int kRowsThreads = 128;
 constexpr int kRowStageStride = 272;
-constexpr int kRowsSmem = kRowsThreads * kRowStageStride;
+constexpr int kRowsSmem = kRowsThreads * kRowStageStride + (kRowsThreads / 32) * 16;
 
 // The 16 words (dims 32g..32g+31, two per word) of group g of a staged row.
 __device__ __forceinline__ void group_words(const uint8_t *row, int g, uint32_t (&w)[16]) {
@@ -309,10 +309,6 @@ __device__ __forceinline__ void int8_group(const uint32_t (&w)[16], float s8, fl
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
 // Quantise one staged row (one new token and kv head, 128 bf16 values) into its INT4
 // record and, when protected, its INT8 copy. FROM8: demotion reading B (the INT4 copy
 // quantised from the INT8 copy). The group loop is not unrolled: the code stays small
@@ -320,7 +316,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 // slot next; each of its groups is requested as soon as this row's group has been used.
 template <bool FROM8>
 __device__ __forceinline__ void quantize_row(uint8_t *row, const RowDst &d,
-                                             const uint8_t *next) {
+                                             const uint8_t *next, uint64_t *next_bar) {
   const bool need8 = FROM8 || d.side != nullptr;
   float s8 = 0.f, r8 = 0.f;
   uint16_t s8_bits = 0;
@@ -427,9 +423,8 @@ __device__ __forceinline__ void quantize_row(uint8_t *row, const RowDst &d,
     pv[g] = static_cast<uint32_t>(__half_as_ushort(scale_h)) |
             (static_cast<uint32_t>(__half_as_ushort(min_h)) << 16);
     if (next != nullptr) {  // group g of this slot is consumed: fetch the next row's
-      const uint32_t st = static_cast<uint32_t>(__cvta_generic_to_shared(row + 64 * g));
-#pragma unroll
-      for (int i = 0; i < 4; ++i) cp_async16(st + 16 * i, next + 64 * g + 16 * i);
+      fence_proxy_async_smem();  // the reads above come before the async write
+      bulk_g2s(row + 64 * g, next + 64 * g, 64, next_bar);
     }
   }
   if (d.codes != nullptr)
@@ -440,9 +435,11 @@ __device__ __forceinline__ void quantize_row(uint8_t *row, const RowDst &d,
 
 // A warp = 32 consecutive CSR rows (lane = row) of one kv head; consecutive warps are
 // the heads of the same rows, so the rows' lookups hit the same L1 lines. Each thread
-// first stages its row's K (256 B) into shared memory with asynchronous copies and
-// prefetches its V into L2, then finds where the row goes while they land; V is staged
-// into the same slot once K is quantised.
+// first stages its row's K (256 B) into shared memory with one bulk copy (TMA engine,
+// completion on the warp's mbarrier) and prefetches its V into L2, then finds where the
+// row goes while they land; V is staged into the same slot, group by group, as K's
+// groups are consumed (a second mbarrier). One bulk copy per row instead of sixteen
+// 16-byte copies keeps the memory-instruction queue free for the arithmetic.
 template <bool FROM8>
 __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
                                                          const uint16_t *__restrict__ k_new,
@@ -461,17 +458,23 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
   bool live = row < total_new;
 
   uint8_t *stage = rows_smem + threadIdx.x * kRowStageStride;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rows_smem + kRowsThreads * kRowStageStride) +
+                   2 * (threadIdx.x >> 5);  // this warp's: K rows, V rows
   const size_t rowoff = (static_cast<size_t>(live ? row : r0) * H + h) * kHeadDim;
-  if (live) {
-    const uint8_t *ks = reinterpret_cast<const uint8_t *>(k_new + rowoff);
+  const int n_k = __popc(__ballot_sync(0xffffffffu, live));
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&bars[0], n_k * 256u);
+  }
+  __syncwarp();
+  if (live) {  // one bulk copy per K row; V is prefetched into L2 and staged after K
     const uint8_t *vs = reinterpret_cast<const uint8_t *>(v_new + rowoff);
-    const uint32_t st = static_cast<uint32_t>(__cvta_generic_to_shared(stage));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) cp_async16(st + 16 * i, ks + 16 * i);
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(vs));  // V is staged after K is done
+    bulk_g2s(stage, k_new + rowoff, 256, &bars[0]);
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(vs));
     asm volatile("prefetch.global.L2 [%0];" ::"l"(vs + 128));
   }
-  asm volatile("cp.async.commit_group;" ::: "memory");
 
   // the row's sequence: the warp finds the first row's sequence b0, then reads the CSR
   // offsets, lengths and side-set indices of sequences b0 .. b0+31 in one round, and each
@@ -564,12 +567,24 @@ __global__ void __launch_bounds__(kRowsThreads) append_rows_kernel(CacheView c,
       }
     }
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's own copies
+  // the V rows the warp will stage: those still live after the lookups
+  const int n_v = __popc(__ballot_sync(0xffffffffu, live));
+  if (lane == 0) mbar_arrive_expect_tx(&bars[1], n_v * 256u);
+  // every lane waits for the warp's K copies (none may exit with one in flight); the
+  // waits are bounded, and a wait that gives up waits once more before returning
+  if (!mbar_wait_bounded(&bars[0], 0)) {
+    if (lane == 0) set_err(err, KV4_DEVERR_TIMEOUT);
+    mbar_wait_bounded(&bars[0], 0);
+    return;
+  }
   if (!live) return;
-  quantize_row<FROM8>(stage, dk, reinterpret_cast<const uint8_t *>(v_new + rowoff));
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  quantize_row<FROM8>(stage, dv, nullptr);
+  quantize_row<FROM8>(stage, dk, reinterpret_cast<const uint8_t *>(v_new + rowoff), &bars[1]);
+  if (!mbar_wait_bounded(&bars[1], 0)) {
+    set_err(err, KV4_DEVERR_TIMEOUT);
+    mbar_wait_bounded(&bars[1], 0);
+    return;
+  }
+  quantize_row<FROM8>(stage, dv, nullptr, nullptr);
 }
 
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
