@@ -59,44 +59,41 @@ def attention_bytes(wl, lens, cache="kv4"):
 
     Per token and KV head: 160 B when read from INT4 (64 B K codes + 16 B K params +
     the same for V), 260 B when read from INT8 (128 B codes + 2 B scale, K and V).
-    Plus the query read and the output write (bf16). `unique` counts a group's shared
-    prompt pages and shared sink set once; `logical` counts them per sequence.
-    Comparison caches: 512 B per token and head for BF16, 260 B for KV8, at every
-    position; shared prompt positions counted once in `unique`."""
+    Plus the query read and the output write (bf16). `logical` counts every sequence's
+    reads; `unique` counts each stored byte read once: with a shared prompt, a group's
+    sink set and the prompt positions of its shared INT4 pages once for the group (a
+    prompt position inside a member's recent window is read from that member's own
+    ring). Comparison caches: 512 B per token and head for BF16, 260 B for KV8, at every
+    position; a group's shared prompt positions counted once in `unique`."""
     lens = np.asarray(lens, dtype=np.int64)
+    H = wl.num_kv_heads
+    io = lens.size * wl.num_q_heads * wl.head_dim * 2 * 2
+    G = wl.group_seqs if wl.shared_prefix else 1
+    P = wl.prompt_len if wl.shared_prefix else 0
+    groups = [lens[g:g + G] for g in range(0, lens.size, G)]
     if cache in ("bf16", "kv8"):
         per = 512 if cache == "bf16" else 260
-        H = wl.num_kv_heads
         logical = int(lens.sum()) * per * H
-        io = lens.size * wl.num_q_heads * wl.head_dim * 2 * 2
-        unique = logical
-        if wl.shared_prefix:
-            shared = np.minimum(wl.prompt_len, lens)
-            dup = 0
-            for g in range((lens.size + wl.group_seqs - 1) // wl.group_seqs):
-                sl = slice(g * wl.group_seqs, (g + 1) * wl.group_seqs)
-                dup += int(shared[sl].min()) * per * (lens[sl].size - 1)
-            unique = logical - dup * H
+        unique = sum(int(min(P, gl.max())) + int(np.maximum(0, gl - P).sum())
+                     for gl in groups) * per * H
         return int(unique + io), int(logical + io)
-    S, R, H = wl.num_sinks, wl.num_recent, wl.num_kv_heads
+    S, R = wl.num_sinks, wl.num_recent
     prot = np.minimum(lens, S + R)
     int4 = np.maximum(0, lens - S - R)
-    logical = (int4 * 160 + prot * 260).sum() * H
-    io = lens.size * wl.num_q_heads * wl.head_dim * 2 * 2
-    unique = logical
-    if wl.shared_prefix:
-        P = wl.prompt_len
-        shared_int4 = np.maximum(0, np.minimum(P, lens - R) - S)  # prompt part of INT4 range
-        shared_sink = np.minimum(lens, S)
-        groups = (lens.size + wl.group_seqs - 1) // wl.group_seqs
-        dup = 0
-        for g in range(groups):
-            sl = slice(g * wl.group_seqs, (g + 1) * wl.group_seqs)
-            n = lens[sl].size
-            # counted n times, should be once (all sequences in a group share them)
-            dup += (shared_int4[sl].min() * 160 + shared_sink[sl].min() * 260) * (n - 1)
-        unique = logical - dup * H
-    return int(unique + io), int(logical + io)
+    logical = int((int4 * 160 + prot * 260).sum()) * H
+    unique = 0
+    for gl in groups:
+        ring = np.maximum(0, gl - np.maximum(S, gl - R))  # recent window: per sequence
+        if P:  # sink set per group; INT4 prompt pages shared, the rest per sequence
+            sink = int(min(S, gl.max()))
+            shared4 = max(0, int(min(P, (gl - R).max())) - S)
+            own4 = np.maximum(0, gl - R - max(P, S))
+            unique += sink * 260 + shared4 * 160 + int((ring * 260 + own4 * 160).sum())
+        else:
+            sink = np.minimum(S, gl)
+            own4 = np.maximum(0, gl - R - S)
+            unique += int(((sink + ring) * 260 + own4 * 160).sum())
+    return int(unique * H + io), int(logical + io)
 
 
 def time_prefill(sess, wl, dev, max_rows=1 << 20, reps=5):

@@ -84,3 +84,50 @@ def test_reference_arm_prints_the_contract_line():
     assert d["config"]["workload"].startswith("tiny")
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def _brute_force_bytes(wl, lens, cache):
+    """Position by position: which stored copy every read touches, and its bytes."""
+    H, S, R = wl.num_kv_heads, wl.num_sinks, wl.num_recent
+    P = wl.prompt_len if wl.shared_prefix else 0
+    logical, seen = 0, set()
+    for b, L in enumerate(lens):
+        g = wl.group_of(b)
+        for p in range(int(L)):
+            if cache != "kv4":
+                nbytes = 512 if cache == "bf16" else 260
+                where = ("page", g, p) if p < P else ("page", b, p)
+            elif p < S:
+                nbytes = 260
+                where = ("sink", g if P else b, p)
+            elif p >= L - R:
+                nbytes = 260
+                where = ("ring", b, p)
+            else:
+                nbytes = 160
+                where = ("page", g, p) if p < P else ("page", b, p)
+            logical += nbytes * H
+            seen.add((where, nbytes))
+    unique = sum(nb for _, nb in seen) * H
+    io = len(lens) * wl.num_q_heads * wl.head_dim * 4
+    return unique + io, logical + io
+
+
+@pytest.mark.parametrize("cache", ["kv4", "bf16", "kv8"])
+def test_algorithmic_bytes_match_a_position_count(cache):
+    """The roofline numerator (bench.attention_bytes) against a count of every read,
+    with and without shared prompts, sequences shorter than the protected set and
+    recent windows reaching into the prompt."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from quantized_kv_cache_kv4_b200 import workload as W
+    rng = np.random.default_rng(3)
+    cases = [W.custom_workload(rng.integers(1, 700, 12), num_sinks=4, num_recent=32),
+             W.custom_workload(rng.integers(65, 500, 12), num_sinks=16, num_recent=128,
+                               prompt_len=64, group_seqs=4),
+             W.custom_workload([65, 70, 400, 900, 66, 1000, 129, 130], num_sinks=4,
+                               num_recent=96, prompt_len=64, group_seqs=4)]
+    for wl in cases:
+        got = bench.attention_bytes(wl, wl.seq_lens, cache)
+        assert got == _brute_force_bytes(wl, wl.seq_lens, cache), (wl.seq_lens, cache)
