@@ -18,8 +18,11 @@
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned and allocated by the caller. The
- *     library never allocates, frees or synchronises; every call is asynchronous on
- *     the given stream (NULL = the legacy default stream).
+ *     library never allocates or frees device memory at call time and never
+ *     synchronises; every call is asynchronous on the given stream (NULL = the legacy
+ *     default stream). (kv4_decode_step creates one stream and two events per host
+ *     thread and device on first use; kv4_decode_attention_noalloc uses a fixed
+ *     device array of the library's own.)
  *   - Arguments are checked on the host before anything is launched; a failed check
  *     returns a negative kv4_status and launches nothing.
  *   - Data-dependent checks run on the device: a kernel that meets a bad page id,
