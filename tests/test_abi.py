@@ -223,3 +223,29 @@ def test_plain_c_program_uses_the_abi(kv4, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
 
+
+def test_binding_structs_match_the_c_layout(kv4, tmp_path):
+    """The ctypes structures of the Python binding against the C compiler's layout of
+    the header's structs (sizes and every field offset)."""
+    exe = tmp_path / "c_abi_layout"
+    build = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I",
+                            os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "c_abi_layout.c"), "-o", str(exe)],
+                           capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60).stdout
+    c_layout = dict((k, int(v)) for k, v in (line.rsplit(" ", 1) for line in out.splitlines()))
+    py = {"kv4_config": kv4.Config, "kv4_int4_pool": kv4.Int4Pool,
+          "kv4_int8_side": kv4.Int8Side, "kv4_batch": kv4.Batch,
+          "kv4_paged_pool": kv4.PagedPool}
+    checked = 0
+    for key, val in c_layout.items():
+        kind, name = key.split(" ", 1)
+        if kind == "sizeof":
+            assert ctypes.sizeof(py[name]) == val, name
+        else:
+            struct, field = name.split(".")
+            assert getattr(py[struct], field).offset == val, name
+        checked += 1
+    assert checked == 5 + 9 + 5 + 10 + 7 + 5
+
