@@ -93,3 +93,28 @@ def test_plain_reciprocal_product_is_not_enough():
             if rn32(Fraction(float(a)) * Fraction(float(y))) != exact(a, b):
                 misses += 1
     assert misses > 0
+
+
+def test_rounding_by_the_magic_add_and_the_code_extraction():
+    """The kernels round a quotient q to the nearest-even integer by one binary32 add,
+    y = q + 1.5*2^23 (the add itself rounds to an integer for |q| < 2^22), and read the
+    code from y's bits: the low nibble is the INT4 code for results in [0, 15], the low
+    byte the int8 code (two's complement) for results in [-127, 127]; two INT4 codes
+    pack into a byte as y_even + (y_odd << 4)."""
+    rng = np.random.default_rng(4)
+    magic = np.float32(12582912.0)
+    q = np.concatenate([rng.uniform(-200, 200, 20000),
+                        np.arange(-255, 256) / 2.0]).astype(np.float32)  # includes ties
+    y = (q + magic).astype(np.float32)
+    assert np.array_equal(y - magic, np.rint(q))             # nearest-even integer
+    bits = y.view(np.uint32)
+    r = np.rint(q).astype(np.int64)
+    m4 = (r >= 0) & (r <= 15)
+    assert np.array_equal(bits[m4] & 0xF, r[m4])
+    m8 = (r >= -127) & (r <= 127)
+    low = (bits[m8] & 0xFF).astype(np.uint8).view(np.int8)
+    assert np.array_equal(low, r[m8].astype(np.int8))
+    ce, co = rng.integers(0, 16, 1000), rng.integers(0, 16, 1000)
+    ye = (ce.astype(np.float32) + magic).view(np.uint32).astype(np.uint64)
+    yo = (co.astype(np.float32) + magic).view(np.uint32).astype(np.uint64)
+    assert np.array_equal((ye + (yo << 4)) & 0xFF, ce | (co << 4))
