@@ -47,3 +47,29 @@ def test_fp16_products_with_subnormal_codes_are_exact_in_fp32():
     prod32 = p.astype(np.float32) * code.astype(np.float32)
     assert np.array_equal(prod32.astype(np.float64),
                           p.astype(np.float64) * c * 2.0 ** -24)
+
+
+def test_fixed_point_query_split():
+    """The query in 15-bit fixed point (the integer QK^T): with 2^e the step such that
+    max|q| < 2^(e+14), each element is rounded to n = rint(q / 2^e), |n| <= 2^14, split
+    into a signed high byte and an unsigned low byte, n = 256 hi + lo; the rounding is
+    at most 2^-14 max|q|, and elements of magnitude at least 2^7 steps (a power of two
+    between max|q|/128 and max|q|/64: their 8 significant bf16 bits then lie on the
+    step grid) are exact."""
+    rng = np.random.default_rng(2)
+    for scale in (1e-30, 1e-3, 1.0, 7.5, 2e6):
+        q = (rng.standard_normal(128) * scale).astype(np.float32)
+        q = (q.view(np.uint32) & 0xFFFF0000).view(np.float32)  # bf16 values
+        amax = float(np.abs(q).max())
+        _, ex = np.frexp(amax)  # amax < 2^ex
+        step = 2.0 ** (int(ex) - 14)
+        n = np.rint(q.astype(np.float64) / step).astype(np.int64)
+        assert np.abs(n).max() <= 2 ** 14
+        lo, hi = n & 0xFF, n >> 8
+        assert np.all((hi >= -128) & (hi <= 127)) and np.all((lo >= 0) & (lo <= 255))
+        assert np.array_equal(256 * hi + lo, n)
+        err = np.abs(n * step - q.astype(np.float64))
+        assert err.max() <= 2.0 ** -14 * amax
+        big = np.abs(q) >= 128 * step
+        assert np.all(err[big] == 0)
+        assert 128 * step > amax / 128 and 128 * step <= amax / 64
