@@ -135,7 +135,14 @@ def _check(status: int, what: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor argument (None -> NULL). The library reads every array
+    densely from its first element, so a tensor must be a contiguous CUDA tensor."""
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("kv4 arguments must be contiguous CUDA tensors "
+                         f"(got device={t.device}, contiguous={t.is_contiguous()})")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):

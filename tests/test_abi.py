@@ -249,3 +249,11 @@ def test_binding_structs_match_the_c_layout(kv4, tmp_path):
         checked += 1
     assert checked == 5 + 9 + 5 + 10 + 7 + 5
 
+
+def test_binding_refuses_host_or_strided_tensors(kv4):
+    """The binding passes bare pointers, so it refuses tensors the library would misread."""
+    import torch
+    assert kv4._ptr(None) is None
+    with pytest.raises(ValueError):
+        kv4._ptr(torch.zeros(4, 4))  # host memory
+
