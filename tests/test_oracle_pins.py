@@ -174,6 +174,41 @@ def test_int4_codes_are_the_exact_nearest_level():
     assert near_tie < 0.01 * codes.size
 
 
+def test_exact_ties_round_to_even():
+    """Quotients that are exact half-integers take the even neighbour, for INT4 and INT8
+    alike. The groups are built so that the stored scale is a power of two s (INT4: min
+    m*s and max (m+15)*s; INT8: amax 127*s) and the other values sit at (k + 1/2)*s, so
+    every quotient is exactly k + 1/2 and representable: no rounding of the quotient
+    itself can hide the tie rule."""
+    checked4 = checked8 = 0
+    for e in range(-6, 3):
+        s = 2.0 ** e
+        for m in (0, -3, 2):
+            g = np.zeros(32, np.float32)
+            g[0], g[1] = m * s, (m + 15) * s
+            ks = np.arange(30) % 15
+            g[2:] = (m + ks + 0.5) * s
+            assert np.array_equal(_bf16(g), g)
+            x = np.zeros(128, np.float32)
+            x[:32] = g
+            codes, sc, mn = O.quantize_int4(x)
+            assert float(sc[0]) == s and float(mn[0]) == m * s
+            want = [0, 15] + [k if k % 2 == 0 else k + 1 for k in ks]
+            assert codes[:32].tolist() == want, (e, m)
+            checked4 += 30
+        row = np.zeros(128, np.float32)
+        row[0] = 127 * s
+        ks = np.arange(-63, 64)  # both parities, both signs
+        row[1:1 + len(ks)] = (ks + 0.5) * s
+        assert np.array_equal(_bf16(row), row)
+        c8, s8 = O.quantize_int8(row)
+        assert float(s8) == s
+        want8 = [k if k % 2 == 0 else k + 1 for k in ks]
+        assert c8[0] == 127 and c8[1:1 + len(ks)].tolist() == want8, e
+        checked8 += len(ks)
+    assert checked4 > 500 and checked8 > 500
+
+
 def test_int4_reconstruction_bound_and_special_groups():
     rng = np.random.default_rng(2)
     G = _groups(rng, 120).reshape(-1, 128)
