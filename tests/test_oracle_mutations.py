@@ -1,6 +1,6 @@
 """The oracle's pins catch plausible mistakes.
 
-Each case below plants one mistake in the CPU oracle (on the CPU, by replacing one of
+Each of the 31 cases below plants one mistake in the CPU oracle (on the CPU, by replacing one of
 its functions for the duration of the case: a dropped term, a wrong sign, index or
 operand, another rounding rule, an off-by-one region edge) and checks that the pins of
 ``test_oracle_pins.py`` named beside it fail. A pin set that let such a mistake through
@@ -182,6 +182,46 @@ def _expected_pages_slot_shifted(rec, L, page_row):
                        for a in arrs) for pid, arrs in pages.items()}
 
 
+def _records_v_from_k(k, v, reading="A"):
+    """V records quantised from the K stream."""
+    return _orig["token_records"](k, k, reading)
+
+
+def _side_short_context_in_ring(rec, L, S, R):
+    """While the context is shorter than the sink count, tokens go to the ring instead
+    of the sink store (sink membership decided by the length, not the position)."""
+    return _orig["expected_side"](rec, L, S if L >= S else 0, R)
+
+
+def _side_ring_one_short(rec, L, S, R):
+    """A ring that keeps one position fewer than the recent window."""
+    return _orig["expected_side"](rec, L, S, R - 1 if R > 1 else R)
+
+
+def _int8_tensor_amax(x):
+    """INT8 scale from the largest magnitude of the whole tensor, not of each row."""
+    x = np.asarray(x, dtype=np.float32)
+    scale_h = O.to_f16(np.full(x.shape[:-1], np.abs(x).max(), np.float32) / np.float32(127.0))
+    s32 = scale_h.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        codes = np.clip(np.rint(x / s32), -127, 127)
+    return np.where(s32 == 0, 0, codes).astype(np.int8), scale_h
+
+
+def _int4_interleaved_groups(x):
+    """INT4 groups of every fourth dim instead of 32 consecutive dims."""
+    x = np.asarray(x, dtype=np.float32)
+    D = x.shape[-1]
+    perm = np.arange(D).reshape(D // O.GROUP, O.GROUP).T.reshape(-1)
+    codes, scale_h, min_h = _orig["quantize_int4"](x[..., perm])
+    return codes[..., np.argsort(perm)], scale_h, min_h
+
+
+def _pack_int8_transposed(codes):
+    """INT8 strips holding every eighth dim instead of 16 consecutive dims."""
+    return codes.reshape(codes.shape[:-1] + (16, 8)).swapaxes(-1, -2)
+
+
 MUTATIONS = {
     # name: (oracle function, replacement, pins that must fail)
     "to_f16 truncates": ("to_f16", _to_f16_truncating,
@@ -239,6 +279,19 @@ MUTATIONS = {
                               ["test_baseline_references_reduce_to_pinned_cases"]),
     "page slots shifted": ("expected_pages", _expected_pages_slot_shifted,
                            ["test_expected_pages_layout"]),
+    "V records from K": ("token_records", _records_v_from_k,
+                         ["test_expected_pages_layout", "test_token_record_layouts_by_hand"]),
+    "short context in the ring": ("expected_side", _side_short_context_in_ring,
+                                  ["test_ring_window_matches_sequential_appends"]),
+    "ring one short": ("expected_side", _side_ring_one_short,
+                       ["test_ring_window_matches_sequential_appends"]),
+    "INT8 scale per tensor": ("quantize_int8", _int8_tensor_amax,
+                              ["test_int8_exact_nearest_and_symmetry"]),
+    "INT4 groups interleaved": ("quantize_int4", _int4_interleaved_groups,
+                                ["test_int4_golden_group_a", "test_token_record_layouts_by_hand",
+                                 "test_int4_codes_are_the_exact_nearest_level"]),
+    "INT8 strips transposed": ("pack_int8_token", _pack_int8_transposed,
+                               ["test_token_record_layouts_by_hand"]),
 }
 
 

@@ -294,24 +294,32 @@ def test_protected_set_over_144_is_rejected():
 
 
 def test_ring_window_matches_sequential_appends():
-    """expected_side's window formula equals literally appending tokens one by one."""
+    """expected_side's window formula equals literally appending tokens one by one: K
+    and V, codes and scales, sink store and ring, including contexts shorter than the
+    sink count and the empty context."""
     rng = np.random.default_rng(4)
-    for (S, R, L) in [(4, 32, 37), (4, 32, 20), (16, 128, 300), (0, 16, 50), (3, 5, 5), (2, 8, 9)]:
+    for (S, R, L) in [(4, 32, 37), (4, 32, 20), (16, 128, 300), (0, 16, 50), (3, 5, 5),
+                      (2, 8, 9), (16, 128, 5), (4, 32, 3), (4, 32, 0)]:
         k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
-        rec = O.token_records(k, k)
+        v = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+        rec = O.token_records(k, v)
         sim_sink, sim_ring = {}, {}
         for pos in range(L):  # append procedure: sink slot pos, else ring slot pos mod R
             if pos < S:
                 sim_sink[pos] = pos
             else:
                 sim_ring[pos % R] = pos
-        sk, sks, _, _, rk, rks, _, _ = O.expected_side(rec, L, S, R)
-        for slot in range(sk.shape[1] * 16):
-            want = rec["k8"][sim_sink[slot]] if slot in sim_sink else 0
-            assert np.array_equal(sk[:, slot // 16, :, slot % 16, :], np.broadcast_to(want, (2, 8, 16)))
-        for slot in range(rk.shape[1] * 16):
-            want = rec["ks"][sim_ring[slot]] if slot in sim_ring else 0
-            assert np.array_equal(rks[:, slot], np.broadcast_to(want, (2,)))
+        sk, sks, sv, svs, rk, rks, rv, rvs = O.expected_side(rec, L, S, R)
+        for sim, arrays in ((sim_sink, ((sk, sks, "k"), (sv, svs, "v"))),
+                            (sim_ring, ((rk, rks, "k"), (rv, rvs, "v")))):
+            for codes, scales, name in arrays:
+                for slot in range(codes.shape[1] * 16):
+                    pos = sim.get(slot)
+                    want_c = rec[name + "8"][pos] if pos is not None else 0
+                    want_s = rec[name + "s"][pos] if pos is not None else 0
+                    assert np.array_equal(codes[:, slot // 16, :, slot % 16, :],
+                                          np.broadcast_to(want_c, (2, 8, 16))), (S, R, L, slot)
+                    assert np.array_equal(scales[:, slot], np.broadcast_to(want_s, (2,)))
 
 
 # --------------------------------------------------------------------------
@@ -537,15 +545,54 @@ def test_expected_pages_layout():
     rng = np.random.default_rng(11)
     L = 21
     k = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
-    rec = O.token_records(k, k)
+    v = _bf16(rng.normal(0, 1, (L, 2, 128)).astype(np.float32))
+    rec = O.token_records(k, v)
     pages = O.expected_pages(rec, L, np.array([7, 3]))
     assert set(pages) == {7, 3}
-    kc, kp, _, _ = pages[3]
+    kc, kp, vc, vp = pages[3]
     # page 3 holds positions 16..20 in slots 0..4, zeros after
     assert np.array_equal(kc[:, :, :5, :], rec["k4"][16:21].transpose(1, 2, 0, 3))
     assert np.all(kc[:, :, 5:, :] == 0) and np.all(kp[:, 5:] == 0)
-    # nibble order: dim 2i in the low nibble of byte i
-    c, s, m = O.quantize_int4(k[16])
-    assert np.array_equal(kc[1, 2, 0, 5] & 0xF, c[1, 64 + 10])
-    assert np.array_equal(kc[1, 2, 0, 5] >> 4, c[1, 64 + 11])
-    assert kp[1, 0, 2, 0] == s[1, 2].view(np.uint16) and kp[1, 0, 2, 1] == m[1, 2].view(np.uint16)
+    assert np.all(vc[:, :, 5:, :] == 0) and np.all(vp[:, 5:] == 0)
+    # nibble order: dim 2i in the low nibble of byte i; K slots from k, V slots from v
+    for codes, params, x in ((kc, kp, k), (vc, vp, v)):
+        c, s, m = O.quantize_int4(x[16])
+        assert np.array_equal(codes[1, 2, 0, 5] & 0xF, c[1, 64 + 10])
+        assert np.array_equal(codes[1, 2, 0, 5] >> 4, c[1, 64 + 11])
+        assert params[1, 0, 2, 0] == s[1, 2].view(np.uint16)
+        assert params[1, 0, 2, 1] == m[1, 2].view(np.uint16)
+
+
+def test_token_record_layouts_by_hand():
+    """Records of tokens whose codes are known in advance. INT4: each group holds its
+    min m and max m + 15s with s a power of two, so the scale is s and dim d gets code
+    d mod 16 (K) or 15 - d mod 16 (V); byte i of group g packs dims 32g+2i (low nibble)
+    and 32g+2i+1 (high nibble). INT8: amax 127s, dim d of K at (d - 63)s (dim 127 at
+    127s), of V at (63 - d)s; byte i of strip c is the code of dim 16c+i."""
+    s = 2.0 ** -3
+    d = np.arange(128)
+    k4 = ((d % 16) * s - 1.0).astype(np.float32)
+    v4 = ((15 - d % 16) * s + 0.5).astype(np.float32)
+    rec = O.token_records(k4[None, None], v4[None, None])
+    for name, code_of in (("k", lambda i: i % 16), ("v", lambda i: 15 - i % 16)):
+        strips = rec[name + "4"][0, 0]
+        for g in range(4):
+            for i in range(16):
+                lo, hi = code_of(32 * g + 2 * i), code_of(32 * g + 2 * i + 1)
+                assert strips[g, i] == lo | (hi << 4), (name, g, i)
+        params = rec[name + "p"][0, 0]
+        assert np.all(params[:, 0] == np.float16(s).view(np.uint16))
+    assert np.all(rec["kp"][0, 0, :, 1] == np.float16(-1.0).view(np.uint16))
+    assert np.all(rec["vp"][0, 0, :, 1] == np.float16(0.5).view(np.uint16))
+    k8 = np.where(d < 127, (d - 63) * s, 127 * s).astype(np.float32)
+    v8 = ((63 - d) * s).astype(np.float32)
+    v8[127] = -127 * s
+    rec = O.token_records(k8[None, None], v8[None, None])
+    want_k = np.where(d < 127, d - 63, 127)
+    want_v = np.where(d < 127, 63 - d, -127)
+    for name, want in (("k", want_k), ("v", want_v)):
+        strips = rec[name + "8"][0, 0]
+        for c in range(8):
+            for i in range(16):
+                assert strips[c, i] == want[16 * c + i], (name, c, i)
+        assert rec[name + "s"][0, 0] == np.float16(s).view(np.uint16)
