@@ -257,3 +257,46 @@ def test_binding_refuses_host_or_strided_tensors(kv4):
     with pytest.raises(ValueError):
         kv4._ptr(torch.zeros(4, 4))  # host memory
 
+
+
+def _prototypes():
+    """{name: (return type, [parameter declarations])} of the header's functions."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for m in re.finditer(r"([A-Za-z_][\w \t\*]*?)\b(kv4_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
+        params = [" ".join(p.split()) for p in m.group(3).split(",")]
+        out[m.group(2)] = (" ".join(m.group(1).split()), [] if params == ["void"] else params)
+    return out
+
+
+def test_binding_signatures_match_the_header(kv4):
+    """Every function the binding declares takes as many parameters as the header's
+    prototype, each of the same kind and width: pointers (and the stream handle) as
+    pointers, int32_t as 32-bit, size_t as size_t, enums as int; and returns the
+    prototype's type."""
+    protos = _prototypes()
+    assert set(protos) == set(kv4.EXPORTS)
+    ptr_types = (ctypes.c_void_p, ctypes._Pointer)
+
+    def kind(ct):
+        if ct in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(ct, ptr_types):
+            return "pointer"
+        return {ctypes.c_int32: "int32", ctypes.c_int: "int32", ctypes.c_size_t: "size_t"}[ct]
+
+    def c_kind(decl):
+        if "*" in decl or decl.startswith("kv4_stream_t"):
+            return "pointer"
+        if decl.startswith("size_t"):
+            return "size_t"
+        if decl.split()[0] in ("int32_t", "kv4_status", "kv4_baseline_format"):
+            return "int32"
+        raise AssertionError(f"unclassified parameter {decl!r}")
+
+    for name, (ret, params) in protos.items():
+        fn = getattr(kv4._lib, name)
+        assert len(fn.argtypes) == len(params), name
+        for decl, ct in zip(params, fn.argtypes):
+            assert kind(ct) == c_kind(decl), (name, decl, ct)
+        assert kind(fn.restype) == c_kind(ret), (name, ret, fn.restype)
