@@ -88,7 +88,8 @@ typedef enum {
 #define KV4_DEVERR_SIDE_IDX 4u   /* sink_idx / ring_idx outside the side store */
 #define KV4_DEVERR_Q_RANGE 8u    /* reserved: no longer raised (queries enter the dot
                                     products in per-query fixed point, any finite value) */
-#define KV4_DEVERR_WORKSPACE 16u /* the batch needs more work items than the workspace holds */
+#define KV4_DEVERR_WORKSPACE 16u /* the batch needs more work items than the workspace holds
+                                    (the call then writes zero outputs, lse = -inf) */
 #define KV4_DEVERR_TIMEOUT 32u   /* a bounded wait for an async copy gave up */
 
 #define KV4_MAX_PROTECTED 144

@@ -247,7 +247,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
-    w.unit_offsets[B * H] = H * tot[0];
+    // a workspace too small leaves every unit empty (all offsets 0): the merge then
+    // reads no partial state and writes zero outputs with lse = -inf
+    w.unit_offsets[B * H] = fits ? H * tot[0] : 0;
     *w.n_items = fits ? te_all : 0;
     *w.counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);

@@ -435,13 +435,18 @@ def test_device_error_flags_without_faulting():
     torch.cuda.synchronize()
     assert int(err.item()) & 1
     # a workspace planned for shorter sequences overflows (3 regions per sequence needed,
-    # room for 2) -> flag, no fault
+    # room for 2) -> flag, no fault; every unit is left empty, so the merge reads no
+    # partial state and writes zeros with lse = -inf
     err.zero_()
     small = kv4.BatchTensors(sess.page_table, sess.step_lens[0], sess.sink_idx, sess.ring_idx, 16)
     ws = torch.empty(kv4.workspace_size(sess.cfg, 2, 16), dtype=torch.uint8, device="cuda")
-    kv4.decode_attention(sess.cache, small, sess.q[0], sess.out, ws, err=err)
+    sess.out.fill_(1.0)
+    o32 = torch.full((2, 8, 128), 7.0, dtype=torch.float32, device="cuda")
+    lse = torch.zeros((2, 8), dtype=torch.float32, device="cuda")
+    kv4.decode_attention(sess.cache, small, sess.q[0], sess.out, ws, o32, lse, err)
     torch.cuda.synchronize()
     assert int(err.item()) & 16
+    assert torch.all(sess.out == 0) and torch.all(o32 == 0) and torch.all(torch.isneginf(lse))
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (16, 2)])
