@@ -229,9 +229,10 @@ MUTATIONS = {
     "to_f16 overflows to inf": ("to_f16", _to_f16_unsaturated,
                                 ["test_to_f16_is_round_nearest_even_with_saturation"]),
     "INT4 rounds half up": ("quantize_int4", _int4_with(round_fn=_half_up),
-                            ["test_exact_ties_round_to_even"]),
+                            ["test_int4_golden_group_a", "test_exact_ties_round_to_even"]),
     "INT4 rounds half away from zero": ("quantize_int4", _int4_with(round_fn=_half_away),
-                                        ["test_exact_ties_round_to_even"]),
+                                        ["test_int4_golden_group_a",
+                                         "test_exact_ties_round_to_even"]),
     "INT4 range over 16 levels": ("quantize_int4", _int4_with(levels=16.0),
                                   ["test_int4_golden_group_a",
                                    "test_int4_codes_are_the_exact_nearest_level"]),
