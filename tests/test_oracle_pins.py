@@ -596,3 +596,44 @@ def test_token_record_layouts_by_hand():
             for i in range(16):
                 assert strips[c, i] == want[16 * c + i], (name, c, i)
         assert rec[name + "s"][0, 0] == np.float16(s).view(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# order and end points of the quantisers, on generated bf16 rows
+# --------------------------------------------------------------------------
+
+def test_codes_preserve_order_and_reach_the_end_levels():
+    """Rounding to the nearest level is monotone, so within a group a larger value never
+    gets a smaller code, and INT8 codes keep the order of the values. The group minimum
+    gets code 0: its stored fp16 rounding is within half an fp16 step of it (exact for
+    bf16 values in the fp16 normal range) and a non-zero scale is at least one step. When the stored scale is an fp16 normal number (at
+    least 2^-14) its relative rounding error is at most 2^-11, so the maximum's quotient
+    is 15 (INT8: 127) within 0.01 and the maximum gets code 15 (the largest magnitude
+    +-127). A subnormal scale has only 2^-24 absolute precision, and there the end code
+    may be one or more levels short (found by this test: an INT8 row with amax 2^-11
+    gives 126). Rows drawn by hypothesis over magnitudes from 2^-12 to 2^12."""
+    from hypothesis import given, settings, strategies as st
+
+    rows = st.lists(st.floats(min_value=-1.0, max_value=1.0, allow_nan=False, width=32),
+                    min_size=128, max_size=128)
+
+    @settings(max_examples=300, derandomize=True, deadline=None)
+    @given(rows, st.integers(min_value=-12, max_value=12))
+    def check(vals, e):
+        x = _bf16(np.array(vals, np.float32) * np.float32(2.0 ** e))
+        codes, sc, mn = O.quantize_int4(x)
+        for g in range(4):
+            xs, cs = x[32 * g:32 * g + 32], codes[32 * g:32 * g + 32].astype(int)
+            order = np.argsort(xs, kind="stable")
+            assert np.all(np.diff(cs[order]) >= 0)
+            assert cs[np.argmin(xs)] == 0
+            if sc[g] >= 2.0 ** -14:
+                assert cs[np.argmax(xs)] == 15
+        c8, s8 = O.quantize_int8(x)
+        order = np.argsort(x, kind="stable")
+        assert np.all(np.diff(c8.astype(int)[order]) >= 0)
+        if s8 >= 2.0 ** -14:
+            i = np.argmax(np.abs(x))
+            assert c8[i] == (127 if x[i] > 0 else -127)
+
+    check()
