@@ -141,7 +141,8 @@ typedef struct {
                                 a prompt may share one); may be NULL if S == 0 */
   const int32_t *ring_idx;   /* [num_seqs]: recent ring of each sequence; NULL = identity */
   int32_t num_seqs;
-  int32_t max_seq_len;       /* host-side upper bound on seq_lens, sizes the workspace */
+  int32_t max_seq_len;       /* host-side upper bound on seq_lens, sizes the workspace; a
+                                longer sequence may overflow it (KV4_DEVERR_WORKSPACE) */
 } kv4_batch;
 
 /*
