@@ -300,3 +300,23 @@ def test_binding_signatures_match_the_header(kv4):
         for decl, ct in zip(params, fn.argtypes):
             assert kind(ct) == c_kind(decl), (name, decl, ct)
         assert kind(fn.restype) == c_kind(ret), (name, ret, fn.restype)
+
+
+def test_workspace_fallback_to_longest_chunks_always_fits(kv4):
+    """A workspace sized for (num_seqs, max_seq_len) with the automatic chunk choice also
+    holds any smaller or equal batch split into 64-page chunks, the fallback the call
+    takes when that batch's own automatic split would need more room (automatic sizes
+    themselves are not monotone: longer sequences get longer chunks); and 64-page sizes
+    grow with the batch. Checked on random shapes for four head configurations."""
+    import numpy as np
+    rng = np.random.default_rng(3)
+    for hq, hkv, s, r in ((32, 8, 16, 128), (8, 2, 4, 32), (16, 2, 0, 0), (12, 3, 7, 13)):
+        auto = _cfg(kv4, num_q_heads=hq, num_kv_heads=hkv, num_sinks=s, num_recent=r)
+        c64 = _cfg(kv4, num_q_heads=hq, num_kv_heads=hkv, num_sinks=s, num_recent=r,
+                   chunk_pages=64)
+        for _ in range(200):
+            B1, L1 = int(rng.integers(1, 3000)), int(rng.integers(0, 20000))
+            B2, L2 = int(rng.integers(1, B1 + 1)), int(rng.integers(0, L1 + 1))
+            big = kv4.workspace_size(auto, B1, L1)
+            assert big >= kv4.workspace_size(c64, B2, L2), (hq, hkv, B1, L1, B2, L2)
+            assert kv4.workspace_size(c64, B1, L1) >= kv4.workspace_size(c64, B2, L2)
