@@ -1,6 +1,6 @@
 """The oracle's pins catch plausible mistakes.
 
-Each of the 31 cases below plants one mistake in the CPU oracle (on the CPU, by replacing one of
+Each of the 35 cases below plants one mistake in the CPU oracle (on the CPU, by replacing one of
 its functions for the duration of the case: a dropped term, a wrong sign, index or
 operand, another rounding rule, an off-by-one region edge) and checks that the pins of
 ``test_oracle_pins.py`` named beside it fail. A pin set that let such a mistake through
@@ -42,18 +42,22 @@ def _to_f16_unsaturated(x):
         return np.asarray(x, dtype=np.float32).astype(np.float16)
 
 
-def _int4_with(round_fn=np.rint, levels=15.0, top=15):
+def _int4_with(round_fn=np.rint, levels=15.0, top=15, reciprocal=False, range_f16=False):
     """quantize_int4 with one step changed: the integer rounding, the number of
-    levels the range is divided into, or the top code of the clamp."""
+    levels the range is divided into, the top code of the clamp, the quotient taken as
+    a product with the rounded reciprocal of the scale, or the range rounded to fp16
+    before the division (the scale rounded twice)."""
     def quantize_int4(x):
         x = np.asarray(x, dtype=np.float32)
         g = x.reshape(x.shape[:-1] + (x.shape[-1] // O.GROUP, O.GROUP))
         mn, mx = g.min(axis=-1), g.max(axis=-1)
         min_h = O.to_f16(mn)
-        scale_h = O.to_f16((mx - mn) / np.float32(levels))
+        rng = O.to_f16(mx - mn).astype(np.float32) if range_f16 else mx - mn
+        scale_h = O.to_f16(rng / np.float32(levels))
         s32 = scale_h.astype(np.float32)[..., None]
-        with np.errstate(divide="ignore", invalid="ignore"):
-            q = (g - min_h.astype(np.float32)[..., None]) / s32
+        with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+            num = g - min_h.astype(np.float32)[..., None]
+            q = num * (np.float32(1.0) / s32) if reciprocal else num / s32
             codes = np.clip(round_fn(q), 0, top)
         codes = np.where(s32 == 0, 0, codes)
         return codes.reshape(x.shape).astype(np.uint8), scale_h, min_h
@@ -71,6 +75,15 @@ def _int8_with(round_fn=np.rint, div=127.0):
         codes = np.where(s32 == 0, 0, codes)
         return codes.astype(np.int8), scale_h
     return quantize_int8
+
+
+def _near_ties_up(q):
+    """Nearest integer, except that a quotient within 2^-9 of a half-integer (but not
+    exactly on it) goes to the upper neighbour: a tie rule applied with a tolerance."""
+    a = np.abs(q)
+    fr = a - np.floor(a)
+    near = (np.abs(fr - np.float32(0.5)) <= np.float32(2.0 ** -9)) & (fr != np.float32(0.5))
+    return np.where(near, np.sign(q) * np.ceil(a), np.rint(q))
 
 
 def _half_up(q):
@@ -239,6 +252,14 @@ MUTATIONS = {
     "INT4 top code 14": ("quantize_int4", _int4_with(top=14),
                          ["test_int4_golden_group_a",
                           "test_int4_reconstruction_bound_and_special_groups"]),
+    "INT4 near-ties rounded up": ("quantize_int4", _int4_with(round_fn=_near_ties_up),
+                                  ["test_int4_codes_are_the_exact_nearest_level"]),
+    "INT4 quotient by reciprocal product": ("quantize_int4", _int4_with(reciprocal=True),
+                                            ["test_exact_ties_at_scales_without_an_exact_reciprocal"]),
+    "INT4 scale rounded twice": ("quantize_int4", _int4_with(range_f16=True),
+                                 ["test_int4_codes_are_the_exact_nearest_level"]),
+    "INT8 near-ties rounded up": ("quantize_int8", _int8_with(round_fn=_near_ties_up),
+                                  ["test_int8_exact_nearest_and_symmetry"]),
     "INT8 rounds half away from zero": ("quantize_int8", _int8_with(round_fn=_half_away),
                                         ["test_int8_golden_rows", "test_exact_ties_round_to_even"]),
     "INT8 rounds half up": ("quantize_int8", _int8_with(round_fn=_half_up),
