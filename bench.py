@@ -360,10 +360,13 @@ def run_gpu(args, rank, world, local_rank):
     wl = rank_workload(args.workload, rank, args.sinks, args.recent)
     if args.demotion == "B":
         wl.name += "-demotionB"
+    if args.prefix == "shared" and args.cache == "kv4":
+        wl.name += "-prefix-shared"
     W, K = args.warmup, args.steps
     # one session per layer (same lengths and paging, own data); they share a workspace
     if args.cache == "kv4":
-        make_session = lambda *a, **kw: DecodeSession(*a, demotion=args.demotion, **kw)
+        make_session = lambda *a, **kw: DecodeSession(*a, demotion=args.demotion,
+                                                      prefix=args.prefix, **kw)
     else:
         fmt = kv4.BASELINE_BF16 if args.cache == "bf16" else kv4.BASELINE_KV8
         make_session = lambda *a, **kw: BaselineSession(*a, fmt=fmt, **kw)
@@ -520,14 +523,14 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
-            "gpu_launches": 4 * K * nl,
+            "gpu_launches": (5 if args.cache == "kv4" and args.prefix == "shared" else 4) * K * nl,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
         if prefill is not None:
             line["prefill"] = {**prefill, "peak_gbs": peak, "frac": prefill["gbs"] / peak}
         print(json.dumps(line), flush=True)
-    del g_app, g_att, layers
+    del layers
     if world > 1:
         dist.destroy_process_group()
 
@@ -545,6 +548,9 @@ def main(argv=None):
                     help="KV4-RL cache (default) or a comparison cache: all-INT8 or BF16")
     ap.add_argument("--demotion", default="A", choices=["A", "B"],
                     help="INT4 copies from the bf16 input (A) or from the INT8 copy (B)")
+    ap.add_argument("--prefix", default="off", choices=["off", "shared"],
+                    help="shared-prefix read: pages shared by a group's sequences read by "
+                         "every sequence (off, the default) or once per group (shared)")
     ap.add_argument("--sinks", type=int, default=None, help="override S (protection sweep)")
     ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
     ap.add_argument("--prefill", action="store_true",

@@ -110,7 +110,21 @@ typedef struct {
                            append (reading A, the default); 1 = the position's INT8 copy,
                            dequantised (reading B: what demotion out of the recent window
                            would write). Attention is the same for both. */
+  int32_t prefix_mode;  /* shared-prefix read (KV4_PREFIX_*): 0 = off (the default): every
+                           sequence reads all its pages on its own; 1 = shared: consecutive
+                           sequences whose page tables map their leading INT4 pages to the
+                           same physical pages -- the responses of one prompt -- form a
+                           group whose shared pages are read once per kv head for up to 16
+                           query heads of the group (4 sequences at GQA 4) and merged as one
+                           more region per sequence. Results agree within the attention
+                           tolerance either way (the regions differ, so the rounding does).
+                           On the 1024-sequence rollout batch the shared read removes 13 %
+                           of the attention kernel's time but costs more in its own kernel
+                           and in the sharing detection, so it is off by default. */
 } kv4_config;
+
+#define KV4_PREFIX_OFF 0
+#define KV4_PREFIX_SHARED 1
 
 typedef struct {
   uint8_t *k_codes;   /* see "INT4 pool" above */
@@ -312,6 +326,22 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
                                          const void *q, void *out, float *out_f32, float *lse,
                                          void *workspace, size_t ws_bytes, int32_t *err_flag,
                                          kv4_stream_t stream);
+
+/*
+ * Testing hook for the error path of the bounded waits. No passage of the pages defines
+ * it; it exists so that the library's tests can make a wait give up without any fault.
+ * The next kv4_decode_attention, kv4_decode_step or kv4_baseline_decode_attention call
+ * made by this host thread -- that one only -- withholds the first shared-memory copy of
+ * work item `item` of its attention kernel (nothing is issued for it, so nothing is in
+ * flight) and gives each bounded wait of its kernels `wait_limit` attempts (0 keeps the
+ * normal limit). The wait on the withheld copy gives up: the call ORs KV4_DEVERR_TIMEOUT
+ * into *err_flag, writes that work item's partial state as empty, lets the warp that held
+ * it take no further work, and computes the rest of the batch as usual; the call returns
+ * normally and the context stays usable. Work items are numbered in the order the
+ * attention's work list holds them (full INT4 chunks first, in sequence order). item < 0
+ * cancels a pending request.
+ */
+void kv4_test_withhold_copy(int32_t item, uint32_t wait_limit);
 
 /* Human-readable name of a status code (static string). */
 const char *kv4_status_string(kv4_status status);

@@ -13,7 +13,8 @@ namespace {
 kv4_status check_config(const kv4_config *cfg) {
   if (cfg == nullptr) return KV4_ERR_INVALID_ARG;
   if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_sinks < 0 ||
-      cfg->num_recent < 0 || cfg->chunk_pages < 0 || cfg->demotion < 0 || cfg->demotion > 1)
+      cfg->num_recent < 0 || cfg->chunk_pages < 0 || cfg->demotion < 0 || cfg->demotion > 1 ||
+      cfg->prefix_mode < 0 || cfg->prefix_mode > 1)
     return KV4_ERR_INVALID_ARG;
   if (cfg->head_dim != kv4::kHeadDim || cfg->page_size != kv4::kPage ||
       cfg->group_size != kv4::kGroup)
@@ -113,12 +114,31 @@ kv4_status make_view(const kv4_config *cfg, const kv4_int4_pool *pool, const kv4
   return KV4_OK;
 }
 
-// The comparison baselines have no protected set: the config is used with S = R = 0.
+// The comparison baselines have no protected set and no shared-prefix read: the config
+// is used with S = R = 0 and the prefix read off.
 kv4_config without_protection(const kv4_config *cfg) {
   kv4_config c = *cfg;
   c.num_sinks = 0;
   c.num_recent = 0;
+  c.prefix_mode = KV4_PREFIX_OFF;
   return c;
+}
+
+bool prefix_on(const kv4_config *cfg) { return cfg->prefix_mode == KV4_PREFIX_SHARED; }
+
+// kv4_test_withhold_copy: a one-shot setting of this host thread, taken by its next
+// attention call.
+struct WithheldCopy {
+  int32_t item = -1;
+  uint32_t wait_limit = 0;
+};
+thread_local WithheldCopy g_withheld;
+
+void take_test_hook(kv4::Workspace *w) {
+  if (g_withheld.item < 0) return;
+  w->fault_item = g_withheld.item;
+  if (g_withheld.wait_limit > 0) w->wait_limit = g_withheld.wait_limit;
+  g_withheld = WithheldCopy{};
 }
 
 kv4_status make_baseline_view(kv4_baseline_format fmt, const kv4_config *cfg,
@@ -159,15 +179,15 @@ kv4_status carve_workspace(const kv4_config *cfg, const kv4::CacheView &v,
                            const kv4_batch *batch, void *workspace, size_t ws_bytes,
                            kv4::Workspace *w) {
   size_t need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
-                                     chunk_of(cfg, batch->num_seqs, batch->max_seq_len), w,
-                                     workspace);
+                                     chunk_of(cfg, batch->num_seqs, batch->max_seq_len),
+                                     prefix_on(cfg), w, workspace);
   // A workspace sized for a larger batch or longer sequences (and so for longer automatic
   // chunks) may be too small for a finer automatic split of this one: fall back to the
   // longest chunks, for which any workspace sized with this config at larger or equal
   // (num_seqs, max_seq_len) is large enough.
   if (ws_bytes < need && cfg->chunk_pages == 0)
     need = kv4::workspace_bytes(batch->num_seqs, batch->max_seq_len, v.num_kv_heads, v.gqa,
-                                kv4::kMaxChunkPages, w, workspace);
+                                kv4::kMaxChunkPages, prefix_on(cfg), w, workspace);
   return ws_bytes < need ? KV4_ERR_WORKSPACE_TOO_SMALL : KV4_OK;
 }
 
@@ -218,7 +238,8 @@ size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_s
   if (check_config(cfg) != KV4_OK || num_seqs < 0 || max_seq_len < 0) return 0;
   return kv4::workspace_bytes(num_seqs, max_seq_len, cfg->num_kv_heads,
                               cfg->num_q_heads / cfg->num_kv_heads,
-                              chunk_of(cfg, num_seqs, max_seq_len), nullptr, nullptr);
+                              chunk_of(cfg, num_seqs, max_seq_len), prefix_on(cfg), nullptr,
+                              nullptr);
 }
 
 kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
@@ -252,8 +273,10 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   kv4::Workspace w;
   st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
+  take_test_hook(&w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  if (e == cudaSuccess) e = kv4::launch_prefix(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
@@ -278,6 +301,7 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   kv4::Workspace w;
   st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
+  take_test_hook(&w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // The second stream and its events are not created while the caller's stream is being
   // captured into a graph; a first call made there builds the work list on the caller's
@@ -302,6 +326,7 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
                            err_flag, s);
   // join, then the attention and the merge behind both
   if (e == cudaSuccess && ss != nullptr) e = cudaStreamWaitEvent(s, ss->join, 0);
+  if (e == cudaSuccess) e = kv4::launch_prefix(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
@@ -370,6 +395,7 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
   kv4::Workspace w;
   st = carve_workspace(&c, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
+  take_test_hook(&w);
   w.heads_per_warp = 1;  // one kv head per warp and entry
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
@@ -379,6 +405,11 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
                           static_cast<uint16_t *>(out), out_f32, lse, s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
+}
+
+void kv4_test_withhold_copy(int32_t item, uint32_t wait_limit) {
+  g_withheld.item = item < 0 ? -1 : item;
+  g_withheld.wait_limit = wait_limit;
 }
 
 const char *kv4_status_string(kv4_status status) {
@@ -393,6 +424,6 @@ const char *kv4_status_string(kv4_status status) {
   return "unknown status";
 }
 
-int32_t kv4_version(void) { return 400; }
+int32_t kv4_version(void) { return 500; }
 
 }  // extern "C"

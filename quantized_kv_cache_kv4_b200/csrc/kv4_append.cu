@@ -593,19 +593,18 @@ cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint1
   if (total_new == 0) return cudaSuccess;
   const int threads = 256;
   if (new_indptr != nullptr) {  // CSR rows: one thread per (row, kv head)
-    static int configured_device = -1;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev != configured_device) {
-      e = cudaFuncSetAttribute(append_rows_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(append_rows_kernel<true>,
+    static PerDevice configured;
+    int done = 0;
+    cudaError_t e = once_per_device(configured, [](int, int *v) {
+      cudaError_t r = cudaFuncSetAttribute(append_rows_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(append_rows_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsSmem);
-      if (e != cudaSuccess) return e;
-      configured_device = dev;
-    }
+      *v = 1;
+      return r;
+    }, &done);
+    if (e != cudaSuccess) return e;
     const long long warps = static_cast<long long>((total_new + 31) / 32) * c.num_kv_heads;
     const unsigned blocks =
         static_cast<unsigned>((warps * 32 + kRowsThreads - 1) / kRowsThreads);

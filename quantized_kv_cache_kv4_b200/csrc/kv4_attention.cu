@@ -5,8 +5,9 @@
 //
 // Kernels:
 //   plan_kernel  turns seq_lens into a work list. Region 0 of a sequence is its INT8
-//                protected set; regions 1.. are chunks of `chunk_pages` INT4 pages; one
-//                entry per region and one or two kv heads. Entries
+//                protected set; then the regions of its group's shared INT4 pages (if
+//                any); then chunks of `chunk_pages` of its own INT4 pages; one entry per
+//                region and one or two kv heads. Entries
 //                come in four classes (full chunks, long partial chunks, protected sets,
 //                short chunks) so that the longest work starts first.
 //   attn_kernel  persistent; every warp repeatedly takes one entry from an atomic counter
@@ -26,6 +27,13 @@
 //                N dimension (8) holds head A's queries in columns 0-3 and head B's in
 //                columns 4-7 (zeros in the other half of each B operand), so every lane's
 //                softmax and scaling work is useful.
+//   prefix_kernel the shared-prefix read (kv4_config.prefix_mode): consecutive sequences
+//                whose page tables map their leading INT4 pages to the same physical pages
+//                (the responses of one prompt, ai4snews summary, "Interpretation" para. 3:
+//                groups of eight responses) form a group; one warp reads each shared page
+//                of a kv head once for up to four members (16 query columns, two MMA N
+//                tiles) and writes one partial state per member, merged as an extra
+//                region. The members' own chunks start after the shared pages.
 //   merge_kernel one warp per (unit, query): fixed-order exact merge -> bf16 out; also
 //                the kernel behind kv4_regional_merge.
 #include <math_constants.h>
@@ -42,7 +50,9 @@ namespace kv4 {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanSeqsPerCta = 32;  // sequences per CTA, until kPlanMaxCtas is reached
 constexpr int kPlanMaxCtas = 148;
-constexpr int kScanN = 5;            // values scanned together per sequence
+constexpr int kScanN = 6;            // values scanned together per sequence
+constexpr int kPrefixCols = 16;      // query columns of one prefix entry (two MMA N tiles)
+constexpr int kMaxPrefixPages = 256;  // leading INT4 pages compared for sharing
 
 // Exclusive block-wide scan of kScanN values at once (warp shuffles + one warp over the
 // 32 warp totals per value); totals returned in tot.
@@ -105,14 +115,115 @@ __device__ int key_rank(int key, int (*cnt)[33], int *chunk_tot) {
   return rank;
 }
 
+// Inclusive block-wide max-scan of v (1024 threads); warp_max: shared scratch [32].
+__device__ int block_max_scan(int v, int *warp_max) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v = max(v, y);
+  }
+  if (lane == 31) warp_max[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    int t = warp_max[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, off);
+      if (lane >= off) t = max(t, y);
+    }
+    warp_max[lane] = t;
+  }
+  __syncthreads();
+  if (wid > 0) v = max(v, warp_max[wid - 1]);
+  __syncthreads();
+  return v;
+}
+
+// Pages at the head of sequence b's INT4 range that hold the same physical pages as in
+// sequence b-1's page table: returns p0 plus the number of equal page ids from page p0 on,
+// compared over the pages holding positions of both sequences (at most kMaxPrefixPages).
+__device__ int pages_shared_with_prev(const CacheView &c, int b, int p0) {
+  const int cap = c.max_pages * kPage;
+  int L1 = c.seq_lens[b], L0 = c.seq_lens[b - 1];
+  if (L1 < 0 || L1 > cap) L1 = 0;
+  if (L0 < 0 || L0 > cap) L0 = 0;
+  const int np = min((min(L1, L0) + kPage - 1) / kPage, p0 + kMaxPrefixPages);
+  const int32_t *r1 = c.page_table + static_cast<size_t>(b) * c.max_pages;
+  const int32_t *r0 = r1 - c.max_pages;
+  // eight pages per round, their loads issued together (one memory latency per round)
+  for (int k = p0; k < np; k += 8) {
+    int a[8], z[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = k + i < np;
+      a[i] = in ? r1[k + i] : 0;
+      z[i] = in ? r0[k + i] : 1;
+    }
+    int first = 8;
+#pragma unroll
+    for (int i = 7; i >= 0; --i)
+      if (a[i] != z[i]) first = i;
+    if (first < 8) return k + first;
+  }
+  return max(p0, np);
+}
+
+struct PrefixRun {
+  int pe = 0;    // end page of the group's shared INT4 pages (0: not in a group)
+  int nmem = 0;  // members of the prefix entry this sequence leads (0: it leads none)
+};
+
+// Groups of the sequences base .. base+1023 (one per thread): maximal runs of consecutive
+// sequences each sharing at least one INT4 page with its predecessor (the run's first
+// sequence, or the block's first, starts it). The group's shared pages are [S/16, pe) with
+// pe the smallest shared count of its members; groups of one sequence read nothing
+// together. Members are taken kPrefixCols / G at a time into prefix entries. All threads
+// of the block call this together (it synchronises the block).
+__device__ PrefixRun prefix_runs(const CacheView &c, const Workspace &w, int base, int *run_min,
+                                 int *run_len, int *warp_max) {
+  const int t = threadIdx.x, b = base + t;
+  const int p0 = c.num_sinks / kPage;
+  int k = 0;
+  bool share = false;
+  if (b < c.num_seqs && t > 0) {
+    k = pages_shared_with_prev(c, b, p0);
+    share = k > p0;
+  }
+  const int lead = block_max_scan(share ? -1 : t, warp_max);
+  run_min[t] = 0x7fffffff;
+  run_len[t] = 0;
+  __syncthreads();
+  if (b < c.num_seqs) {
+    atomicAdd(&run_len[lead], 1);
+    if (share) atomicMin(&run_min[lead], k);
+  }
+  __syncthreads();
+  PrefixRun pr;
+  if (b < c.num_seqs) {
+    const int n = run_len[lead];
+    if (n >= 2) {
+      pr.pe = run_min[lead];
+      const int pos = t - lead;
+      const int M = max(1, kPrefixCols / c.gqa);
+      if (pos % M == 0) pr.nmem = min(M, n - pos);
+    }
+  }
+  __syncthreads();
+  return pr;
+}
+
 struct SeqPlan {
   Regions g;
-  int pages;   // INT4 pages of the sequence's INT4 range
-  int nfull;   // INT4 chunks of exactly chunk_pages pages
+  PrefixRun pr;
+  int pages;   // pages of the sequence's own INT4 chunks
+  int nfull;   // own INT4 chunks of exactly chunk_pages pages
   int key = -1;  // short last chunk: 31 - its pages (sort key), else -1
   bool last_long;  // the shorter last chunk (if any) has at least half the pages
-  // scanned values: regions (protected set + INT4 chunks), then entries per class
-  // (full chunks, long partial chunks, protected sets, short chunks)
+  // scanned values: regions (protected set, shared-prefix regions, own INT4 chunks), then
+  // entries per class: full chunks, long partial chunks, protected sets, short chunks (the
+  // attention kernel's), then shared-prefix chunks (led by the first member of each prefix
+  // entry; the prefix kernel's, at the end of the list)
   int n[kScanN];
 };
 
@@ -123,6 +234,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
   // the last entries of the kernel are the shortest
   __shared__ int key_cnt[32][33];
   __shared__ int key_chunk[32], key_tot[32], key_run[32];
+  __shared__ int run_min[kPlanThreads], run_len[kPlanThreads], warp_max[32];
+  const bool prefix = w.prefix_end != nullptr;
   const int B = c.num_seqs, H = c.num_kv_heads, C = w.chunk_pages;
   const int S = c.num_sinks, R = c.num_recent;
   const int hpw = w.heads_per_warp;
@@ -131,7 +244,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
   const int my_lo = blockIdx.x * per;
   const int my_hi = min(B, my_lo + per);
 
-  auto plan_of = [&](int b) {
+  auto plan_of = [&](int b, const PrefixRun &pr) {
     SeqPlan sp{};
     if (b >= B) return sp;
     int L = c.seq_lens[b];
@@ -139,30 +252,35 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
       if (b >= my_lo && b < my_hi) set_err(err, KV4_DEVERR_SEQ_LEN);
       L = 0;
     }
-    sp.g = regions_of(L, S, R, C);
+    sp.pr = pr;
+    sp.g = regions_of(L, S, R, C, pr.pe);
     sp.pages = sp.g.n_chunks ? (sp.g.int4_hi - 1) / kPage - sp.g.first_page + 1 : 0;
     sp.nfull = sp.pages / C;
     const bool has_last = sp.g.n_chunks > sp.nfull;
     sp.last_long = 2 * (sp.pages - sp.nfull * C) >= C;
-    sp.n[0] = sp.g.has_prot + sp.g.n_chunks;
+    sp.n[0] = sp.g.has_prot + sp.g.n_prompt + sp.g.n_chunks;
     sp.n[1] = sp.nfull * nslots;
     sp.n[2] = has_last && sp.last_long ? nslots : 0;
     sp.n[3] = sp.g.has_prot * nslots;
     sp.n[4] = has_last && !sp.last_long ? nslots : 0;
+    sp.n[5] = pr.nmem ? sp.g.n_prompt * H : 0;
     sp.key = sp.n[4] ? 31 - (sp.pages - sp.nfull * C) : -1;
     return sp;
+  };
+  auto runs_of = [&](int base) {
+    return prefix ? prefix_runs(c, w, base, run_min, run_len, warp_max) : PrefixRun{};
   };
 
   // pass 1: totals over every sequence. A batch of at most kPlanThreads sequences is
   // one block-wide pass, whose exclusive offsets and key ranks are kept for pass 2.
   const bool single = B <= kPlanThreads;
-  int tot[kScanN] = {0, 0, 0, 0, 0};
+  int tot[kScanN] = {0, 0, 0, 0, 0, 0};
   SeqPlan keep{};
-  int keep_off[kScanN] = {0, 0, 0, 0, 0};
+  int keep_off[kScanN] = {0, 0, 0, 0, 0, 0};
   int keep_rank = 0;
   if (threadIdx.x < 32) key_tot[threadIdx.x] = 0;
   for (int base = 0; base < B; base += kPlanThreads) {
-    SeqPlan sp = plan_of(base + threadIdx.x);
+    SeqPlan sp = plan_of(base + threadIdx.x, runs_of(base));
     int off[kScanN], t[kScanN];
 #pragma unroll
     for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
@@ -187,30 +305,39 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     }
   }
   __syncthreads();
-  const int te_all = tot[1] + tot[2] + tot[3] + tot[4];
+  const int te_all = tot[1] + tot[2] + tot[3] + tot[4] + tot[5];
   const bool fits = tot[0] <= w.cap_pairs && te_all <= w.cap_entries;
 
   // pass 2: offsets up to this CTA's slice; entries of the slice (every unit empty if
   // the workspace is too small)
   // class bases: full chunks at 0, then long partial chunks, protected sets, short chunks
-  const int class_base[kScanN] = {0, 0, tot[1], tot[1] + tot[2], tot[1] + tot[2] + tot[3]};
+  int class_base[kScanN] = {0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int i = 2; i < kScanN; ++i) class_base[i] = class_base[i - 1] + tot[i - 1];
   auto write_seq = [&](int b, const SeqPlan &sp, const int (&off)[kScanN], int short_rank) {
     const int pairs = sp.n[0];
     for (int h = 0; h < H; ++h) w.unit_offsets[b * H + h] = H * off[0] + h * pairs;
+    if (prefix) w.prefix_end[b] = sp.pr.pe;
     if (pairs == 0) return;
     const Regions &g = sp.g;
-    int ef = off[1], el = off[2], epr = off[3];
-    const int es = tot[1] + tot[2] + tot[3] + short_rank * nslots;
+    int ef = off[1], el = off[2], epr = off[3], ep = off[5];
+    const int es = class_base[4] + short_rank * nslots;
+    const int own = g.has_prot + g.n_prompt;  // region index of the first own chunk
     if (g.has_prot)
       for (int s = 0; s < nslots; ++s)
         w.entries[epr++] = make_int4(b, 0, s * hpw, min(hpw, H - s * hpw));
+    // this sequence leads a prefix entry: one per prompt chunk ci and kv head, encoded
+    // with region -1 - ci and the member count in place of the head count
+    if (sp.n[5])
+      for (int ci = 0; ci < g.n_prompt; ++ci)
+        for (int h = 0; h < H; ++h) w.entries[ep++] = make_int4(b, -1 - ci, h, sp.pr.nmem);
     for (int ch = 0; ch < sp.nfull; ++ch)
       for (int s = 0; s < nslots; ++s)
-        w.entries[ef++] = make_int4(b, g.has_prot + ch, s * hpw, min(hpw, H - s * hpw));
+        w.entries[ef++] = make_int4(b, own + ch, s * hpw, min(hpw, H - s * hpw));
     if (g.n_chunks > sp.nfull) {
       int e = sp.last_long ? el : es;
       for (int s = 0; s < nslots; ++s)
-        w.entries[e++] = make_int4(b, g.has_prot + sp.nfull, s * hpw, min(hpw, H - s * hpw));
+        w.entries[e++] = make_int4(b, own + sp.nfull, s * hpw, min(hpw, H - s * hpw));
     }
   };
   if (single) {  // the kept pass-1 offsets are final
@@ -228,7 +355,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     for (int i = 0; i < kScanN; ++i) run[i] = class_base[i];
     for (int base = 0; base < my_hi; base += kPlanThreads) {
       const int b = base + threadIdx.x;
-      SeqPlan sp = fits ? plan_of(b) : SeqPlan{};
+      const PrefixRun pr = runs_of(base);
+      SeqPlan sp = fits ? plan_of(b, pr) : SeqPlan{};
       int off[kScanN], t[kScanN];
 #pragma unroll
       for (int i = 0; i < kScanN; ++i) off[i] = sp.n[i];
@@ -250,15 +378,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     // a workspace too small leaves every unit empty (all offsets 0): the merge then
     // reads no partial state and writes zero outputs with lse = -inf
     w.unit_offsets[B * H] = fits ? H * tot[0] : 0;
-    *w.n_items = fits ? te_all : 0;
+    *w.n_items = fits ? te_all - tot[5] : 0;  // the attention kernel's entries
     *w.counter = 0;
+    *w.pn_items = fits ? tot[5] : 0;          // then the prefix kernel's
+    *w.pcounter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
   }
 }
 
 // ------------------------- INT8 protected set ----------------------------
 // One kv head's protected set: sink tiles then recent-ring tiles, INT8 codes.
-__device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t *__restrict__ q,
+__device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t *__restrict__ q,
                                   int b, int h, int L, float *rec, int32_t *err) {
   const int G = c.gqa, H = c.num_kv_heads;
   const int lane = x.lane, gid = x.gid, tig = x.tig;
@@ -279,8 +409,8 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   }
 
   auto issue = [&](int k) {
+    const int st = k % kStages;
     if (lane == 0) {
-      const int st = k % kStages;
       uint8_t *dst = x.stage0 + st * kStageBytes;
       const int8_t *kc, *vc;
       const uint16_t *ks, *vs;
@@ -302,7 +432,8 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
     }
   };
   const int npre = min(nt, kStages);
-  for (int k = 0; k < npre; ++k) issue(k);
+  for (int k = 0; k < npre; ++k)
+    if (prologue_copy(x, k)) issue(k);
 
   // query fragments (B operand of QK^T, m16n8k32): lane column gid = query gid; k-step
   // ks: b0 = dims 32ks+4tig..+3, b1 = dims 32ks+16+4tig..+3, as bytes of
@@ -357,7 +488,7 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
   for (int k = 0; k < nt; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      for (int kk = k + 1; kk < min(nt, k + kStages); ++kk) wait_stage(x, kk % kStages, err);
+      drain_copies(x, k, min(nt, k + kStages));
       write_empty(rec, G, lane);
       return;
     }
@@ -467,7 +598,7 @@ __device__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t
 constexpr int kOffScale8P = 2 * kInt8CodeBytes;                       // scales of slot hs at +32 hs
 constexpr int kInt8PairBytes = 2 * kInt8CodeBytes + 2 * kInt8ScaleBytes;  // 4160 per stage
 
-__device__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Workspace &w,
+__device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Workspace &w,
                                        const uint16_t *__restrict__ q, int b, int h0, int nh,
                                        int L, int r, int32_t *err) {
   constexpr int CPH = 4;  // MMA columns per kv head slot
@@ -497,8 +628,8 @@ __device__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Wor
   // copy k: tile k/2, K part (k even) or V part (k odd), both heads; a spare slot (one
   // head left) gets a copy of head h0
   auto issue = [&](int k) {
+    const int st = k % kStages;
     if (lane == 0) {
-      const int st = k % kStages;
       uint8_t *dst = x.stage0 + st * kStageBytes;
       const int tile = k >> 1;
       const bool vpart = (k & 1) != 0;
@@ -524,11 +655,12 @@ __device__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Wor
     }
   };
   int issued = min(nv, kStages);
-  for (int k = 0; k < issued; ++k) issue(k);
-  // A bounded wait gave up on copy k: wait for the later copies in flight, write empty
+  for (int k = 0; k < issued; ++k)
+    if (prologue_copy(x, k)) issue(k);
+  // The bounded wait for copy k gave up: wait for the copies still in flight, write empty
   // states.
   auto give_up = [&](int k) {
-    for (int kk = k + 1; kk < issued; ++kk) wait_stage(x, kk % kStages, err);
+    drain_copies(x, k, issued);
     for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
   };
 
@@ -742,7 +874,7 @@ __device__ __forceinline__ int row_token_hi(int r) { return 8 + ((r + 4) & 7); }
 // One chunk of INT4 pages for HPW kv heads (h0 .. h0+nh-1, nh <= HPW). MMA column
 // col (0..7) belongs to head slot col / CPH and query j = col % CPH of that head.
 template <int HPW>
-__device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
+__device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
                              const uint16_t *__restrict__ q, int b, int h0, int nh, int r,
                              int chunk, const Regions &rg, int32_t *err) {
   constexpr int CPH = 8 / HPW;  // MMA columns per kv head slot
@@ -776,8 +908,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   constexpr int kOffVp = kOffKp + HPW * kInt4ParamBytes;
   auto issue = [&](int k) {
     const int pk = __shfl_sync(0xffffffffu, k < 32 ? pid : pid2, k & 31);
+    const int st = k % kStages;
     if (lane == 0) {
-      const int st = k % kStages;
       uint8_t *dst = x.stage0 + st * kStageBytes;
       const size_t blk = static_cast<size_t>(pk) * H + h0;
       fence_proxy_async_smem();
@@ -806,7 +938,8 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
     }
   };
   const int npre = min(np, kStages);
-  for (int k = 0; k < npre; ++k) issue(k);
+  for (int k = 0; k < npre; ++k)
+    if (prologue_copy(x, k)) issue(k);
 
   // ---- query fragments (B operand of QK^T). Lane column gid = (slot gid/CPH, query
   // gid%CPH); slot hs's fragments are zero unless the column is in slot hs.
@@ -906,7 +1039,7 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
   for (int k = 0; k < np; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      for (int kk = k + 1; kk < min(np, k + kStages); ++kk) wait_stage(x, kk % kStages, err);
+      drain_copies(x, k, min(np, k + kStages));
       for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
       return;
     }
@@ -1075,6 +1208,386 @@ __device__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
 }
 
 // ---------------------------------------------------------------------------
+// shared-prefix read
+// ---------------------------------------------------------------------------
+// One entry = one chunk of a group's shared INT4 pages, one kv head, up to
+// kPrefixCols / G consecutive member sequences. Column c of the 16 query columns (MMA N
+// tiles c / 8) is query c % G of member c / G. Every page is copied into shared memory
+// once and its K and V codes are unpacked once for all members; the arithmetic per column
+// is that of process_int4 (integer QK^T on the fixed-point query, online softmax,
+// P' = p * vscale in fp16 against the V codes as fp16 subnormals, sum p * vmin in fp32).
+// Member m's tokens outside its INT4 range [S, L_m - R) are masked, so a member whose
+// recent window starts inside the shared pages reads those positions from its ring only.
+// The entries run in prefix_kernel, whose warps have the attention kernel's shared-memory
+// layout: a ring of kStages one-head page blocks and the per-lane query operands in the
+// stage area, the P' tile of both N tiles in the INT4 tile. (A separate kernel rather than
+// a class of attn_kernel: compiled into one kernel, the two paths share one register
+// allocation, and the INT4 path lost 8-10 % to it.)
+constexpr int kPfxOffVc = kInt4CodeBytes;
+constexpr int kPfxOffKp = 2 * kInt4CodeBytes;
+constexpr int kPfxOffVp = 2 * kInt4CodeBytes + kInt4ParamBytes;
+constexpr int kPfxStageBytes = 2 * kInt4CodeBytes + 2 * kInt4ParamBytes;  // 2560: one kv head
+// per-lane query operands: [N tile][group][lane] uint4 (hi b0, hi b1, lo b0, lo b1) and
+// float2 group sums of the lane's C-fragment columns
+constexpr int kPfxOffQ = kStages * kPfxStageBytes;
+constexpr int kPfxOffQs = kPfxOffQ + 2 * 4 * 32 * 16;
+static_assert(kPfxOffQs + 2 * 4 * 32 * 8 <= kStages * kStageBytes,
+              "the shared-prefix ring and query operands fit the warp's stage area");
+static_assert(2 * 4 * 8 * kPWordsPerCol * 4 == kPtileBytes, "two N tiles of P'");
+
+// Prompt chunk ci of kv head h for the nmem group members b0 .. b0+nmem-1.
+__device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, const Workspace &w,
+                               const uint16_t *__restrict__ q, int b0, int ci, int h, int nmem,
+                               int32_t *err) {
+  const int G = c.gqa, H = c.num_kv_heads;
+  const int S = c.num_sinks, R = c.num_recent;
+  const int lane = x.lane, gid = x.gid, tig = x.tig;
+  const int p0 = S / kPage + ci * w.chunk_pages;
+  const int np = min(w.chunk_pages, w.prefix_end[b0] - p0);
+  uint4 *qop = reinterpret_cast<uint4 *>(x.stage0 + kPfxOffQ);
+  float2 *qsum_t = reinterpret_cast<float2 *>(x.stage0 + kPfxOffQs);
+
+  // this thread's C-fragment columns (N tile t, 2tig + e): the end of the member's INT4
+  // range (0 for a column without a member)
+  int hi[2][2];
+  int hi_min = 0x7fffffff;
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int mi = (8 * t + 2 * tig + e) / G;
+      hi[t][e] = mi < nmem ? c.seq_lens[b0 + mi] - R : 0;
+    }
+  for (int mi = 0; mi < nmem; ++mi) hi_min = min(hi_min, c.seq_lens[b0 + mi] - R);
+
+  const int *pt = c.page_table + static_cast<size_t>(b0) * c.max_pages + p0;
+  int pid = 0, pid2 = 0;
+  if (lane < np) pid = pt[lane];
+  if (lane + 32 < np) pid2 = pt[lane + 32];
+  const bool bad = (lane < np && (pid < 0 || pid >= c.num_pages)) ||
+                   (lane + 32 < np && (pid2 < 0 || pid2 >= c.num_pages));
+  auto write_empty_all = [&]() {
+    for (int mi = 0; mi < nmem; ++mi) {
+      const int L = c.seq_lens[b0 + mi];
+      const int r = regions_of(L, S, R, w.chunk_pages).has_prot + ci;
+      write_empty(record_of(w, H, G, b0 + mi, h, r), G, lane);
+    }
+  };
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
+    write_empty_all();
+    return;
+  }
+
+  auto issue = [&](int k) {
+    const int pk = __shfl_sync(0xffffffffu, k < 32 ? pid : pid2, k & 31);
+    const int st = k % kStages;
+    if (lane == 0) {
+      uint8_t *dst = x.stage0 + st * kPfxStageBytes;
+      const size_t blk = static_cast<size_t>(pk) * H + h;
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&x.bars[st], kPfxStageBytes);
+      bulk_g2s(dst, c.k_codes + blk * kInt4CodeBytes, kInt4CodeBytes, &x.bars[st]);
+      bulk_g2s(dst + kPfxOffVc, c.v_codes + blk * kInt4CodeBytes, kInt4CodeBytes, &x.bars[st]);
+      bulk_g2s(dst + kPfxOffKp, reinterpret_cast<const uint8_t *>(c.k_params) + blk * kInt4ParamBytes,
+               kInt4ParamBytes, &x.bars[st]);
+      bulk_g2s(dst + kPfxOffVp, reinterpret_cast<const uint8_t *>(c.v_params) + blk * kInt4ParamBytes,
+               kInt4ParamBytes, &x.bars[st]);
+    }
+  };
+  const int npre = min(np, kStages);
+  for (int k = 0; k < npre; ++k)
+    if (prologue_copy(x, k)) issue(k);
+
+  // ---- query fragments (B operand of QK^T) of column 8t + gid of N tile t, as in
+  // process_int4: q = qstep * (256*hi + lo), b0 = dims 8tig+{0,2,4,6}, b1 = 8tig+{1,3,5,7}
+  float2 kq[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int col = 8 * t + gid, mb = col / G, jb = col - mb * G;
+    const bool live = mb < nmem;
+    const uint16_t *qrow = q + (static_cast<size_t>(b0 + (live ? mb : 0)) * H * G + h * G + jb) * kHeadDim;
+    float qv[4][8];
+    float qsum[4];
+    float amax = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint4 v = load_q8(qrow, 32 * g + 8 * tig, live);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        qv[g][2 * i] = __uint_as_float(w4[i] << 16);
+        qv[g][2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+        sum += qv[g][2 * i] + qv[g][2 * i + 1];
+        amax = fmaxf(amax, fmaxf(fabsf(qv[g][2 * i]), fabsf(qv[g][2 * i + 1])));
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      qsum[g] = sum;
+    }
+    const float qstep = query_step(amax);
+    const float inv = 1.0f / qstep;  // a power of two: exact
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int qi = __float2int_rn(qv[g][i] * inv);
+        const int sel = i & 1, byte = i >> 1;
+        lb[sel] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * byte);
+        hb[sel] |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * byte);
+      }
+      qop[(t * 4 + g) * 32 + lane] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
+      qsum_t[(t * 4 + g) * 32 + lane] = make_float2(__shfl_sync(0xffffffffu, qsum[g], 4 * (2 * tig)),
+                                                    __shfl_sync(0xffffffffu, qsum[g], 4 * (2 * tig + 1)));
+    }
+    kq[t].x = __shfl_sync(0xffffffffu, qstep, 4 * (2 * tig)) * kScaleLog2;
+    kq[t].y = __shfl_sync(0xffffffffu, qstep, 4 * (2 * tig + 1)) * kScaleLog2;
+  }
+
+  float m[2][2], l[2][2];
+  float o[4][2][2][4];  // [group][m-tile][N tile]
+  float mt[4][2][2];    // sum p * vmin per group, N tile and column
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    m[t][0] = m[t][1] = kNegBig;
+    l[t][0] = l[t][1] = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      mt[g][t][0] = mt[g][t][1] = 0.f;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) o[g][u][t][0] = o[g][u][t][1] = o[g][u][t][2] = o[g][u][t][3] = 0.f;
+    }
+  }
+
+  const int r8 = lane & 7;
+  const int mhalf = (lane >> 3) & 1;
+  const int strip_off = (lane >> 4) * 256;
+  const int ld_k = strip_off + (mhalf ? row_token_hi(r8) : r8) * 16;
+  const int ld_v = strip_off + (mhalf ? ((r8 & 1) ? 8 + (r8 >> 1) : 4 + (r8 >> 1))
+                                      : ((r8 & 1) ? 12 + (r8 >> 1) : (r8 >> 1))) * 16;
+  const int t0 = gid, t1 = row_token_hi(gid);
+  uint32_t *pt_mine = x.ptile + (2 * tig) * kPWordsPerCol + gid;
+
+  for (int k = 0; k < np; ++k) {
+    const int st = k % kStages;
+    if (!wait_stage(x, st, err)) {
+      drain_copies(x, k, min(np, k + kStages));
+      write_empty_all();
+      return;
+    }
+    const uint8_t *sp = x.stage0 + st * kPfxStageBytes;
+    const uint32_t sa = smem_u32(sp);
+
+    // ---- logits of both N tiles ----
+    const uint4 kp[2] = {*reinterpret_cast<const uint4 *>(sp + kPfxOffKp + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + kPfxOffKp + t1 * 16)};
+    float2 sc0[2], sc1[2], mn0[2], mn1[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) sc0[t] = sc1[t] = mn0[t] = mn1[t] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {
+      uint32_t kw[4];
+      ldsm_x4(kw, sa + gp * 512 + ld_k);
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = 2 * gp + gg;
+        const uint32_t wlo = kw[2 * gg], whi = kw[2 * gg + 1];
+        const uint32_t a0 = wlo & 0x0F0F0F0Fu, a1 = whi & 0x0F0F0F0Fu;
+        const uint32_t a2 = (wlo >> 4) & 0x0F0F0F0Fu, a3 = (whi >> 4) & 0x0F0F0F0Fu;
+        const uint32_t w0 = g == 0 ? kp[0].x : g == 1 ? kp[0].y : g == 2 ? kp[0].z : kp[0].w;
+        const uint32_t w1 = g == 0 ? kp[1].x : g == 1 ? kp[1].y : g == 2 ? kp[1].z : kp[1].w;
+        const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint4 qo = qop[(t * 4 + g) * 32 + lane];
+          const float2 qs = qsum_t[(t * 4 + g) * 32 + lane];
+          int32_t ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+          mma_u8s8(ah, a0, a1, a2, a3, qo.x, qo.y);
+          mma_u8u8(al, a0, a1, a2, a3, qo.z, qo.w);
+          float acc[4];  // exact integer dot products, |.| < 2^24
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = static_cast<float>(ah[i] * 256 + al[i]);
+          sc0[t] = ffma2(make_float2(f0.x, f0.x), make_float2(acc[0], acc[1]), sc0[t]);
+          mn0[t] = ffma2(make_float2(f0.y, f0.y), qs, mn0[t]);
+          sc1[t] = ffma2(make_float2(f1.x, f1.x), make_float2(acc[2], acc[3]), sc1[t]);
+          mn1[t] = ffma2(make_float2(f1.y, f1.y), qs, mn1[t]);
+        }
+      }
+    }
+    const float2 k1 = make_float2(kScaleLog2, kScaleLog2);
+    float s[2][2][2];  // [N tile][token t0 / t1][column e]
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const float2 sl0 = ffma2(sc0[t], kq[t], fmul2(mn0[t], k1));
+      const float2 sl1 = ffma2(sc1[t], kq[t], fmul2(mn1[t], k1));
+      s[t][0][0] = sl0.x;
+      s[t][0][1] = sl0.y;
+      s[t][1][0] = sl1.x;
+      s[t][1][1] = sl1.y;
+    }
+    const int tok0 = (p0 + k) * kPage;
+    if (tok0 < S || tok0 + kPage > hi_min) {  // some member does not read all 16 tokens
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (!(tok0 + t0 >= S && tok0 + t0 < hi[t][e])) s[t][0][e] = -CUDART_INF_F;
+          if (!(tok0 + t1 >= S && tok0 + t1 < hi[t][e])) s[t][1][e] = -CUDART_INF_F;
+        }
+    }
+    // ---- online softmax per column; the rescale is skipped while no running max moves ----
+    float a[2][2];
+    bool moved = false;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = fmaxf(s[t][0][e], s[t][1][e]);
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        const float mn = fmaxf(m[t][e], v);
+        const bool mv = mn != m[t][e];
+        a[t][e] = mv ? fast_exp2(m[t][e] - mn) : 1.0f;
+        moved |= mv;
+        m[t][e] = mn;
+        s[t][0][e] = fast_exp2(s[t][0][e] - mn);
+        s[t][1][e] = fast_exp2(s[t][1][e] - mn);
+        l[t][e] = fmaf(l[t][e], a[t][e], s[t][0][e] + s[t][1][e]);
+      }
+    if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float2 a2 = make_float2(a[t][0], a[t][1]);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          mt[g][t][0] *= a[t][0];
+          mt[g][t][1] *= a[t][1];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const float2 x0 = fmul2(make_float2(o[g][u][t][0], o[g][u][t][1]), a2);
+            const float2 x1 = fmul2(make_float2(o[g][u][t][2], o[g][u][t][3]), a2);
+            o[g][u][t][0] = x0.x; o[g][u][t][1] = x0.y; o[g][u][t][2] = x1.x; o[g][u][t][3] = x1.y;
+          }
+        }
+      }
+    }
+    // ---- P'_g = p * vscale_g as fp16 token pairs per column; sum p * vmin_g on the side ----
+    const uint4 vp[2] = {*reinterpret_cast<const uint4 *>(sp + kPfxOffVp + t0 * 16),
+                         *reinterpret_cast<const uint4 *>(sp + kPfxOffVp + t1 * 16)};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t w0 = g == 0 ? vp[0].x : g == 1 ? vp[0].y : g == 2 ? vp[0].z : vp[0].w;
+      const uint32_t w1 = g == 0 ? vp[1].x : g == 1 ? vp[1].y : g == 2 ? vp[1].z : vp[1].w;
+      const float2 f0 = h2_to_f2(w0), f1 = h2_to_f2(w1);
+      const float2 sv = make_float2(f0.x, f1.x);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float2 pe0 = make_float2(s[t][0][0], s[t][1][0]), pe1 = make_float2(s[t][0][1], s[t][1][1]);
+        const float2 q0 = fmul2(pe0, sv), q1 = fmul2(pe1, sv);
+        pt_mine[((t * 4 + g) * 8) * kPWordsPerCol] = pack_h2(q0.x, q0.y);
+        pt_mine[((t * 4 + g) * 8 + 1) * kPWordsPerCol] = pack_h2(q1.x, q1.y);
+        mt[g][t][0] = fmaf(pe0.x, f0.y, fmaf(pe0.y, f1.y, mt[g][t][0]));
+        mt[g][t][1] = fmaf(pe1.x, f0.y, fmaf(pe1.y, f1.y, mt[g][t][1]));
+      }
+    }
+    __syncwarp();
+    // ---- O^T += V^T P' per group and N tile ----
+#pragma unroll
+    for (int gp = 0; gp < 2; ++gp) {
+      uint32_t vw[4];
+      ldsm_x4_t(vw, sa + kPfxOffVc + gp * 512 + ld_v);
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g = 2 * gp + gg;
+        uint32_t vl[4], vh[4];
+        nib_pairs_v_sub(vw[2 * gg], vl);
+        nib_pairs_v_sub(vw[2 * gg + 1], vh);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t *pb = x.ptile + ((t * 4 + g) * 8 + gid) * kPWordsPerCol + tig;
+          const uint32_t b01 = pb[0], b23 = pb[4];
+          mma_f16(o[g][0][t], vl[0], vl[1], vh[0], vh[1], b01, b23);
+          mma_f16(o[g][1][t], vl[2], vl[3], vh[2], vh[3], b01, b23);
+        }
+      }
+    }
+    __syncwarp();
+    if (k + kStages < np) issue(k + kStages);
+  }
+
+  // ---- finish: reduce over the 8 token lanes, write each member's partial ----
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) l[t][e] += __shfl_xor_sync(0xffffffffu, l[t][e], off);
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)
+          mt[g][t][e] += __shfl_xor_sync(0xffffffffu, mt[g][t][e], off);
+    }
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int col = 8 * t + 2 * tig + e, mi = col / G, j = col - mi * G;
+      if (mi >= nmem) continue;
+      const int r = regions_of(c.seq_lens[b0 + mi], S, R, w.chunk_pages).has_prot + ci;
+      float *rr = record_of(w, H, G, b0 + mi, h, r) + j * kRecordFloats;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 v = make_float4(fmaf(o[g][0][t][e], kUnscaleV, mt[g][t][e]),
+                                     fmaf(o[g][0][t][2 + e], kUnscaleV1, mt[g][t][e]),
+                                     fmaf(o[g][1][t][e], kUnscaleV, mt[g][t][e]),
+                                     fmaf(o[g][1][t][2 + e], kUnscaleV1, mt[g][t][e]));
+        *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
+      }
+      if (gid == 0) {
+        rr[kHeadDim] = m[t][e] * kLn2;
+        rr[kHeadDim + 1] = l[t][e];
+      }
+    }
+}
+
+__global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(CacheView c, Workspace w,
+                                                                             const uint16_t *__restrict__ q,
+                                                                             int32_t *err) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  WarpCtx x;
+  const int warp = threadIdx.x >> 5;
+  x.lane = threadIdx.x & 31;
+  x.gid = x.lane >> 2;
+  x.tig = x.lane & 3;
+  uint8_t *mine = smem + warp * kWarpSmem;
+  x.stage0 = mine;
+  x.ptile = reinterpret_cast<uint32_t *>(mine + kStages * kStageBytes);
+  x.ptile8 = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes + kPtileBytes);
+  x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes + kPtile8Bytes);
+  init_warp<false>(x, w);
+  if (x.lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&x.bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const int base = *w.n_items;  // the prefix entries follow the attention kernel's
+  const int n_items = *w.pn_items;
+  for (;;) {
+    int item = 0;
+    if (x.lane == 0) item = atomicAdd(w.pcounter, 1);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    if (item >= n_items) break;
+    const int4 en = w.entries[base + item];
+    process_prefix(x, c, w, q, en.x, -1 - en.y, en.z, en.w, err);
+    if (x.dead) break;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // exact regional merge
 // ---------------------------------------------------------------------------
 // One warp merges query j of unit u over its regions r0 .. r0+n-1:
@@ -1155,7 +1668,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
 }
 
 
-template <int HPW>
+template <int HPW, bool HOOK>
 __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(CacheView c, Workspace w,
                                                                            const uint16_t *__restrict__ q,
                                                                            int32_t *err) {
@@ -1170,8 +1683,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
   x.ptile = reinterpret_cast<uint32_t *>(mine + kStages * kStageBytes);
   x.ptile8 = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes + kPtileBytes);
   x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes + kPtile8Bytes);
-  x.parity = 0;
-  x.dead = false;
+  init_warp<HOOK>(x, w);
   // the INT4 P' tile's unused columns stay zero for the whole kernel
   for (int i = x.lane; i < kPtileBytes / 4; i += 32) x.ptile[i] = 0u;
   if (x.lane == 0) {
@@ -1187,17 +1699,19 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
     if (x.lane == 0) item = atomicAdd(w.counter, 1);
     item = __shfl_sync(0xffffffffu, item, 0);
     if (item >= n_items) break;
+    x.fault = withheld_item<HOOK>(w, item);
     const int4 en = w.entries[item];
     const int b = en.x, r = en.y, h0 = en.z, nh = en.w;
     const int L = c.seq_lens[b];
-    const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages);
+    const int pe = w.prefix_end ? w.prefix_end[b] : 0;
+    const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages, pe);
     if (r < rg.has_prot) {
       if constexpr (HPW == 2)
         process_protected_pair(x, c, w, q, b, h0, nh, L, r, err);
       else
         process_protected(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
     } else
-      process_int4<HPW>(x, c, w, q, b, h0, nh, r, r - rg.has_prot, rg, err);
+      process_int4<HPW>(x, c, w, q, b, h0, nh, r, r - rg.has_prot - rg.n_prompt, rg, err);
     if (x.dead) break;
   }
 }
@@ -1212,28 +1726,45 @@ cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_fla
   return cudaGetLastError();
 }
 
-template <int HPW>
+template <int HPW, bool HOOK>
 static cudaError_t launch_attn_t(const CacheView &c, const Workspace &w, const uint16_t *q,
                                  int32_t *err_flag, cudaStream_t s) {
-  static int configured_device = -1;
-  static int grid = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev != configured_device) {
-    e = cudaFuncSetAttribute(attn_kernel<HPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kCtaSmem);
-    if (e != cudaSuccess) return e;
+  static PerDevice grids;  // persistent grid per device
+  int grid = 0;
+  cudaError_t e = once_per_device(grids, [](int dev, int *g) {
+    cudaError_t r = cudaFuncSetAttribute(attn_kernel<HPW, HOOK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kCtaSmem);
     int sms = 0, per_sm = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<HPW>, kWarps * 32,
-                                                      kCtaSmem);
-    if (e != cudaSuccess) return e;
-    grid = sms * (per_sm > 0 ? per_sm : 1);
-    configured_device = dev;
-  }
-  attn_kernel<HPW><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<HPW, HOOK>,
+                                                        kWarps * 32, kCtaSmem);
+    *g = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  }, &grid);
+  if (e != cudaSuccess) return e;
+  attn_kernel<HPW, HOOK><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefix(const CacheView &c, const Workspace &w, const uint16_t *q,
+                          int32_t *err_flag, cudaStream_t s) {
+  if (w.prefix_end == nullptr) return cudaSuccess;
+  static PerDevice grids;  // persistent grid per device
+  int grid = 0;
+  cudaError_t e = once_per_device(grids, [](int dev, int *g) {
+    cudaError_t r = cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kCtaSmem);
+    int sms = 0, per_sm = 0;
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefix_kernel, kWarps * 32,
+                                                        kCtaSmem);
+    *g = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  }, &grid);
+  if (e != cudaSuccess) return e;
+  prefix_kernel<<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
   return cudaGetLastError();
 }
 
@@ -1241,8 +1772,11 @@ int heads_per_warp_for(int gqa) { return gqa <= 4 ? 2 : 1; }
 
 cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
                              int32_t *err_flag, cudaStream_t s) {
-  return w.heads_per_warp == 2 ? launch_attn_t<2>(c, w, q, err_flag, s)
-                               : launch_attn_t<1>(c, w, q, err_flag, s);
+  if (w.fault_item >= 0)  // the testing hook is armed for this call
+    return w.heads_per_warp == 2 ? launch_attn_t<2, true>(c, w, q, err_flag, s)
+                                 : launch_attn_t<1, true>(c, w, q, err_flag, s);
+  return w.heads_per_warp == 2 ? launch_attn_t<2, false>(c, w, q, err_flag, s)
+                               : launch_attn_t<1, false>(c, w, q, err_flag, s);
 }
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
@@ -1256,30 +1790,42 @@ cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int
 }
 
 size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads, int32_t gqa,
-                       int32_t chunk_pages, Workspace *carve, void *base) {
+                       int32_t chunk_pages, bool prefix, Workspace *carve, void *base) {
   const long long pages = (static_cast<long long>(max_seq_len) + kPage - 1) / kPage + 1;
-  const long long per_seq = 1 + (pages + chunk_pages - 1) / chunk_pages;
+  // regions per sequence: the protected set and the INT4 chunks; with the shared-prefix
+  // read the INT4 pages are cut once more (shared pages | own pages): one region more
+  const long long per_seq = (prefix ? 2 : 1) + (pages + chunk_pages - 1) / chunk_pages;
   const long long cap = static_cast<long long>(num_seqs) * per_seq;
   const long long cap_e = cap * num_kv_heads;
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
-  size_t off = 256;  // counter, n_items
+  size_t off = 256;  // counter, n_items, prefix counter, prefix n_items
   const size_t ent_off = off;
   off = up(off + static_cast<size_t>(cap_e) * sizeof(int4));
   const size_t units_off = off;
   off = up(off + (static_cast<size_t>(num_seqs) * num_kv_heads + 1) * sizeof(int32_t));
+  size_t pend_off = 0;
+  if (prefix) {
+    pend_off = off;
+    off = up(off + static_cast<size_t>(num_seqs) * sizeof(int32_t));
+  }
   const size_t part_off = off;
   off = up(off + static_cast<size_t>(cap) * num_kv_heads * gqa * kRecordFloats * sizeof(float));
   if (carve) {
     uint8_t *p = static_cast<uint8_t *>(base);
     carve->counter = reinterpret_cast<int32_t *>(p);
     carve->n_items = reinterpret_cast<int32_t *>(p) + 1;
+    carve->pcounter = reinterpret_cast<int32_t *>(p) + 2;
+    carve->pn_items = reinterpret_cast<int32_t *>(p) + 3;
     carve->entries = reinterpret_cast<int4 *>(p + ent_off);
     carve->unit_offsets = reinterpret_cast<int32_t *>(p + units_off);
+    carve->prefix_end = prefix ? reinterpret_cast<int32_t *>(p + pend_off) : nullptr;
     carve->partials = reinterpret_cast<float *>(p + part_off);
     carve->cap_pairs = static_cast<int32_t>(cap);
     carve->cap_entries = static_cast<int32_t>(cap_e);
     carve->chunk_pages = chunk_pages;
     carve->heads_per_warp = heads_per_warp_for(gqa);
+    carve->wait_limit = kWaitLimit;
+    carve->fault_item = -1;
   }
   return off;
 }

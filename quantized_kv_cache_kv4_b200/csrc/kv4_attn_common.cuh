@@ -47,25 +47,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // ---------------------------------------------------------------------------
 struct Regions {
   int has_prot;          // 1 if the INT8 protected set is non-empty
-  int first_page;        // first page of the INT4 range
+  int n_prompt;          // regions over pages shared with the sequence's prefix group
+  int first_page;        // first page of the sequence's own INT4 chunks
   int int4_lo, int4_hi;  // INT4 token range [lo, hi)
-  int n_chunks;
+  int n_chunks;          // the sequence's own INT4 chunks
 };
 
-__device__ __forceinline__ Regions regions_of(int L, int S, int R, int C) {
+// Regions of a sequence of length L, in merge order: the protected set (if any), then
+// n_prompt regions over the INT4 pages [S/16, pe) that the sequence's prefix group reads
+// once for all its members (pe = 0: no group), then its own chunks of C pages from
+// max(S/16, pe) on. A group member's prompt regions exist even where its own INT4 range
+// does not reach them (their partial states are then empty), so every member of a group
+// has the same region layout up to its own chunks.
+__device__ __forceinline__ Regions regions_of(int L, int S, int R, int C, int pe = 0) {
   Regions g;
   const int n_sink = min(S, L);
   const int rec_lo = max(S, L - R);
   g.has_prot = (n_sink > 0 || rec_lo < L) ? 1 : 0;
   g.int4_lo = S;
   g.int4_hi = L - R;
+  const int p0 = S / kPage;
+  g.n_prompt = pe > p0 ? (pe - p0 + C - 1) / C : 0;
+  g.first_page = max(p0, pe);
+  g.n_chunks = 0;
   if (g.int4_hi > g.int4_lo) {
-    g.first_page = g.int4_lo / kPage;
     const int last = (g.int4_hi - 1) / kPage;
-    g.n_chunks = (last - g.first_page + 1 + C - 1) / C;
-  } else {
-    g.first_page = 0;
-    g.n_chunks = 0;
+    if (last >= g.first_page) g.n_chunks = (last - g.first_page + C) / C;
   }
   return g;
 }
@@ -79,9 +86,18 @@ struct WarpCtx {
   uint16_t *ptile8;    // INT8 P' tile [8 heads][16 tokens]
   uint64_t *bars;      // kStages mbarriers
   uint32_t parity;     // bit s = parity of the next completion of stage s
+  uint32_t wait_limit; // attempts of one bounded wait
   int lane, gid, tig;
+  bool fault;          // testing hook: the current entry's first copy is withheld
   bool dead;           // a bounded wait gave up: stop taking work
 };
+
+// Whether an entry's copy k is issued by its prologue: the testing hook withholds copy 0
+// of the chosen work item (nothing is issued, nothing is in flight, and the bounded wait
+// on its stage gives up). Copies issued inside the page loops have k >= kStages.
+__device__ __forceinline__ bool prologue_copy(const WarpCtx &x, int k) {
+  return !(x.fault && k == 0);
+}
 
 // Online softmax update for this thread's two heads (2tig, 2tig+1) with logits of
 // tokens (gid, gid+8) in log2 units. Returns p in s[][] and the rescale factors.
@@ -102,14 +118,50 @@ __device__ __forceinline__ void softmax_step(float (&s)[2][2], float (&m)[2], fl
   }
 }
 
+// Bounded wait for the next completion of `stage`; the stage's parity bit flips either
+// way (a wait that gave up leaves the warp dead, and drain_copies knows its parity).
 __device__ __forceinline__ bool wait_stage(WarpCtx &x, int stage, int32_t *err) {
-  const bool ok = mbar_wait_bounded(&x.bars[stage], (x.parity >> stage) & 1u);
+  const bool ok = mbar_wait_bounded(&x.bars[stage], (x.parity >> stage) & 1u, x.wait_limit);
   x.parity ^= 1u << stage;
   if (!ok) {
     x.dead = true;
     if (x.lane == 0) set_err(err, KV4_DEVERR_TIMEOUT);
   }
   return ok;
+}
+
+// After the wait for copy `from` gave up: wait for copies from .. to-1 (every copy of the
+// entry issued and not yet waited for, the one that timed out included, with the parity
+// its wait had before it flipped), each up to 16 times the normal limit, so that none
+// lands in shared memory after the warp (and possibly its CTA) has finished. A copy that
+// does not complete even then is left behind; the TIMEOUT bit already marks the call's
+// results as void. The warp takes no further work, so the parities are not kept.
+__device__ inline void drain_copies(const WarpCtx &x, int from, int to) {
+  const uint32_t longer = x.wait_limit > 0x0FFFFFFFu ? 0xFFFFFFFFu : x.wait_limit * 16u;
+  for (int k = from; k < to; ++k) {
+    if (!prologue_copy(x, k)) continue;  // withheld by the testing hook: never issued
+    const int st = k % kStages;
+    const uint32_t par = ((x.parity >> st) & 1u) ^ (k == from ? 1u : 0u);
+    mbar_wait_bounded(&x.bars[st], par, longer);
+  }
+}
+
+// Per-warp state at the start of a persistent attention kernel. Kernels are instantiated
+// twice: HOOK = false for normal calls (the constant wait limit and the absent hook fold
+// into the code: nothing of the testing hook is left in it), HOOK = true only for a call
+// with the testing hook armed (the wait limit and the withheld work item from the
+// workspace descriptor).
+template <bool HOOK>
+__device__ __forceinline__ void init_warp(WarpCtx &x, const Workspace &w) {
+  x.parity = 0;
+  x.wait_limit = HOOK ? w.wait_limit : kWaitLimit;
+  x.fault = false;
+  x.dead = false;
+}
+
+template <bool HOOK>
+__device__ __forceinline__ bool withheld_item(const Workspace &w, int item) {
+  return HOOK && item == w.fault_item;
 }
 
 // Write the empty partial state (-inf, 0, 0) for the G heads of a record group.

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256) baseline_append_kernel(CacheView c,
 // attention: one kv head per warp, MMA N columns = the head's G queries
 // ---------------------------------------------------------------------------
 template <int F>
-__device__ void process_baseline(WarpCtx &x, const CacheView &c, const Workspace &w,
+__device__ __forceinline__ void process_baseline(WarpCtx &x, const CacheView &c, const Workspace &w,
                                  const uint16_t *__restrict__ q, int b, int h, int r,
                                  const Regions &rg, int32_t *err) {
   const int G = c.gqa, H = c.num_kv_heads;
@@ -124,8 +124,8 @@ __device__ void process_baseline(WarpCtx &x, const CacheView &c, const Workspace
   auto issue = [&](int k) {
     const int page = k >> 1;
     const int pk = __shfl_sync(0xffffffffu, page < 32 ? pid : pid2, page & 31);
+    const int st = k % kStages;
     if (lane == 0) {
-      const int st = k % kStages;
       uint8_t *dst = x.stage0 + st * kStageBytes;
       const size_t blk = static_cast<size_t>(pk) * H + h;
       const bool vpart = (k & 1) != 0;
@@ -144,9 +144,10 @@ __device__ void process_baseline(WarpCtx &x, const CacheView &c, const Workspace
     }
   };
   int issued = min(nv, kStages);
-  for (int k = 0; k < issued; ++k) issue(k);
+  for (int k = 0; k < issued; ++k)
+    if (prologue_copy(x, k)) issue(k);
   auto give_up = [&](int k) {
-    for (int kk = k + 1; kk < issued; ++kk) wait_stage(x, kk % kStages, err);
+    drain_copies(x, k, issued);
     write_empty(rec, G, lane);
   };
 
@@ -382,7 +383,7 @@ __device__ void process_baseline(WarpCtx &x, const CacheView &c, const Workspace
   }
 }
 
-template <int F>
+template <int F, bool HOOK>
 __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) baseline_attn_kernel(
     CacheView c, Workspace w, const uint16_t *__restrict__ q, int32_t *err) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -396,8 +397,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) baseline_attn_ker
   x.ptile = reinterpret_cast<uint32_t *>(mine + kStages * kStageBytes);
   x.ptile8 = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes + kPtileBytes);
   x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes + kPtile8Bytes);
-  x.parity = 0;
-  x.dead = false;
+  init_warp<HOOK>(x, w);
   if (x.lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&x.bars[s], 1);
     fence_barrier_init();
@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) baseline_attn_ker
     if (x.lane == 0) item = atomicAdd(w.counter, 1);
     item = __shfl_sync(0xffffffffu, item, 0);
     if (item >= n_items) break;
+    x.fault = withheld_item<HOOK>(w, item);
     const int4 en = w.entries[item];
     const int b = en.x, r = en.y, h = en.z;
     const Regions rg = regions_of(c.seq_lens[b], 0, 0, w.chunk_pages);
@@ -435,35 +436,34 @@ cudaError_t launch_baseline_append(int fmt, const CacheView &c, const uint16_t *
   return cudaGetLastError();
 }
 
-template <int F>
+template <int F, bool HOOK>
 static cudaError_t launch_baseline_attn_t(const CacheView &c, const Workspace &w,
                                           const uint16_t *q, int32_t *err_flag, cudaStream_t s) {
-  static int configured_device = -1;
-  static int grid = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev != configured_device) {
-    e = cudaFuncSetAttribute(baseline_attn_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kCtaSmem);
-    if (e != cudaSuccess) return e;
+  static PerDevice grids;  // persistent grid per device
+  int grid = 0;
+  cudaError_t e = once_per_device(grids, [](int dev, int *g) {
+    cudaError_t r = cudaFuncSetAttribute(baseline_attn_kernel<F, HOOK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kCtaSmem);
     int sms = 0, per_sm = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, baseline_attn_kernel<F>,
-                                                      kWarps * 32, kCtaSmem);
-    if (e != cudaSuccess) return e;
-    grid = sms * (per_sm > 0 ? per_sm : 1);
-    configured_device = dev;
-  }
-  baseline_attn_kernel<F><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, baseline_attn_kernel<F, HOOK>,
+                                                        kWarps * 32, kCtaSmem);
+    *g = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  }, &grid);
+  if (e != cudaSuccess) return e;
+  baseline_attn_kernel<F, HOOK><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
   return cudaGetLastError();
 }
 
 cudaError_t launch_baseline_attention(int fmt, const CacheView &c, const Workspace &w,
                                       const uint16_t *q, int32_t *err_flag, cudaStream_t s) {
-  return fmt == kFmtBf16 ? launch_baseline_attn_t<kFmtBf16>(c, w, q, err_flag, s)
-                         : launch_baseline_attn_t<kFmtKv8>(c, w, q, err_flag, s);
+  if (w.fault_item >= 0)  // the testing hook is armed for this call
+    return fmt == kFmtBf16 ? launch_baseline_attn_t<kFmtBf16, true>(c, w, q, err_flag, s)
+                           : launch_baseline_attn_t<kFmtKv8, true>(c, w, q, err_flag, s);
+  return fmt == kFmtBf16 ? launch_baseline_attn_t<kFmtBf16, false>(c, w, q, err_flag, s)
+                         : launch_baseline_attn_t<kFmtKv8, false>(c, w, q, err_flag, s);
 }
 
 }  // namespace kv4

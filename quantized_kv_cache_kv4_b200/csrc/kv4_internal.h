@@ -5,9 +5,39 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/kv4.h"
 
 namespace kv4 {
+
+constexpr int kMaxDevices = 64;
+
+// Per-device launch set-up done once: `configure(dev)` (kernel attributes, the persistent
+// grid size) runs under the table's lock the first time a device is seen, and its
+// positive result is kept for that device; later calls only read it. Safe for host
+// threads driving different devices at once.
+struct PerDevice {
+  std::mutex mu;
+  int value[kMaxDevices] = {};
+};
+
+template <class F>
+cudaError_t once_per_device(PerDevice &t, F configure, int *value) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(t.mu);
+  if (t.value[dev] <= 0) {
+    int v = 0;
+    e = configure(dev, &v);
+    if (e != cudaSuccess) return e;
+    t.value[dev] = v > 0 ? v : 1;
+  }
+  *value = t.value[dev];
+  return cudaSuccess;
+}
 
 // Everything a kernel needs about the cache and the batch, by value.
 struct CacheView {
@@ -43,7 +73,17 @@ struct Workspace {
   int32_t cap_entries;    // work entries the entry list holds
   int32_t chunk_pages;
   int32_t heads_per_warp;  // kv heads one warp serves in an INT4 region entry (1 or 2)
+  // shared-prefix read (nullptr prefix_end: off): pages shared by consecutive sequences
+  // are read once per group of up to 16 / gqa members, in entries (first member,
+  // -1 - prompt chunk, kv head, members)
+  int32_t *prefix_end;     // [num_seqs] end page of the group's shared INT4 pages, 0 = none
+  int32_t *pcounter;       // [1] dynamic work counter of the prefix kernel
+  int32_t *pn_items;       // [1] shared-prefix entries (listed after the n_items others)
+  uint32_t wait_limit;     // attempts of one bounded wait for a copy (kWaitLimit)
+  int32_t fault_item;      // testing hook: work item whose first copy is withheld, -1 none
 };
+
+constexpr uint32_t kWaitLimit = 1u << 22;  // bounded-wait attempts in normal operation
 
 // Where the merged attention output goes.
 struct Outputs {
@@ -56,7 +96,8 @@ struct Outputs {
 int heads_per_warp_for(int gqa);
 
 size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_heads,
-                       int32_t gqa, int32_t chunk_pages, Workspace *carve, void *base);
+                       int32_t gqa, int32_t chunk_pages, bool prefix, Workspace *carve,
+                       void *base);
 
 cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint16_t *v_new,
                           const int32_t *new_indptr, int32_t total_new, int32_t *err_flag,
@@ -67,6 +108,11 @@ cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_fla
 
 cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
                              int32_t *err_flag, cudaStream_t s);
+
+// The shared-prefix read (launches nothing when w.prefix_end is nullptr).
+cudaError_t launch_prefix(const CacheView &c, const Workspace &w, const uint16_t *q,
+                          int32_t *err_flag, cudaStream_t s);
+
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
                          int32_t group, uint16_t *out, float *out_f32, float *lse,

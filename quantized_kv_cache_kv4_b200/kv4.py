@@ -32,7 +32,7 @@ EXPORTS = ("kv4_workspace_size", "kv4_quantize_append", "kv4_decode_attention",
            "kv4_decode_step", "kv4_regional_merge", "kv4_status_string", "kv4_version",
            "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes",
            "kv4_baseline_append", "kv4_baseline_workspace_size",
-           "kv4_baseline_decode_attention")
+           "kv4_baseline_decode_attention", "kv4_test_withhold_copy")
 
 BASELINE_BF16 = 1  # kv4_baseline_format
 BASELINE_KV8 = 2
@@ -43,7 +43,7 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("group_size", ctypes.c_int32), ("num_sinks", ctypes.c_int32),
                 ("num_recent", ctypes.c_int32), ("chunk_pages", ctypes.c_int32),
-                ("demotion", ctypes.c_int32)]
+                ("demotion", ctypes.c_int32), ("prefix_mode", ctypes.c_int32)]
 
 
 class Int4Pool(ctypes.Structure):
@@ -115,6 +115,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                   ctypes.POINTER(PagedPool),
                                                   ctypes.POINTER(Batch), P, P, P, P, P,
                                                   ctypes.c_size_t, P, P]
+    lib.kv4_test_withhold_copy.restype = None
+    lib.kv4_test_withhold_copy.argtypes = [ctypes.c_int32, ctypes.c_uint32]
     lib.kv4_status_string.restype = ctypes.c_char_p
     lib.kv4_status_string.argtypes = [ctypes.c_int]
     lib.kv4_version.restype = ctypes.c_int32
@@ -152,12 +154,13 @@ def _stream(stream):
 
 
 DEMOTION = {"A": 0, "B": 1}  # kv4_config.demotion
+PREFIX = {"off": 0, "shared": 1}  # kv4_config.prefix_mode
 
 
 def make_config(num_q_heads, num_kv_heads, num_sinks, num_recent, chunk_pages=0,
-                demotion="A") -> Config:
+                demotion="A", prefix="off") -> Config:
     return Config(num_q_heads, num_kv_heads, HEAD_DIM, PAGE, GROUP, num_sinks, num_recent,
-                  chunk_pages, DEMOTION[demotion])
+                  chunk_pages, DEMOTION[demotion], PREFIX[prefix])
 
 
 @dataclasses.dataclass

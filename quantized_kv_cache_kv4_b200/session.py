@@ -25,7 +25,7 @@ class DecodeSession:
                  chunk_pages: int = 0, keep_streams=(), keep_bits: bool = False,
                  build: bool = True,
                  max_rows_per_call: int = 1 << 20, workspace: torch.Tensor | None = None,
-                 demotion: str = "A"):
+                 demotion: str = "A", prefix: str = "off"):
         self.wl = wl
         self.layer = layer
         self.steps = steps
@@ -33,7 +33,7 @@ class DecodeSession:
         self.paging = make_paging(wl, extra_tokens=steps)
         self.demotion = demotion
         self.cfg = kv4.make_config(wl.num_q_heads, wl.num_kv_heads, wl.num_sinks,
-                                   wl.num_recent, chunk_pages, demotion)
+                                   wl.num_recent, chunk_pages, demotion, prefix)
         self.cache = self._allocate_cache()
         B = wl.num_seqs
         self.L0 = wl.seq_lens.astype(np.int64)  # lengths after step 0's append

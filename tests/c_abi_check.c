@@ -28,11 +28,12 @@ static kv4_config config(int32_t hq, int32_t hkv, int32_t s, int32_t r, int32_t 
   c.num_recent = r;
   c.chunk_pages = chunk;
   c.demotion = 0;
+  c.prefix_mode = KV4_PREFIX_OFF;
   return c;
 }
 
 int main(void) {
-  CHECK(kv4_version() >= 400);
+  CHECK(kv4_version() >= 500);
   CHECK(strcmp(kv4_status_string(KV4_OK), "ok") == 0);
   CHECK(strstr(kv4_status_string(KV4_ERR_PROTECTED_TOO_LARGE), "144") != NULL);
 

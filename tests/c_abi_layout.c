@@ -14,6 +14,7 @@ int main(void) {
   OFF(kv4_config, num_q_heads); OFF(kv4_config, num_kv_heads); OFF(kv4_config, head_dim);
   OFF(kv4_config, page_size); OFF(kv4_config, group_size); OFF(kv4_config, num_sinks);
   OFF(kv4_config, num_recent); OFF(kv4_config, chunk_pages); OFF(kv4_config, demotion);
+  OFF(kv4_config, prefix_mode);
   SIZE(kv4_int4_pool);
   OFF(kv4_int4_pool, k_codes); OFF(kv4_int4_pool, v_codes); OFF(kv4_int4_pool, k_params);
   OFF(kv4_int4_pool, v_params); OFF(kv4_int4_pool, num_pages);

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(kv4):
 
 def test_status_strings_and_version(kv4):
     lib = kv4._lib
-    assert lib.kv4_version() == 400
+    assert lib.kv4_version() == 500
     assert lib.kv4_status_string(0) == b"ok"
     assert b"144" in lib.kv4_status_string(-3)
     assert lib.kv4_status_string(-99) == b"unknown status"
@@ -54,11 +54,14 @@ def test_status_strings_and_version(kv4):
 
 def _cfg(kv4, **kw):
     d = dict(num_q_heads=32, num_kv_heads=8, num_sinks=16, num_recent=128, chunk_pages=0)
-    raw_demotion = kw.pop("demotion", None)  # an int: written to the struct as is
+    raw_demotion = kw.pop("demotion", None)  # ints: written to the struct as they are
+    raw_prefix = kw.pop("prefix_mode", None)
     d.update(kw)
     c = kv4.make_config(**d)
     if raw_demotion is not None:
         c.demotion = raw_demotion
+    if raw_prefix is not None:
+        c.prefix_mode = raw_prefix
     return c
 
 
@@ -82,6 +85,8 @@ def test_workspace_size_host_only(kv4):
     (dict(chunk_pages=65), -2),
     (dict(demotion=2), -1),
     (dict(demotion=-1), -1),
+    (dict(prefix_mode=2), -1),
+    (dict(prefix_mode=-1), -1),
     (dict(num_sinks=-1), -1),
 ])
 def test_config_rejected_before_launch(kv4, kw, status):
@@ -190,7 +195,8 @@ def test_baseline_argument_checks(kv4):
     lib = kv4._lib
     c = _cfg(kv4)
     none_prot = _cfg(kv4, num_sinks=0, num_recent=0)
-    # the baselines ignore the protected set: same workspace as KV4-RL without one
+    # the baselines ignore the protected set and read no shared prefix: same workspace as
+    # KV4-RL without either
     assert kv4.baseline_workspace_size(c, 64, 2048) == kv4.workspace_size(none_prot, 64, 2048)
     pool = kv4.PagedPool(1 << 20, 1 << 20, 1 << 20, 1 << 20, 10)
     batch = kv4.Batch(1 << 20, 64, 1 << 20, 0, 0, 2, 1000)
@@ -247,7 +253,7 @@ def test_binding_structs_match_the_c_layout(kv4, tmp_path):
             struct, field = name.split(".")
             assert getattr(py[struct], field).offset == val, name
         checked += 1
-    assert checked == 5 + 9 + 5 + 10 + 7 + 5
+    assert checked == 5 + 10 + 5 + 10 + 7 + 5
 
 
 def test_binding_refuses_host_or_strided_tensors(kv4):
@@ -281,17 +287,24 @@ def test_binding_signatures_match_the_header(kv4):
     ptr_types = (ctypes.c_void_p, ctypes._Pointer)
 
     def kind(ct):
+        if ct is None:
+            return "void"
         if ct in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(ct, ptr_types):
             return "pointer"
-        return {ctypes.c_int32: "int32", ctypes.c_int: "int32", ctypes.c_size_t: "size_t"}[ct]
+        return {ctypes.c_int32: "int32", ctypes.c_int: "int32", ctypes.c_uint32: "uint32",
+                ctypes.c_size_t: "size_t"}[ct]
 
     def c_kind(decl):
         if "*" in decl or decl.startswith("kv4_stream_t"):
             return "pointer"
         if decl.startswith("size_t"):
             return "size_t"
+        if decl == "void":
+            return "void"
         if decl.split()[0] in ("int32_t", "kv4_status", "kv4_baseline_format"):
             return "int32"
+        if decl.split()[0] == "uint32_t":
+            return "uint32"
         raise AssertionError(f"unclassified parameter {decl!r}")
 
     for name, (ret, params) in protos.items():

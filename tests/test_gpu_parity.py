@@ -210,6 +210,93 @@ def test_pairs_sharing_prompt_pages(C):
     sess.check_err()
 
 
+def _prefix_entries(sess):
+    """Shared-prefix entries of the last attention call on sess's workspace: the count in
+    its fourth int32, the entries (negative region) after the attention kernel's."""
+    head = sess.workspace[:16].view(torch.int32).cpu().tolist()
+    n_att, n_pfx = head[1], head[3]
+    ent = sess.workspace[256:256 + 16 * (n_att + n_pfx)].view(torch.int32).view(-1, 4)
+    assert bool((ent[n_att:, 1] < 0).all()) and bool((ent[:n_att, 1] >= 0).all())
+    return n_pfx
+
+
+PREFIX_CASES = [
+    # name, lens, Hq, Hkv, S, R, prompt_len, group_seqs, chunk_pages
+    ("groups-of-8-gqa4", [700, 900, 410, 1300, 260, 2000, 520, 640, 333, 1000, 1500, 270,
+                          800, 300, 450, 999], 32, 8, 16, 128, 256, 8, 0),
+    # members whose recent window starts inside the shared pages (L - R < prompt)
+    ("recent-inside-prompt", [300, 500, 280, 290, 1000, 262], 8, 2, 16, 128, 256, 3, 0),
+    # runs of 9: prefix entries of 4, 4 and 1 member
+    ("groups-of-9", [400 + 37 * i for i in range(18)], 8, 2, 16, 128, 160, 9, 0),
+    ("gqa8-two-per-entry", [500, 700, 350, 900, 420, 610], 16, 2, 16, 128, 192, 3, 0),
+    ("gqa2-eight-per-entry", [330, 600, 470, 520, 710, 380, 450, 900, 640], 4, 2, 16, 64, 128, 9, 0),
+    ("gqa1-sixteen-per-entry", [200 + 20 * i for i in range(17)], 3, 3, 4, 32, 96, 17, 0),
+    # sinks not page-aligned: the first shared page holds sink positions
+    ("unaligned-sinks", [300, 410, 390, 520, 288], 8, 2, 7, 13, 64, 5, 0),
+    # the shared pages in several chunks (and members' own chunks after them)
+    ("prompt-in-chunks", [900, 1000, 700, 650, 1200, 880], 8, 2, 16, 128, 320, 3, 4),
+    ("no-protected-set", [300, 400, 500, 200], 8, 2, 0, 0, 128, 4, 3),
+]
+
+
+@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,P,grp,C", PREFIX_CASES,
+                         ids=[c[0] for c in PREFIX_CASES])
+def test_shared_prefix_read(name, lens, Hq, Hkv, S, R, P, grp, C):
+    """Groups of sequences whose page tables share their leading pages: with the
+    shared-prefix read, the shared pages are read once per group (prefix entries present)
+    and every sequence's attention is within the tolerance of the oracle, over two decode
+    steps; the same batch with the read off (the default) agrees with the oracle too."""
+    _, session, W = _mods()
+    wl = W.custom_workload(lens, num_q_heads=Hq, num_kv_heads=Hkv, num_sinks=S, num_recent=R,
+                           prompt_len=P, group_seqs=grp, seed=zlib.crc32(name.encode()) & 0xFFFF,
+                           outlier_channels=2, outlier_scale=8.0)
+    for prefix in ("shared", "off"):
+        sess = session.DecodeSession(wl, steps=2, keep_streams=range(len(lens)), chunk_pages=C,
+                                     prefix=prefix)
+        for s in range(2):
+            sess.append_step(s)
+            torch.cuda.synchronize()
+            check_attention(sess, range(len(lens)), step=s)
+            if prefix == "shared":
+                assert _prefix_entries(sess) > 0
+        sess.check_err()
+
+
+def test_bounded_wait_gives_up_without_a_fault():
+    """The error path of the bounded waits, run on a GPU without any fault: the testing
+    hook withholds the first copy of work item 0 (nothing is issued for it, so nothing is
+    in flight) and gives each wait 64 attempts. The call returns; the flag holds
+    KV4_DEVERR_TIMEOUT alone; item 0's partial state is empty, so its sequence's output is
+    the oracle's attention without that chunk's positions; every other sequence is computed
+    as usual; the hook is taken by that one call, and the next call matches the oracle
+    with no error (the context stays usable)."""
+    kv4, _, W = _mods()
+    lens, S, R, C = [2100, 1030, 40, 1500], 16, 128, 8
+    wl = W.custom_workload(lens, num_q_heads=8, num_kv_heads=2, num_sinks=S, num_recent=R,
+                           seed=5, outlier_channels=2, outlier_scale=8.0)
+    sess = make_session(wl, chunk_pages=C)
+    kv4._lib.kv4_test_withhold_copy(0, 64)
+    o16, o32, lse = run_attention(sess)
+    flag = int(sess.err.item())
+    assert flag == 32, kv4.decode_err(flag)
+    # work item 0 is the work list's first full INT4 chunk: sequence 0, region 1 (after its
+    # protected set), kv heads 0 and 1 in one entry
+    assert sess.workspace[256:272].view(torch.int32).cpu().tolist() == [0, 1, 0, 2]
+    k, v = sess.streams[0]
+    L = lens[0]
+    K, V = O.effective_kv(k[:L], v[:L], S, R)
+    keep = np.ones(L, bool)
+    keep[S:S + kv4.PAGE * C] = False  # the chunk's pages [1, 1 + C) hold positions 16 .. 143
+    oref, lref = O.attention(sess.q[0, 0].float().cpu().numpy(), K[keep], V[keep])
+    scale = np.abs(oref).max()
+    assert np.abs(o32[0] - oref).max() <= TOL * scale
+    assert np.all(np.abs(lse[0] - lref) <= TOL * np.maximum(1, np.abs(lref)))
+    check_attention(sess, [1, 2, 3], got=(o16, o32, lse))
+    sess.err.zero_()
+    check_attention(sess, range(len(lens)))
+    sess.check_err()
+
+
 def test_code_decisions_at_exact_ties():
     """Inputs whose code quotients are exact half-integers: INT4 positions on the grid
     x = j/4 with group min 0 and max 7.5 (scale exactly 0.5, so (x - min)/scale = j/2),
