@@ -523,7 +523,11 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
-            "gpu_launches": (5 if args.cache == "kv4" and args.prefix == "shared" else 4) * K * nl,
+            # per step and layer: plan, append, attention, merge (+ the lift kernel, and the
+        # prefix kernel with the shared-prefix read) for KV4-RL; plan, append, attention,
+        # merge for a comparison cache
+        "gpu_launches": (4 + (1 if args.cache == "kv4" else 0)
+                         + (1 if args.cache == "kv4" and args.prefix == "shared" else 0)) * K * nl,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

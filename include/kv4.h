@@ -162,12 +162,19 @@ typedef struct {
 /*
  * Bytes of device workspace kv4_decode_attention needs for a batch of num_seqs
  * sequences no longer than max_seq_len. Returns 0 for invalid arguments.
+ * (Infrastructure of this library: no passage of the pages defines it.)
  */
 size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len);
 
 /*
  * Quantise and append new tokens' K/V: the per-step write path (with n = 1 per
  * sequence), also usable for bulk prefill.
+ * Defined by: the whole context kept in calibration-free INT4 in a paged format, with
+ * INT8 copies of the attention-sink and recent positions (ai4snews summary,
+ * "Interpretation" para. 3; kipquest abstract, "calibration-free INT4 KV
+ * quantization"; aimodeling article, "INT4 as the base, INT8 insurance for critical
+ * positions": paged INT4 format, INT8 side cache). The demotion of a position leaving
+ * the recent window is the overwrite of its INT8 copy described below.
  *
  *   k_new, v_new: bf16 [total_new][Hkv][128], device.
  *   new_indptr:   int32 [num_seqs+1], device, CSR row ranges: rows new_indptr[b] ..
@@ -191,7 +198,12 @@ kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
                                int32_t *err_flag, kv4_stream_t stream);
 
 /*
- * Decode-step attention: for every sequence b and query head j,
+ * Decode-step attention. Defined by: attention over the INT4 pages and the INT8 copies
+ * of the protected positions through an integer attention path and an exact regional
+ * softmax merge (ai4snews summary, "Interpretation" para. 3), with higher-fidelity
+ * probability-value arithmetic on the protected positions (aimodeling article, "INT4 as
+ * the base, INT8 insurance for critical positions"). For every sequence b and query
+ * head j,
  *   O[b, j] = softmax(K_eff q / sqrt(128)) V_eff over positions [0, seq_lens[b]),
  * where K_eff/V_eff are the INT8 dequantised copies on protected positions and the
  * INT4 dequantised values elsewhere. Each region (the protected set, and each chunk of
@@ -208,7 +220,9 @@ kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
  *            (including the max); -inf for empty sequences (NULL to skip).
  *   workspace, ws_bytes: device scratch of at least kv4_workspace_size(cfg, num_seqs,
  *            max_seq_len) bytes, 256-byte aligned; contents need no initialisation.
- * A sequence of length 0 yields O = 0.
+ * A sequence of length 0 yields O = 0. The probability weights p * vscale enter the PV
+ * product in fp16; where the V scales are small (below 2^-6) they are lifted by an exact
+ * power of two first, so that small values keep fp16's relative precision.
  */
 kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool,
                                 const kv4_int8_side *side, const kv4_batch *batch,
@@ -261,10 +275,13 @@ kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offse
  * kv4_decode_attention, minus the workspace: the scratch space is a fixed array of
  * KV4_NOALLOC_SCRATCH_BYTES bytes in the library's device image, which every GPU that
  * loads the library holds until the process exits. Nothing is allocated or freed.
- *   - A batch whose kv4_workspace_size(cfg, num_seqs, max_seq_len) exceeds
- *     KV4_NOALLOC_SCRATCH_BYTES is rejected with KV4_ERR_WORKSPACE_TOO_SMALL.
+ *   - The call behaves as kv4_decode_attention given that array as a workspace of
+ *     KV4_NOALLOC_SCRATCH_BYTES bytes, the fall-back to 64-page chunks included: a batch
+ *     that does not fit even then is rejected with KV4_ERR_WORKSPACE_TOO_SMALL.
  *   - The first call on a device looks up the array's device address (with that device
  *     current); make that first call before capturing a stream into a CUDA graph.
+ *   - The address is kept for the device's primary context: do not use the call across
+ *     cudaDeviceReset (or another teardown of the primary context) in one process.
  *   - All calls share the one array per device: calls whose kernels overlap on the GPU
  *     (different streams without ordering between them) race and give wrong results.
  *     Calls ordered on one stream are safe; each call re-initialises what it reads.
@@ -275,7 +292,8 @@ kv4_status kv4_decode_attention_noalloc(const kv4_config *cfg, const kv4_int4_po
                                         const void *q, void *out, float *out_f32, float *lse,
                                         int32_t *err_flag, kv4_stream_t stream);
 
-/* Size of the fixed scratch array kv4_decode_attention_noalloc uses, in bytes. */
+/* Size of the fixed scratch array kv4_decode_attention_noalloc uses, in bytes. (The
+ * paper has no counterpart.) */
 size_t kv4_noalloc_scratch_bytes(void);
 
 /* ---------------------------------------------------------------------------------------
@@ -343,10 +361,11 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
  */
 void kv4_test_withhold_copy(int32_t item, uint32_t wait_limit);
 
-/* Human-readable name of a status code (static string). */
+/* Human-readable name of a status code (static string). (Infrastructure of this
+ * library: no passage of the pages defines it.) */
 const char *kv4_status_string(kv4_status status);
 
-/* Library version: major*10000 + minor*100 + patch. */
+/* Library version: major*10000 + minor*100 + patch. (Infrastructure: no passage.) */
 int32_t kv4_version(void);
 
 #ifdef __cplusplus

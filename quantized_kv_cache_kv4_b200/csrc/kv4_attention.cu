@@ -382,13 +382,31 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     *w.counter = 0;
     *w.pn_items = fits ? tot[5] : 0;          // then the prefix kernel's
     *w.pcounter = 0;
+    *w.lift_count = 0;
+    *w.lift_counter = 0;
     if (!fits) set_err(err, KV4_DEVERR_WORKSPACE);
   }
 }
 
+// How an entry's probability weights are formed (see lift_for_scale):
+//   kDecide  attn_kernel, every entry: no lift; when its last page's V scales are small
+//            enough to want one (lift >= kLiftMin; checked after the page loop, where it
+//            costs the loop nothing), the entry writes nothing and returns kWantLift (it
+//            goes on the lift list);
+//   kLifted  lift_kernel, for the listed entries: with the lift; returns kOverflow,
+//            having written nothing, when a later weight overflowed fp16;
+//   kPlain   lift_kernel, after an overflow: no lift and no decision.
+// The lifted arithmetic lives in its own kernel because attn_kernel runs at its register
+// limit: compiled into it, even unused, it slowed the main path by several percent.
+constexpr int kDecide = 0, kLifted = 1, kPlain = 2;
+constexpr int kDone = 0, kWantLift = 1, kOverflow = 2;
+constexpr float kLiftMin = 6.0f;  // lift only weights whose largest V scale is below 2^-6
+
 // ------------------------- INT8 protected set ----------------------------
 // One kv head's protected set: sink tiles then recent-ring tiles, INT8 codes.
-__device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c, const uint16_t *__restrict__ q,
+// Returns kDone, kWantLift (MODE kDecide) or kOverflow (MODE kLifted).
+template <int MODE>
+__device__ __forceinline__ int process_protected(WarpCtx &x, const CacheView &c, const uint16_t *__restrict__ q,
                                   int b, int h, int L, float *rec, int32_t *err) {
   const int G = c.gqa, H = c.num_kv_heads;
   const int lane = x.lane, gid = x.gid, tig = x.tig;
@@ -405,7 +423,7 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
       (ring_tiles && (ring < 0 || ring >= c.num_rings))) {
     if (lane == 0) set_err(err, KV4_DEVERR_SIDE_IDX);
     write_empty(rec, G, lane);
-    return;
+    return kDone;
   }
 
   auto issue = [&](int k) {
@@ -484,13 +502,23 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
   for (int cc = 0; cc < 8; ++cc) o[cc][0] = o[cc][1] = o[cc][2] = o[cc][3] = 0.f;
   const int ld_off = ((lane >> 4) * 256) + ((lane >> 3) & 1) * 128 + (lane & 7) * 16;
   const int ring_base = L - R;  // ring slot s holds position ring_base + ((s - ring_base) mod R)
+  float lift = 0.f;
+  if (MODE == kLifted) {  // the lift from the largest V scale of the first tile
+    if (!peek_stage(x, 0, err)) {
+      drain_copies(x, 0, npre, 0);
+      write_empty(rec, G, lane);
+      return kDone;
+    }
+    const uint16_t *v0 = reinterpret_cast<const uint16_t *>(x.stage0 + kOffVs8);
+    lift = lift_for_scale(page_max_scale(max(v0[gid], v0[gid + 8])));
+  }
 
   for (int k = 0; k < nt; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      drain_copies(x, k, min(nt, k + kStages));
+      drain_copies(x, k, min(nt, k + kStages), k);
       write_empty(rec, G, lane);
-      return;
+      return kDone;
     }
     uint8_t *sp = x.stage0 + st * kStageBytes;
     const uint32_t sa = smem_u32(sp);
@@ -526,7 +554,7 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
       s[hf][1] = valid ? d1 * sk * kq.y : -CUDART_INF_F;
     }
     float alpha[2];
-    softmax_step(s, m, l, alpha);
+    softmax_step(s, m, l, alpha, lift);
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc)
 #pragma unroll
@@ -566,6 +594,15 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
     if (k + kStages < nt) issue(k + kStages);
   }
 
+  if (MODE == kLifted) {
+    const float probe[2] = {o[0][0], o[0][1]};
+    if (any_not_finite(probe)) return kOverflow;
+  }
+  if (MODE == kDecide) {  // the last tile's V scales (still staged) ask for the lift?
+    const uint16_t *vl = reinterpret_cast<const uint16_t *>(
+        x.stage0 + ((nt - 1) % kStages) * kStageBytes + kOffVs8);
+    if (lift_for_scale(page_max_scale(max(vl[gid], vl[gid + 8]))) >= kLiftMin) return kWantLift;
+  }
 #pragma unroll
   for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -584,6 +621,7 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
       }
     }
   }
+  return kDone;
 }
 
 
@@ -598,7 +636,9 @@ __device__ __forceinline__ void process_protected(WarpCtx &x, const CacheView &c
 constexpr int kOffScale8P = 2 * kInt8CodeBytes;                       // scales of slot hs at +32 hs
 constexpr int kInt8PairBytes = 2 * kInt8CodeBytes + 2 * kInt8ScaleBytes;  // 4160 per stage
 
-__device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheView &c, const Workspace &w,
+// Returns kDone, kWantLift (MODE kDecide) or kOverflow (MODE kLifted).
+template <int MODE>
+__device__ __forceinline__ int process_protected_pair(WarpCtx &x, const CacheView &c, const Workspace &w,
                                        const uint16_t *__restrict__ q, int b, int h0, int nh,
                                        int L, int r, int32_t *err) {
   constexpr int CPH = 4;  // MMA columns per kv head slot
@@ -622,7 +662,7 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
       (ring_tiles && (ring < 0 || ring >= c.num_rings))) {
     if (lane == 0) set_err(err, KV4_DEVERR_SIDE_IDX);
     for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
-    return;
+    return kDone;
   }
 
   // copy k: tile k/2, K part (k even) or V part (k odd), both heads; a spare slot (one
@@ -660,7 +700,7 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
   // The bounded wait for copy k gave up: wait for the copies still in flight, write empty
   // states.
   auto give_up = [&](int k) {
-    drain_copies(x, k, issued);
+    drain_copies(x, k, issued, k);
     for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
   };
 
@@ -721,13 +761,26 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
   const int ring_base = L - R;  // ring slot s holds position ring_base + ((s - ring_base) mod R)
   const bool write_p0 = head_c_live && jc0 < G, write_p1 = head_c_live && jc0 + 1 < G;
   const bool col_live = (gid % CPH) < G && (gid / CPH) < nh;  // this lane's B column
+  float lift = 0.f;
+  if (MODE == kLifted) {  // the lift from the largest V scale of the first tile (copy 1)
+    if (!peek_stage(x, 1 % kStages, err)) {
+      drain_copies(x, 0, issued, 1);
+      for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+      return kDone;
+    }
+    const uint16_t *v0 = reinterpret_cast<const uint16_t *>(
+        x.stage0 + (1 % kStages) * kStageBytes + kOffScale8P + hs_c * kInt8ScaleBytes);
+    uint32_t mx = page_max_scale(max(v0[gid], v0[gid + 8]));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));  // one lift for both head slots
+    lift = lift_for_scale(mx);
+  }
 
   for (int j = 0; j < nt; ++j) {
     // ---- K part: logits ----
     const int kk = 2 * j;
     if (!wait_stage(x, kk % kStages, err)) {
       give_up(kk);
-      return;
+      return kDone;
     }
     const uint8_t *spk = x.stage0 + (kk % kStages) * kStageBytes;
     const uint32_t sak = smem_u32(spk);
@@ -776,7 +829,7 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-      const float mn = fmaxf(m[e], t);
+      const float mn = fmaxf(m[e], t - lift);  // running maximum kept as max - lift
       const bool mv = mn != m[e];
       a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
       moved |= mv;
@@ -799,7 +852,7 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
     const int kvc = 2 * j + 1;
     if (!wait_stage(x, kvc % kStages, err)) {
       give_up(kvc);
-      return;
+      return kDone;
     }
     const uint8_t *spv = x.stage0 + (kvc % kStages) * kStageBytes;
     const uint32_t sav = smem_u32(spv);
@@ -841,6 +894,17 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
   }
 
   // ---- finish: reduce the denominators over the 8 position lanes, write the partials ----
+  if (MODE == kLifted) {
+    const float probe[2] = {o[0][0], o[0][1]};
+    if (any_not_finite(probe)) return kOverflow;
+  }
+  if (MODE == kDecide) {  // the last tile's V scales (still staged) ask for the lift?
+    const uint16_t *vl = reinterpret_cast<const uint16_t *>(
+        x.stage0 + ((nv - 1) % kStages) * kStageBytes + kOffScale8P + hs_c * kInt8ScaleBytes);
+    uint32_t mx = page_max_scale(max(vl[gid], vl[gid + 8]));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (lift_for_scale(mx) >= kLiftMin) return kWantLift;
+  }
 #pragma unroll
   for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -862,6 +926,7 @@ __device__ __forceinline__ void process_protected_pair(WarpCtx &x, const CacheVi
       }
     }
   }
+  return kDone;
 }
 
 // ---------------------------- INT4 chunk --------------------------------
@@ -873,8 +938,9 @@ __device__ __forceinline__ int row_token_hi(int r) { return 8 + ((r + 4) & 7); }
 
 // One chunk of INT4 pages for HPW kv heads (h0 .. h0+nh-1, nh <= HPW). MMA column
 // col (0..7) belongs to head slot col / CPH and query j = col % CPH of that head.
-template <int HPW>
-__device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
+// Returns kDone, kWantLift (MODE kDecide) or kOverflow (MODE kLifted).
+template <int HPW, int MODE>
+__device__ __forceinline__ int process_int4(WarpCtx &x, const CacheView &c, const Workspace &w,
                              const uint16_t *__restrict__ q, int b, int h0, int nh, int r,
                              int chunk, const Regions &rg, int32_t *err) {
   constexpr int CPH = 8 / HPW;  // MMA columns per kv head slot
@@ -899,7 +965,7 @@ __device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, con
   if (__any_sync(0xffffffffu, bad)) {
     if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
     for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
-    return;
+    return kDone;
   }
 
   // stage layout: K codes [HPW][1024] | V codes [HPW][1024] | K params [HPW][256] | V params
@@ -1035,13 +1101,32 @@ __device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, con
   const int vp_off = kOffVp + hs_c * kInt4ParamBytes;
   const bool write_p0 = head_c_live && jc0 < G, write_p1 = head_c_live && jc0 + 1 < G;
   uint32_t *pt_mine = x.ptile + (hs_c * 4 * 8 + 2 * tig) * kPWordsPerCol + gid;
+  // the largest V scale of the page staged at `st` over the warp (both head slots)
+  auto page_scale = [&](int st) {
+    const uint8_t *sp = x.stage0 + st * kStageBytes;
+    const uint4 v0 = *reinterpret_cast<const uint4 *>(sp + vp_off + t0 * 16);
+    const uint4 v1 = *reinterpret_cast<const uint4 *>(sp + vp_off + t1 * 16);
+    uint32_t mx = page_max_scale(__vmaxu2(__vmaxu2(__vmaxu2(v0.x, v0.y), __vmaxu2(v0.z, v0.w)),
+                                          __vmaxu2(__vmaxu2(v1.x, v1.y), __vmaxu2(v1.z, v1.w))));
+    if (HPW == 2) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    return mx;
+  };
+  float lift = 0.f;
+  if (MODE == kLifted) {  // the lift from the largest V scale of the first page
+    if (!peek_stage(x, 0, err)) {
+      drain_copies(x, 0, npre, 0);
+      for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+      return kDone;
+    }
+    lift = lift_for_scale(page_scale(0));
+  }
 
   for (int k = 0; k < np; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      drain_copies(x, k, min(np, k + kStages));
+      drain_copies(x, k, min(np, k + kStages), k);
       for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
-      return;
+      return kDone;
     }
     uint8_t *sp = x.stage0 + st * kStageBytes;
     const uint32_t sa = smem_u32(sp);
@@ -1105,7 +1190,7 @@ __device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, con
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
       t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-      const float mn = fmaxf(m[e], t);
+      const float mn = fmaxf(m[e], t - lift);  // running maximum kept as max - lift
       const bool mv = mn != m[e];
       a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
       moved |= mv;
@@ -1172,6 +1257,14 @@ __device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, con
   }
 
   // ---- finish: reduce per-thread sums over the 8 token lanes, write the partial ----
+  if (MODE == kLifted) {
+    const float probe[8] = {o[0][0][0], o[0][0][1], o[1][0][0], o[1][0][1],
+                            o[2][0][0], o[2][0][1], o[3][0][0], o[3][0][1]};
+    if (any_not_finite(probe)) return kOverflow;
+  }
+  // the last page's V scales (still staged) ask for the lift?
+  if (MODE == kDecide && lift_for_scale(page_scale((np - 1) % kStages)) >= kLiftMin)
+    return kWantLift;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
 #pragma unroll
@@ -1205,6 +1298,7 @@ __device__ __forceinline__ void process_int4(WarpCtx &x, const CacheView &c, con
       }
     }
   }
+  return kDone;
 }
 
 // ---------------------------------------------------------------------------
@@ -1235,8 +1329,11 @@ static_assert(kPfxOffQs + 2 * 4 * 32 * 8 <= kStages * kStageBytes,
               "the shared-prefix ring and query operands fit the warp's stage area");
 static_assert(2 * 4 * 8 * kPWordsPerCol * 4 == kPtileBytes, "two N tiles of P'");
 
-// Prompt chunk ci of kv head h for the nmem group members b0 .. b0+nmem-1.
-__device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, const Workspace &w,
+// Prompt chunk ci of kv head h for the nmem group members b0 .. b0+nmem-1. Returns true
+// when the lift chosen on the first page overflowed a later weight: the entry is then to
+// be redone with LIFT = false (nothing was written).
+template <bool LIFT>
+__device__ __forceinline__ bool process_prefix(WarpCtx &x, const CacheView &c, const Workspace &w,
                                const uint16_t *__restrict__ q, int b0, int ci, int h, int nmem,
                                int32_t *err) {
   const int G = c.gqa, H = c.num_kv_heads;
@@ -1276,7 +1373,7 @@ __device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, c
   if (__any_sync(0xffffffffu, bad)) {
     if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
     write_empty_all();
-    return;
+    return false;
   }
 
   auto issue = [&](int k) {
@@ -1369,13 +1466,25 @@ __device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, c
                                       : ((r8 & 1) ? 12 + (r8 >> 1) : (r8 >> 1))) * 16;
   const int t0 = gid, t1 = row_token_hi(gid);
   uint32_t *pt_mine = x.ptile + (2 * tig) * kPWordsPerCol + gid;
+  float lift = 0.f;
+  if (LIFT) {  // the lift from the largest V scale of the first page
+    if (!peek_stage(x, 0, err)) {
+      drain_copies(x, 0, npre, 0);
+      write_empty_all();
+      return false;
+    }
+    const uint4 v0 = *reinterpret_cast<const uint4 *>(x.stage0 + kPfxOffVp + t0 * 16);
+    const uint4 v1 = *reinterpret_cast<const uint4 *>(x.stage0 + kPfxOffVp + t1 * 16);
+    lift = lift_for_scale(page_max_scale(__vmaxu2(__vmaxu2(__vmaxu2(v0.x, v0.y), __vmaxu2(v0.z, v0.w)),
+                                                  __vmaxu2(__vmaxu2(v1.x, v1.y), __vmaxu2(v1.z, v1.w)))));
+  }
 
   for (int k = 0; k < np; ++k) {
     const int st = k % kStages;
     if (!wait_stage(x, st, err)) {
-      drain_copies(x, k, min(np, k + kStages));
+      drain_copies(x, k, min(np, k + kStages), k);
       write_empty_all();
-      return;
+      return false;
     }
     const uint8_t *sp = x.stage0 + st * kPfxStageBytes;
     const uint32_t sa = smem_u32(sp);
@@ -1448,7 +1557,7 @@ __device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, c
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-        const float mn = fmaxf(m[t][e], v);
+        const float mn = fmaxf(m[t][e], v - lift);  // running maximum kept as max - lift
         const bool mv = mn != m[t][e];
         a[t][e] = mv ? fast_exp2(m[t][e] - mn) : 1.0f;
         moved |= mv;
@@ -1519,6 +1628,13 @@ __device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, c
   }
 
   // ---- finish: reduce over the 8 token lanes, write each member's partial ----
+  if (LIFT) {
+    const float probe[16] = {o[0][0][0][0], o[0][0][0][1], o[0][0][1][0], o[0][0][1][1],
+                             o[1][0][0][0], o[1][0][0][1], o[1][0][1][0], o[1][0][1][1],
+                             o[2][0][0][0], o[2][0][0][1], o[2][0][1][0], o[2][0][1][1],
+                             o[3][0][0][0], o[3][0][0][1], o[3][0][1][0], o[3][0][1][1]};
+    if (any_not_finite(probe)) return true;
+  }
 #pragma unroll
   for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -1552,6 +1668,7 @@ __device__ __forceinline__ void process_prefix(WarpCtx &x, const CacheView &c, c
         rr[kHeadDim + 1] = l[t][e];
       }
     }
+  return false;
 }
 
 __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(CacheView c, Workspace w,
@@ -1582,7 +1699,8 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
     item = __shfl_sync(0xffffffffu, item, 0);
     if (item >= n_items) break;
     const int4 en = w.entries[base + item];
-    process_prefix(x, c, w, q, en.x, -1 - en.y, en.z, en.w, err);
+    if (process_prefix<true>(x, c, w, q, en.x, -1 - en.y, en.z, en.w, err))
+      process_prefix<false>(x, c, w, q, en.x, -1 - en.y, en.z, en.w, err);
     if (x.dead) break;
   }
 }
@@ -1705,13 +1823,72 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
     const int L = c.seq_lens[b];
     const int pe = w.prefix_end ? w.prefix_end[b] : 0;
     const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages, pe);
+    int res;
     if (r < rg.has_prot) {
       if constexpr (HPW == 2)
-        process_protected_pair(x, c, w, q, b, h0, nh, L, r, err);
+        res = process_protected_pair<kDecide>(x, c, w, q, b, h0, nh, L, r, err);
       else
-        process_protected(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
-    } else
-      process_int4<HPW>(x, c, w, q, b, h0, nh, r, r - rg.has_prot - rg.n_prompt, rg, err);
+        res = process_protected<kDecide>(x, c, q, b, h0, L, record_of(w, H, G, b, h0, r), err);
+    } else {
+      res = process_int4<HPW, kDecide>(x, c, w, q, b, h0, nh, r, r - rg.has_prot - rg.n_prompt,
+                                       rg, err);
+    }
+    if (res == kWantLift && x.lane == 0) w.lift_items[atomicAdd(w.lift_count, 1)] = item;
+    if (x.dead) break;
+  }
+}
+
+// The entries of the lift list (small V scales): redone with the lift of their weights,
+// and again without it if a later weight overflowed fp16 under the lift.
+template <int HPW>
+__global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) lift_kernel(CacheView c, Workspace w,
+                                                                           const uint16_t *__restrict__ q,
+                                                                           int32_t *err) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int n_items = *w.lift_count;
+  if (n_items == 0) return;
+  WarpCtx x;
+  const int warp = threadIdx.x >> 5;
+  x.lane = threadIdx.x & 31;
+  x.gid = x.lane >> 2;
+  x.tig = x.lane & 3;
+  uint8_t *mine = smem + warp * kWarpSmem;
+  x.stage0 = mine;
+  x.ptile = reinterpret_cast<uint32_t *>(mine + kStages * kStageBytes);
+  x.ptile8 = reinterpret_cast<uint16_t *>(mine + kStages * kStageBytes + kPtileBytes);
+  x.bars = reinterpret_cast<uint64_t *>(mine + kStages * kStageBytes + kPtileBytes + kPtile8Bytes);
+  init_warp<false>(x, w);
+  for (int i = x.lane; i < kPtileBytes / 4; i += 32) x.ptile[i] = 0u;
+  if (x.lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&x.bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const int H = c.num_kv_heads, G = c.gqa;
+  for (;;) {
+    int i = 0;
+    if (x.lane == 0) i = atomicAdd(w.lift_counter, 1);
+    i = __shfl_sync(0xffffffffu, i, 0);
+    if (i >= n_items) break;
+    const int4 en = w.entries[w.lift_items[i]];
+    const int b = en.x, r = en.y, h0 = en.z, nh = en.w;
+    const int L = c.seq_lens[b];
+    const int pe = w.prefix_end ? w.prefix_end[b] : 0;
+    const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages, pe);
+    if (r < rg.has_prot) {
+      if constexpr (HPW == 2) {
+        if (process_protected_pair<kLifted>(x, c, w, q, b, h0, nh, L, r, err) == kOverflow)
+          process_protected_pair<kPlain>(x, c, w, q, b, h0, nh, L, r, err);
+      } else {
+        float *rec = record_of(w, H, G, b, h0, r);
+        if (process_protected<kLifted>(x, c, q, b, h0, L, rec, err) == kOverflow)
+          process_protected<kPlain>(x, c, q, b, h0, L, rec, err);
+      }
+    } else {
+      const int chunk = r - rg.has_prot - rg.n_prompt;
+      if (process_int4<HPW, kLifted>(x, c, w, q, b, h0, nh, r, chunk, rg, err) == kOverflow)
+        process_int4<HPW, kPlain>(x, c, w, q, b, h0, nh, r, chunk, rg, err);
+    }
     if (x.dead) break;
   }
 }
@@ -1770,13 +1947,41 @@ cudaError_t launch_prefix(const CacheView &c, const Workspace &w, const uint16_t
 
 int heads_per_warp_for(int gqa) { return gqa <= 4 ? 2 : 1; }
 
+// The persistent grid of the attention kernel: an empty list costs a launch whose CTAs
+// end at once (about 3 us), a long one (small values everywhere) runs at full width.
+template <int HPW>
+static cudaError_t launch_lift_t(const CacheView &c, const Workspace &w, const uint16_t *q,
+                                 int32_t *err_flag, cudaStream_t s) {
+  static PerDevice grids;
+  int grid = 0;
+  cudaError_t e = once_per_device(grids, [](int dev, int *g) {
+    cudaError_t r = cudaFuncSetAttribute(lift_kernel<HPW>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kCtaSmem);
+    int sms = 0, per_sm = 0;
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lift_kernel<HPW>, kWarps * 32,
+                                                        kCtaSmem);
+    *g = sms * (per_sm > 0 ? per_sm : 1);
+    return r;
+  }, &grid);
+  if (e != cudaSuccess) return e;
+  lift_kernel<HPW><<<grid, kWarps * 32, kCtaSmem, s>>>(c, w, q, err_flag);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
                              int32_t *err_flag, cudaStream_t s) {
+  cudaError_t e;
   if (w.fault_item >= 0)  // the testing hook is armed for this call
-    return w.heads_per_warp == 2 ? launch_attn_t<2, true>(c, w, q, err_flag, s)
-                                 : launch_attn_t<1, true>(c, w, q, err_flag, s);
-  return w.heads_per_warp == 2 ? launch_attn_t<2, false>(c, w, q, err_flag, s)
-                               : launch_attn_t<1, false>(c, w, q, err_flag, s);
+    e = w.heads_per_warp == 2 ? launch_attn_t<2, true>(c, w, q, err_flag, s)
+                              : launch_attn_t<1, true>(c, w, q, err_flag, s);
+  else
+    e = w.heads_per_warp == 2 ? launch_attn_t<2, false>(c, w, q, err_flag, s)
+                              : launch_attn_t<1, false>(c, w, q, err_flag, s);
+  if (e != cudaSuccess) return e;
+  return w.heads_per_warp == 2 ? launch_lift_t<2>(c, w, q, err_flag, s)
+                               : launch_lift_t<1>(c, w, q, err_flag, s);
 }
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
@@ -1798,11 +2003,13 @@ size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_hea
   const long long cap = static_cast<long long>(num_seqs) * per_seq;
   const long long cap_e = cap * num_kv_heads;
   auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
-  size_t off = 256;  // counter, n_items, prefix counter, prefix n_items
+  size_t off = 256;  // counters and counts (work, prefix work, lift list)
   const size_t ent_off = off;
   off = up(off + static_cast<size_t>(cap_e) * sizeof(int4));
   const size_t units_off = off;
   off = up(off + (static_cast<size_t>(num_seqs) * num_kv_heads + 1) * sizeof(int32_t));
+  const size_t lift_off = off;  // the lift list: at most one per entry
+  off = up(off + static_cast<size_t>(cap_e) * sizeof(int32_t));
   size_t pend_off = 0;
   if (prefix) {
     pend_off = off;
@@ -1816,6 +2023,9 @@ size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_hea
     carve->n_items = reinterpret_cast<int32_t *>(p) + 1;
     carve->pcounter = reinterpret_cast<int32_t *>(p) + 2;
     carve->pn_items = reinterpret_cast<int32_t *>(p) + 3;
+    carve->lift_count = reinterpret_cast<int32_t *>(p) + 4;
+    carve->lift_counter = reinterpret_cast<int32_t *>(p) + 5;
+    carve->lift_items = reinterpret_cast<int32_t *>(p + lift_off);
     carve->entries = reinterpret_cast<int4 *>(p + ent_off);
     carve->unit_offsets = reinterpret_cast<int32_t *>(p + units_off);
     carve->prefix_end = prefix ? reinterpret_cast<int32_t *>(p + pend_off) : nullptr;

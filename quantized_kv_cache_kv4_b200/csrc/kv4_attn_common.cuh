@@ -99,17 +99,54 @@ __device__ __forceinline__ bool prologue_copy(const WarpCtx &x, int k) {
   return !(x.fault && k == 0);
 }
 
+// Power-of-two lift of the probability weights P' = p * vscale of one work entry, in
+// log2 units. P' is rounded to fp16 for the PV product, and below 2^-14 an fp16 keeps
+// only 2^-24 of absolute precision; with small values (vscale well below 1) most weights
+// would land there. So the weights are computed as p * 2^E * vscale, with E chosen from
+// the largest V scale s_max on the entry's first page so that s_max * 2^E < 1 (E = 0
+// when s_max >= 1/2, at most 24). The lift needs no correction afterwards: the online
+// softmax keeps its running maximum as m - E, so p arrives as exp2(s - (m - E)) and the
+// partial state (m - E, l 2^E, acc 2^E) is the same state as (m, l, acc) for the exact
+// merge. A later page whose scale would overflow fp16 under the lift makes the kernel
+// redo the entry without it. bits: the fp16 bits of s_max (non-negative).
+__device__ __forceinline__ float lift_for_scale(uint32_t bits) {
+  if (bits == 0u) return 0.f;
+  const float sm = __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+  const int e = static_cast<int>((__float_as_uint(sm) >> 23) & 0xFFu) - 127;  // [2^e, 2^(e+1))
+  return static_cast<float>(min(24, max(0, -1 - e)));
+}
+
+// The largest of the fp16 values v0 .. v7 (non-negative fp16 bits in the low halves of
+// the words, anything in the high halves) over the lanes that share this lane's tig:
+// the V scales of one page's tokens.
+__device__ __forceinline__ uint32_t page_max_scale(uint32_t m) {
+  m &= 0xFFFFu;
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+  return m;
+}
+
+// Whether any of n accumulators of the warp is not finite (an fp16 weight overflowed).
+template <int N>
+__device__ __forceinline__ bool any_not_finite(const float (&v)[N]) {
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < N; ++i) bad |= !(fabsf(v[i]) <= 3.0e38f);
+  return __any_sync(0xffffffffu, bad);
+}
+
 // Online softmax update for this thread's two heads (2tig, 2tig+1) with logits of
 // tokens (gid, gid+8) in log2 units. Returns p in s[][] and the rescale factors.
 __device__ __forceinline__ void softmax_step(float (&s)[2][2], float (&m)[2], float (&l)[2],
-                                             float (&alpha)[2]) {
+                                             float (&alpha)[2], float lift = 0.f) {
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     float t = fmaxf(s[0][e], s[1][e]);
     t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
     t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
     t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-    const float mn = fmaxf(m[e], t);
+    const float mn = fmaxf(m[e], t - lift);  // running maximum kept as max - lift
     alpha[e] = fast_exp2(m[e] - mn);
     m[e] = mn;
     s[0][e] = fast_exp2(s[0][e] - mn);
@@ -130,18 +167,28 @@ __device__ __forceinline__ bool wait_stage(WarpCtx &x, int stage, int32_t *err) 
   return ok;
 }
 
-// After the wait for copy `from` gave up: wait for copies from .. to-1 (every copy of the
-// entry issued and not yet waited for, the one that timed out included, with the parity
-// its wait had before it flipped), each up to 16 times the normal limit, so that none
-// lands in shared memory after the warp (and possibly its CTA) has finished. A copy that
-// does not complete even then is left behind; the TIMEOUT bit already marks the call's
-// results as void. The warp takes no further work, so the parities are not kept.
-__device__ inline void drain_copies(const WarpCtx &x, int from, int to) {
+// Waits for the next completion of `stage` like wait_stage, but on success leaves the
+// stage's parity as it was, so that the page loop's own wait on it returns at once.
+__device__ __forceinline__ bool peek_stage(WarpCtx &x, int stage, int32_t *err) {
+  if (mbar_wait_bounded(&x.bars[stage], (x.parity >> stage) & 1u, x.wait_limit)) return true;
+  x.parity ^= 1u << stage;
+  x.dead = true;
+  if (x.lane == 0) set_err(err, KV4_DEVERR_TIMEOUT);
+  return false;
+}
+
+// After the wait for copy `failed` gave up: wait for copies from .. to-1 (every copy of
+// the entry issued and not yet waited for, the one that timed out included, with the
+// parity its wait had before it flipped), each up to 16 times the normal limit, so that
+// none lands in shared memory after the warp (and possibly its CTA) has finished. A copy
+// that does not complete even then is left behind; the TIMEOUT bit already marks the
+// call's results as void. The warp takes no further work, so the parities are not kept.
+__device__ inline void drain_copies(const WarpCtx &x, int from, int to, int failed) {
   const uint32_t longer = x.wait_limit > 0x0FFFFFFFu ? 0xFFFFFFFFu : x.wait_limit * 16u;
   for (int k = from; k < to; ++k) {
     if (!prologue_copy(x, k)) continue;  // withheld by the testing hook: never issued
     const int st = k % kStages;
-    const uint32_t par = ((x.parity >> st) & 1u) ^ (k == from ? 1u : 0u);
+    const uint32_t par = ((x.parity >> st) & 1u) ^ (k == failed ? 1u : 0u);
     mbar_wait_bounded(&x.bars[st], par, longer);
   }
 }

@@ -147,7 +147,7 @@ __device__ __forceinline__ void process_baseline(WarpCtx &x, const CacheView &c,
   for (int k = 0; k < issued; ++k)
     if (prologue_copy(x, k)) issue(k);
   auto give_up = [&](int k) {
-    drain_copies(x, k, issued);
+    drain_copies(x, k, issued, k);
     write_empty(rec, G, lane);
   };
 

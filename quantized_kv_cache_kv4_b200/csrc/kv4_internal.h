@@ -79,6 +79,9 @@ struct Workspace {
   int32_t *prefix_end;     // [num_seqs] end page of the group's shared INT4 pages, 0 = none
   int32_t *pcounter;       // [1] dynamic work counter of the prefix kernel
   int32_t *pn_items;       // [1] shared-prefix entries (listed after the n_items others)
+  int32_t *lift_count;     // [1] entries on the lift list (small V scales)
+  int32_t *lift_counter;   // [1] dynamic work counter of the lift kernel
+  int32_t *lift_items;     // [cap_entries] work items on the lift list
   uint32_t wait_limit;     // attempts of one bounded wait for a copy (kWaitLimit)
   int32_t fault_item;      // testing hook: work item whose first copy is withheld, -1 none
 };

@@ -21,6 +21,8 @@ __device__ __align__(256) unsigned char kv4_static_scratch[kStaticScratchBytes];
 
 // Device address of the array, looked up once per device. In host code the array's
 // name is only a stand-in, never a device address, so kernels get the looked-up pointer.
+// The address belongs to the device's primary context as it was at the first call: after
+// cudaDeviceReset (a new primary context) it is stale, which kv4.h states as a limit.
 constexpr int kMaxDevices = 64;
 void *g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
@@ -51,11 +53,10 @@ kv4_status kv4_decode_attention_noalloc(const kv4_config *cfg, const kv4_int4_po
                                         const kv4_int8_side *side, const kv4_batch *batch,
                                         const void *q, void *out, float *out_f32, float *lse,
                                         int32_t *err_flag, kv4_stream_t stream) {
-  // The argument checks and the size of the work are those of kv4_decode_attention.
+  // The argument checks, the size of the work and the refusal of a batch too large for
+  // the array (after the fall-back to 64-page chunks) are kv4_decode_attention's own,
+  // given the array as a workspace of kStaticScratchBytes.
   if (cfg == nullptr || batch == nullptr) return KV4_ERR_INVALID_ARG;
-  const size_t need = kv4_workspace_size(cfg, batch->num_seqs, batch->max_seq_len);
-  if (need == 0 && batch->num_seqs > 0) return KV4_ERR_INVALID_ARG;
-  if (need > kStaticScratchBytes) return KV4_ERR_WORKSPACE_TOO_SMALL;
   void *scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return KV4_ERR_CUDA;
   return kv4_decode_attention(cfg, pool, side, batch, q, out, out_f32, lse, scratch,

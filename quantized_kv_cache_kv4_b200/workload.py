@@ -59,6 +59,8 @@ class Workload:
     kv_dist: str = "normal"  # "normal" | "student_t3"
     outlier_channels: int = 0  # key channels per KV head that are scaled up
     outlier_scale: float = 1.0
+    v_scale: float = 1.0  # values drawn with this standard deviation (keys stay at 1)
+    v_small_tokens: int = 0  # v_scale applies to the first this many positions (0 = all)
     prompt_len: int = 0  # shared prompt prefix length (multiple of PAGE_SIZE), 0 = none
     group_seqs: int = 1  # sequences sharing one prompt
     num_layers: int = 1
@@ -143,12 +145,14 @@ def make_workload(name: str) -> Workload:
 
 def custom_workload(seq_lens, num_q_heads=8, num_kv_heads=2, num_sinks=4, num_recent=32,
                     seed=7, kv_dist="normal", outlier_channels=0, outlier_scale=1.0,
-                    prompt_len=0, group_seqs=1, name="custom") -> Workload:
+                    prompt_len=0, group_seqs=1, name="custom", v_scale=1.0,
+                    v_small_tokens=0) -> Workload:
     return Workload(name=name, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
                     num_sinks=num_sinks, num_recent=num_recent,
                     seq_lens=np.asarray(seq_lens, dtype=np.int64), seed=seed,
                     kv_dist=kv_dist, outlier_channels=outlier_channels,
-                    outlier_scale=outlier_scale, prompt_len=prompt_len,
+                    outlier_scale=outlier_scale, v_scale=v_scale,
+                    v_small_tokens=v_small_tokens, prompt_len=prompt_len,
                     group_seqs=group_seqs)
 
 
@@ -188,6 +192,11 @@ def _stream(wl: Workload, stream_id: int, n: int, layer: int, device):
             scale = torch.ones(wl.num_kv_heads, wl.head_dim, device=dev)
             scale.scatter_(1, ids, wl.outlier_scale)
             x = x * scale
+        if kind == "v" and wl.v_scale != 1.0:
+            if wl.v_small_tokens:
+                x[:wl.v_small_tokens] *= wl.v_scale
+            else:
+                x = x * wl.v_scale
         out.append(x.to(torch.bfloat16))
     return out[0], out[1]
 

@@ -262,6 +262,48 @@ def test_shared_prefix_read(name, lens, Hq, Hkv, S, R, P, grp, C):
         sess.check_err()
 
 
+SMALL_V = [
+    # name, lens, Hq, Hkv, S, R, prefix
+    ("int4-int8-gqa4", [600, 2000, 150, 900], 8, 2, 16, 128, "off"),
+    ("one-head-per-warp-gqa8", [700, 1500, 300], 16, 2, 16, 128, "off"),
+    ("shared-prefix", [700, 900, 610, 1300], 8, 2, 16, 128, "shared"),
+]
+
+
+@pytest.mark.parametrize("sigma", [1e-2, 1e-3, 1e-4])
+@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,prefix", SMALL_V, ids=[c[0] for c in SMALL_V])
+def test_small_values(name, lens, Hq, Hkv, S, R, prefix, sigma):
+    """Values V ~ N(0, sigma^2): the probability weights P' = p * vscale would fall into the
+    fp16 subnormal range; the power-of-two lift per work entry keeps them normal. The
+    attention output must stay within the tolerance of the oracle in the INT4 region, the
+    INT8 protected set and the shared-prefix read alike."""
+    _, session, W = _mods()
+    wl = W.custom_workload(lens, num_q_heads=Hq, num_kv_heads=Hkv, num_sinks=S, num_recent=R,
+                           seed=int(-np.log10(sigma)) + 31, outlier_channels=2,
+                           outlier_scale=8.0, v_scale=sigma,
+                           prompt_len=256 if prefix == "shared" else 0,
+                           group_seqs=2 if prefix == "shared" else 1)
+    sess = make_session(wl, prefix=prefix)
+    worst = check_attention(sess, range(len(lens)))
+    assert worst <= TOL
+    sess.check_err()
+
+
+def test_lift_overflow_is_redone_without_the_lift():
+    """An entry whose first page has tiny values (sigma 1e-6) and later pages unit ones:
+    the lift chosen on the first page (2^21 or more) would overflow the later weights in
+    fp16, so the kernel redoes the entry without it. 64-page chunks put positions
+    16 .. 1039 in one entry (tiny up to 511); the INT8 protected set starts with a tiny
+    sink tile and ends with a unit ring. The output must match the oracle (no inf, no
+    NaN)."""
+    _, session, W = _mods()
+    wl = W.custom_workload([1800, 1400, 700], num_q_heads=8, num_kv_heads=2, num_sinks=16,
+                           num_recent=128, seed=77, v_scale=1e-6, v_small_tokens=512)
+    sess = make_session(wl, chunk_pages=64)
+    check_attention(sess, range(3))
+    sess.check_err()
+
+
 def test_bounded_wait_gives_up_without_a_fault():
     """The error path of the bounded waits, run on a GPU without any fault: the testing
     hook withholds the first copy of work item 0 (nothing is issued for it, so nothing is
