@@ -254,6 +254,46 @@ def oracle_sample(wl, budget_s: float, start_seq: int = 0, cache: str = "kv4",
     return units, spent, desc, threads, quant
 
 
+def bench_config(wl, cache, world):
+    """The `config` both arms print: the workload, the cache, how L2 is kept from serving
+    the timed reads, and the data parallelism (so the two arms' lines compare key for key)."""
+    ub, _ = attention_bytes(wl, wl.seq_lens, cache)
+    return {"workload": wl.name, **wl.describe(), "cache": cache,
+            "l2": "inputs larger than L2: the cache read per step is "
+                  f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
+            "parallelism": f"dp{world} (independent replica batches)"}
+
+
+def output_check(sess, step, nseq=8, seed=5):
+    """The attention output of one decode step (in sess.out) against the oracle on a
+    seeded sample of sequences: the worst error of the bf16 output beyond half a bf16 ulp
+    of the reference, relative to the sample's max |O_ref|, and whether it is within the
+    2e-3 tolerance."""
+    from oracle import kv4_oracle as O
+    from quantized_kv_cache_kv4_b200.workload import seq_kv
+    wl = sess.wl
+    rng = np.random.default_rng(seed)
+    seqs = sorted(rng.choice(wl.num_seqs, size=min(nseq, wl.num_seqs), replace=False).tolist())
+    out = sess.out.float().cpu().numpy()
+    refs = {}
+    for b in seqs:
+        L = int(sess.L0[b]) + step
+        k, v = seq_kv(wl, b, L, sess.layer, sess.device)
+        q = sess.q[step, b].float().cpu().numpy()
+        refs[b] = O.decode_reference(q, k.float().cpu().numpy(), v.float().cpu().numpy(),
+                                     wl.num_sinks, wl.num_recent, sess.demotion)[0]
+    scale = max(float(np.abs(r).max()) for r in refs.values())
+    worst = 0.0
+    for b, ref in refs.items():
+        a = np.abs(ref)
+        half_ulp = np.where(a > 0, 2.0 ** (np.floor(np.log2(np.maximum(a, 1e-38))) - 8), 0.0)
+        worst = max(worst, float((np.abs(out[b] - ref) - half_ulp).max()) / scale)
+    return {"step": int(step), "sequences": len(seqs), "max_err_over_scale": worst,
+            "tol": 2e-3, "passed": bool(worst <= 2e-3),
+            "what": "bf16 output of the last timed step (layer 0) against the oracle, beyond "
+                    "half a bf16 ulp, relative to max |O_ref| of the sample"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -273,7 +313,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * total_s / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, **wl.describe(), "cache": args.cache},
+        "config": bench_config(wl, args.cache, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": descs[0] if descs else ""},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -374,6 +414,10 @@ def run_gpu(args, rank, world, local_rank):
     layers = [sess] + [make_session(wl, layer=li, steps=W + K, device=dev,
                                     workspace=sess.workspace)
                        for li in range(1, wl.num_layers)]
+    # the layers after the first of a step reuse its work list (same lengths and paging;
+    # the layers' calls run in order on one stream and share the workspace)
+    for ls in layers[1:]:
+        ls.plan_reuse = args.plan_reuse == "on"
     nl = len(layers)
     stream = torch.cuda.current_stream(dev)
     H = wl.num_kv_heads
@@ -448,6 +492,11 @@ def run_gpu(args, rank, world, local_rank):
     ms_eager_max, _ = combine_ranks(ms_eager, 0, world, dev)
     ms_calls_max, _ = combine_ranks(ms_calls, 0, world, dev)
 
+    # ---- the last timed step's output against the oracle (rank 0, KV4-RL cache): the
+    # timed passes replay steps that already ran, but after the last pass layer 0's
+    # output holds step W+K-1, whose recent window no later token has overwritten ----
+    check = output_check(layers[0], W + K - 1) if rank == 0 and args.cache == "kv4" else None
+
     # ---- roofline of the attention call (plan + split-K attention + merge) ----
     uniq = [attention_bytes(wl, L0 + s, args.cache) for s in range(W, W + K)]
     mean_att_s = statistics.mean(att_ms) / 1000.0
@@ -497,13 +546,11 @@ def run_gpu(args, rank, world, local_rank):
             "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[args.cache],
             "data": "synthetic",
-            "config": {"workload": wl.name, **wl.describe(),
-                       "l2": "inputs larger than L2: the cache read per step is "
-                             f"{ub / 1e9:.2f} GB (L2 is 126 MB)",
-                       "cache": args.cache,
-                       "parallelism": f"dp{world} (independent replica batches)",
-                       "step": "one kv4_decode_step call per layer (append + attention; "
-                               "the work list built on a second stream beside the append)",
+            "config": bench_config(wl, args.cache, world),
+            "method": {"step": "one kv4_decode_step call per layer (append + attention; "
+                               "the work list built on a second stream beside the append"
+                               + ("; layers after the first reuse the first layer's work list"
+                                  if nl > 1 and args.plan_reuse == "on" else "") + ")",
                        "launch": {"graph": "cuda graph per call, replayed (each layer's "
                                            "call of every step)",
                                   "eager": "eager"}[args.launch]},
@@ -523,11 +570,13 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
+            "output_check": check,
             # per step and layer: plan, append, attention, merge (+ the lift kernel, and the
-        # prefix kernel with the shared-prefix read) for KV4-RL; plan, append, attention,
-        # merge for a comparison cache
-        "gpu_launches": (4 + (1 if args.cache == "kv4" else 0)
-                         + (1 if args.cache == "kv4" and args.prefix == "shared" else 0)) * K * nl,
+            # prefix kernel with the shared-prefix read) for KV4-RL; plan, append,
+            # attention, merge for a comparison cache
+            "gpu_launches": ((4 + (1 if args.cache == "kv4" else 0)
+                              + (1 if args.cache == "kv4" and args.prefix == "shared" else 0))
+                             * nl - (nl - 1 if nl > 1 and args.plan_reuse == "on" else 0)) * K,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
@@ -555,6 +604,9 @@ def main(argv=None):
     ap.add_argument("--prefix", default="off", choices=["off", "shared"],
                     help="shared-prefix read: pages shared by a group's sequences read by "
                          "every sequence (off, the default) or once per group (shared)")
+    ap.add_argument("--plan-reuse", default="on", choices=["on", "off"],
+                    help="multi-layer workloads: layers after the first of a step reuse its "
+                         "work list (on, the default) or build their own (off)")
     ap.add_argument("--sinks", type=int, default=None, help="override S (protection sweep)")
     ap.add_argument("--recent", type=int, default=None, help="override R (protection sweep)")
     ap.add_argument("--prefill", action="store_true",

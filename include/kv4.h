@@ -157,6 +157,15 @@ typedef struct {
   int32_t num_seqs;
   int32_t max_seq_len;       /* host-side upper bound on seq_lens, sizes the workspace; a
                                 longer sequence may overflow it (KV4_DEVERR_WORKSPACE) */
+  int32_t plan_reuse;        /* 0: the attention call builds its work list in the workspace
+                                (the default). 1: it uses the work list the previous
+                                attention call on the same workspace left there, which must
+                                have been made with this same batch (lengths, page table,
+                                sink and ring indices, num_seqs, max_seq_len) and config --
+                                e.g. the layers of one decode step after the first. The
+                                kernels stay within their buffers if that does not hold
+                                (entries of an unknown sequence or length are skipped and
+                                flagged), but the results are then void. */
 } kv4_batch;
 
 /*

@@ -58,7 +58,7 @@ kv4_status make_view(const kv4_config *cfg, const kv4_int4_pool *pool, const kv4
   if (st != KV4_OK) return st;
   if (pool == nullptr || side == nullptr || batch == nullptr) return KV4_ERR_INVALID_ARG;
   if (batch->num_seqs < 0 || batch->max_pages <= 0 || batch->max_seq_len < 0 ||
-      pool->num_pages < 0)
+      pool->num_pages < 0 || batch->plan_reuse < 0 || batch->plan_reuse > 1)
     return KV4_ERR_INVALID_ARG;
   if (batch->num_seqs > 0 && (batch->page_table == nullptr || batch->seq_lens == nullptr))
     return KV4_ERR_INVALID_ARG;
@@ -275,13 +275,14 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   if (st != KV4_OK) return st;
   take_test_hook(&w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  cudaError_t e = batch->plan_reuse ? cudaSuccess : kv4::launch_plan(v, w, err_flag, s);
   if (e == cudaSuccess) e = kv4::launch_prefix(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
-                          static_cast<uint16_t *>(out), out_f32, lse, s);
+                          static_cast<uint16_t *>(out), out_f32, lse, w.counter,
+                          kv4::plan_signature_host(v, w), s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -310,9 +311,13 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   cudaError_t e = cudaStreamIsCapturing(s, &capturing);
   if (e != cudaSuccess) return KV4_ERR_CUDA;
   StepStreams *ss = nullptr;
-  e = step_streams(capturing == cudaStreamCaptureStatusNone, &ss);
-  if (e != cudaSuccess) return KV4_ERR_CUDA;
-  if (ss != nullptr) {  // fork: the work list on the second stream beside the append
+  if (!batch->plan_reuse) {  // with a reused work list there is nothing to run beside
+    e = step_streams(capturing == cudaStreamCaptureStatusNone, &ss);
+    if (e != cudaSuccess) return KV4_ERR_CUDA;
+  }
+  if (batch->plan_reuse) {
+    e = cudaSuccess;
+  } else if (ss != nullptr) {  // fork: the work list on the second stream beside the append
     e = cudaEventRecord(ss->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->side, ss->fork, 0);
     if (e == cudaSuccess) e = kv4::launch_plan(v, w, err_flag, ss->side);
@@ -331,7 +336,8 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
-                          static_cast<uint16_t *>(out), out_f32, lse, s);
+                          static_cast<uint16_t *>(out), out_f32, lse, w.counter,
+                          kv4::plan_signature_host(v, w), s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -346,8 +352,8 @@ kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offse
   if (misaligned16(partials) || misaligned16(out) || misaligned16(out_f32))
     return KV4_ERR_INVALID_ARG;
   cudaError_t e = kv4::launch_merge(partials, region_offsets, n_units, group,
-                                    static_cast<uint16_t *>(out), out_f32, lse,
-                                    reinterpret_cast<cudaStream_t>(stream));
+                                    static_cast<uint16_t *>(out), out_f32, lse, nullptr,
+                                    kv4::PlanSig{}, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -398,12 +404,13 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
   take_test_hook(&w);
   w.heads_per_warp = 1;  // one kv head per warp and entry
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = kv4::launch_plan(v, w, err_flag, s);
+  cudaError_t e = batch->plan_reuse ? cudaSuccess : kv4::launch_plan(v, w, err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_baseline_attention(fmt, v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
-                          static_cast<uint16_t *>(out), out_f32, lse, s);
+                          static_cast<uint16_t *>(out), out_f32, lse, w.counter,
+                          kv4::plan_signature_host(v, w), s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 

@@ -378,6 +378,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     // a workspace too small leaves every unit empty (all offsets 0): the merge then
     // reads no partial state and writes zero outputs with lse = -inf
     w.unit_offsets[B * H] = fits ? H * tot[0] : 0;
+    int32_t sig[8];
+    plan_signature(c, w, sig);
+    for (int i = 0; i < 8; ++i) w.counter[8 + i] = sig[i];
     *w.n_items = fits ? te_all - tot[5] : 0;  // the attention kernel's entries
     *w.counter = 0;
     *w.pn_items = fits ? tot[5] : 0;          // then the prefix kernel's
@@ -949,6 +952,11 @@ __device__ __forceinline__ int process_int4(WarpCtx &x, const CacheView &c, cons
   const int p0 = rg.first_page + chunk * w.chunk_pages;
   const int last = (rg.int4_hi - 1) / kPage;
   const int np = min(w.chunk_pages, last - p0 + 1);
+  if (np < 1 || chunk < 0) {  // only with a reused work list whose lengths have changed
+    if (lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    for (int hs = 0; hs < nh; ++hs) write_empty(record_of(w, H, G, b, h0 + hs, r), G, lane);
+    return kDone;
+  }
   // this lane's C-fragment columns 2tig, 2tig+1: head slot and query index
   const int hs_c = (2 * tig) / CPH;
   const int jc0 = (2 * tig) % CPH;
@@ -1181,36 +1189,50 @@ __device__ __forceinline__ int process_int4(WarpCtx &x, const CacheView &c, cons
       if (!(tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi)) s[0][0] = s[0][1] = -CUDART_INF_F;
       if (!(tok0 + t1 >= tok_lo && tok0 + t1 < tok_hi)) s[1][0] = s[1][1] = -CUDART_INF_F;
     }
-    // ---- online softmax; the rescale is skipped while no running max moves ----
-    float a[2];
-    bool moved = false;
+    // ---- online softmax. A page moves a running maximum only if one of its logits
+    // exceeds it; when none does (most pages after an entry's first few), the shuffle
+    // reduction and the rescale are skipped: the same result as the general path's with
+    // an unmoved maximum (alpha = 1). Running maxima are kept as max - lift.
+    const bool raise = fmaxf(s[0][0], s[1][0]) - lift > m[0] ||
+                       fmaxf(s[0][1], s[1][1]) - lift > m[1];
+    if (__any_sync(0xffffffffu, raise)) {
+      float a[2];
+      bool moved = false;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float t = fmaxf(s[0][e], s[1][e]);
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
-      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-      const float mn = fmaxf(m[e], t - lift);  // running maximum kept as max - lift
-      const bool mv = mn != m[e];
-      a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
-      moved |= mv;
-      m[e] = mn;
-      s[0][e] = fast_exp2(s[0][e] - mn);
-      s[1][e] = fast_exp2(s[1][e] - mn);
-      l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
-    }
-    if (__any_sync(0xffffffffu, moved)) {
-      const float2 a2 = make_float2(a[0], a[1]);
+      for (int e = 0; e < 2; ++e) {
+        float t = fmaxf(s[0][e], s[1][e]);
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+        const float mn = fmaxf(m[e], t - lift);
+        const bool mv = mn != m[e];
+        a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
+        moved |= mv;
+        m[e] = mn;
+        s[0][e] = fast_exp2(s[0][e] - mn);
+        s[1][e] = fast_exp2(s[1][e] - mn);
+        l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
+      }
+      if (__any_sync(0xffffffffu, moved)) {
+        const float2 a2 = make_float2(a[0], a[1]);
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        mt[g][0] *= a[0];
-        mt[g][1] *= a[1];
+        for (int g = 0; g < 4; ++g) {
+          mt[g][0] *= a[0];
+          mt[g][1] *= a[1];
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const float2 u = fmul2(make_float2(o[g][t][0], o[g][t][1]), a2);
-          const float2 v = fmul2(make_float2(o[g][t][2], o[g][t][3]), a2);
-          o[g][t][0] = u.x; o[g][t][1] = u.y; o[g][t][2] = v.x; o[g][t][3] = v.y;
+          for (int t = 0; t < 2; ++t) {
+            const float2 u = fmul2(make_float2(o[g][t][0], o[g][t][1]), a2);
+            const float2 v = fmul2(make_float2(o[g][t][2], o[g][t][3]), a2);
+            o[g][t][0] = u.x; o[g][t][1] = u.y; o[g][t][2] = v.x; o[g][t][3] = v.y;
+          }
         }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        s[0][e] = fast_exp2(s[0][e] - m[e]);
+        s[1][e] = fast_exp2(s[1][e] - m[e]);
+        l[e] = fmaf(l[e], 1.0f, s[0][e] + s[1][e]);
       }
     }
     // ---- P'_g = p * vscale_g as fp16 token pairs; sum p * vmin_g on the side ----
@@ -1357,12 +1379,6 @@ __device__ __forceinline__ bool process_prefix(WarpCtx &x, const CacheView &c, c
     }
   for (int mi = 0; mi < nmem; ++mi) hi_min = min(hi_min, c.seq_lens[b0 + mi] - R);
 
-  const int *pt = c.page_table + static_cast<size_t>(b0) * c.max_pages + p0;
-  int pid = 0, pid2 = 0;
-  if (lane < np) pid = pt[lane];
-  if (lane + 32 < np) pid2 = pt[lane + 32];
-  const bool bad = (lane < np && (pid < 0 || pid >= c.num_pages)) ||
-                   (lane + 32 < np && (pid2 < 0 || pid2 >= c.num_pages));
   auto write_empty_all = [&]() {
     for (int mi = 0; mi < nmem; ++mi) {
       const int L = c.seq_lens[b0 + mi];
@@ -1370,6 +1386,17 @@ __device__ __forceinline__ bool process_prefix(WarpCtx &x, const CacheView &c, c
       write_empty(record_of(w, H, G, b0 + mi, h, r), G, lane);
     }
   };
+  if (np <= 0 || p0 + np > c.max_pages) {  // a reused work list that is not this batch's
+    if (lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    write_empty_all();
+    return false;
+  }
+  const int *pt = c.page_table + static_cast<size_t>(b0) * c.max_pages + p0;
+  int pid = 0, pid2 = 0;
+  if (lane < np) pid = pt[lane];
+  if (lane + 32 < np) pid2 = pt[lane + 32];
+  const bool bad = (lane < np && (pid < 0 || pid >= c.num_pages)) ||
+                   (lane + 32 < np && (pid2 < 0 || pid2 >= c.num_pages));
   if (__any_sync(0xffffffffu, bad)) {
     if (lane == 0) set_err(err, KV4_DEVERR_PAGE_ID);
     write_empty_all();
@@ -1691,6 +1718,10 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
     fence_barrier_init();
   }
   __syncwarp();
+  if (!plan_matches(c, w)) {  // a reused work list of another batch: read none of it
+    if (x.lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    return;
+  }
   const int base = *w.n_items;  // the prefix entries follow the attention kernel's
   const int n_items = *w.pn_items;
   for (;;) {
@@ -1721,10 +1752,35 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
 // 13.4 against 17.4 us on the 1024-sequence batch, 7.0 against 8.4 us on 128 x 16384).
 __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
                                                     const int32_t *__restrict__ offs, int n_units,
-                                                    int G, Outputs o) {
+                                                    int G, Outputs o, int32_t *reset,
+                                                    PlanSig want) {
   constexpr int kBatch = 4;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  if (reset != nullptr) {  // the work list must be this call's (see plan_signature)
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ok &= reset[8 + i] == want.v[i];
+    if (!ok) {
+      if (warp < n_units * G) {  // write zero outputs, lse = -inf; read no partial state
+        const size_t row = static_cast<size_t>(warp);
+        *reinterpret_cast<uint2 *>(o.out + row * kHeadDim + 4 * lane) = make_uint2(0u, 0u);
+        if (o.out_f32)
+          *reinterpret_cast<float4 *>(o.out_f32 + row * kHeadDim + 4 * lane) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        if (o.lse && lane == 0) o.lse[row] = -CUDART_INF_F;
+      }
+      return;
+    }
+  }
+  if (reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    // the call's attention kernels are done: zero the work counters of the work list
+    // (counter, prefix counter, lift list count and counter) for a call that reuses it
+    reset[0] = 0;
+    reset[2] = 0;
+    reset[4] = 0;
+    reset[5] = 0;
+  }
   if (warp >= n_units * G) return;
   const int u = warp / G, j = warp - u * G;
   const int r0 = offs[u], n = offs[u + 1] - r0;
@@ -1811,6 +1867,10 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
   __syncwarp();
 
   const int H = c.num_kv_heads, G = c.gqa;
+  if (!plan_matches(c, w)) {  // a reused work list of another batch: read none of it
+    if (x.lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    return;
+  }
   const int n_items = *w.n_items;
   for (;;) {
     int item = 0;
@@ -1821,6 +1881,10 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
     const int4 en = w.entries[item];
     const int b = en.x, r = en.y, h0 = en.z, nh = en.w;
     const int L = c.seq_lens[b];
+    if (L < 0 || L > c.max_pages * kPage) {  // (a reused list whose lengths have changed)
+      if (x.lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
+      continue;
+    }
     const int pe = w.prefix_end ? w.prefix_end[b] : 0;
     const Regions rg = regions_of(L, c.num_sinks, c.num_recent, w.chunk_pages, pe);
     int res;
@@ -1845,6 +1909,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) lift_kernel(Cache
                                                                            const uint16_t *__restrict__ q,
                                                                            int32_t *err) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (!plan_matches(c, w)) return;  // flagged by the attention kernel
   const int n_items = *w.lift_count;
   if (n_items == 0) return;
   WarpCtx x;
@@ -1947,6 +2012,19 @@ cudaError_t launch_prefix(const CacheView &c, const Workspace &w, const uint16_t
 
 int heads_per_warp_for(int gqa) { return gqa <= 4 ? 2 : 1; }
 
+PlanSig plan_signature_host(const CacheView &c, const Workspace &w) {
+  PlanSig p;
+  p.v[0] = 0x4b563450;
+  p.v[1] = c.num_seqs;
+  p.v[2] = c.num_kv_heads;
+  p.v[3] = c.gqa | (w.heads_per_warp << 8) | (w.prefix_end != nullptr ? 1 << 16 : 0);
+  p.v[4] = w.chunk_pages;
+  p.v[5] = c.num_sinks | (c.num_recent << 16);
+  p.v[6] = w.cap_entries;
+  p.v[7] = w.cap_pairs;
+  return p;
+}
+
 // The persistent grid of the attention kernel: an empty list costs a launch whose CTAs
 // end at once (about 3 us), a long one (small values everywhere) runs at full width.
 template <int HPW>
@@ -1985,12 +2063,14 @@ cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint1
 }
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
-                         int32_t group, uint16_t *out, float *out_f32, float *lse, cudaStream_t s) {
+                         int32_t group, uint16_t *out, float *out_f32, float *lse,
+                         const int32_t *reset, const PlanSig &want, cudaStream_t s) {
   const long long warps = static_cast<long long>(n_units) * group;
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps * 32 + 255) / 256;
-  merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(partials, unit_offsets, n_units, group,
-                                                             Outputs{out, out_f32, lse});
+  merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      partials, unit_offsets, n_units, group, Outputs{out, out_f32, lse},
+      const_cast<int32_t *>(reset), want);
   return cudaGetLastError();
 }
 

@@ -223,6 +223,32 @@ __device__ inline void write_empty(float *rec, int G, int lane) {
   }
 }
 
+// Signature of a work list, written by the plan kernel into the workspace's header (ints
+// 8..15) and checked by every kernel that reads the list: a call that reuses the list
+// (kv4_batch.plan_reuse) with another batch shape or workspace layout is refused on the
+// device (KV4_DEVERR_WORKSPACE) before any entry, offset or partial record is read.
+constexpr int32_t kPlanMagic = 0x4b563450;
+__device__ __forceinline__ void plan_signature(const CacheView &c, const Workspace &w,
+                                               int32_t (&sig)[8]) {
+  sig[0] = kPlanMagic;
+  sig[1] = c.num_seqs;
+  sig[2] = c.num_kv_heads;
+  sig[3] = c.gqa | (w.heads_per_warp << 8) | (w.prefix_end != nullptr ? 1 << 16 : 0);
+  sig[4] = w.chunk_pages;
+  sig[5] = c.num_sinks | (c.num_recent << 16);
+  sig[6] = w.cap_entries;
+  sig[7] = w.cap_pairs;
+}
+__device__ __forceinline__ bool plan_matches(const CacheView &c, const Workspace &w) {
+  int32_t want[8];
+  plan_signature(c, w, want);
+  const int32_t *have = w.counter + 8;
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ok &= have[i] == want[i];
+  return ok;
+}
+
 __device__ __forceinline__ float *record_of(const Workspace &w, int H, int G, int b, int h, int r) {
   return w.partials + static_cast<size_t>(w.unit_offsets[b * H + h] + r) * G * kRecordFloats;
 }

@@ -108,6 +108,11 @@ __device__ __forceinline__ void process_baseline(WarpCtx &x, const CacheView &c,
   const int np = min(w.chunk_pages, last - p0 + 1);
   const int nv = 2 * np;  // copies: K part, then V part, of every page
   float *rec = record_of(w, H, G, b, h, r);
+  if (np < 1) {  // only with a reused work list whose lengths have changed
+    if (lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    write_empty(rec, G, lane);
+    return;
+  }
 
   const int *pt = c.page_table + static_cast<size_t>(b) * c.max_pages + p0;
   int pid = 0, pid2 = 0;
@@ -403,6 +408,10 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) baseline_attn_ker
     fence_barrier_init();
   }
   __syncwarp();
+  if (!plan_matches(c, w)) {  // a reused work list of another batch: read none of it
+    if (x.lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
+    return;
+  }
   const int n_items = *w.n_items;
   for (;;) {
     int item = 0;
@@ -412,7 +421,12 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) baseline_attn_ker
     x.fault = withheld_item<HOOK>(w, item);
     const int4 en = w.entries[item];
     const int b = en.x, r = en.y, h = en.z;
-    const Regions rg = regions_of(c.seq_lens[b], 0, 0, w.chunk_pages);
+    const int L = c.seq_lens[b];
+    if (L < 0 || L > c.max_pages * kPage) {  // (a reused list whose lengths have changed)
+      if (x.lane == 0) set_err(err, KV4_DEVERR_SEQ_LEN);
+      continue;
+    }
+    const Regions rg = regions_of(L, 0, 0, w.chunk_pages);
     process_baseline<F>(x, c, w, q, b, h, r, rg, err);
     if (x.dead) break;
   }

@@ -117,9 +117,20 @@ cudaError_t launch_prefix(const CacheView &c, const Workspace &w, const uint16_t
                           int32_t *err_flag, cudaStream_t s);
 
 
+// The signature a work list of (c, w) carries (plan_signature in the kernels; the host
+// copy is what the merge compares with).
+struct PlanSig {
+  int32_t v[8];
+};
+PlanSig plan_signature_host(const CacheView &c, const Workspace &w);
+
+// reset: the workspace's counter block (nullptr for a bare merge); the merge, the last
+// kernel of an attention call, checks there that the work list is the call's (want: its
+// signature; else it writes zero outputs) and zeroes the work counters, so that a
+// following call can reuse the work list without the plan kernel.
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
                          int32_t group, uint16_t *out, float *out_f32, float *lse,
-                         cudaStream_t s);
+                         const int32_t *reset, const PlanSig &want, cudaStream_t s);
 
 // Comparison baselines (kv4_baseline.cu): fmt is a kv4_baseline_format. The view's
 // k_codes / v_codes hold the BF16 or INT8 pages, k_params / v_params the KV8 scales.

@@ -65,7 +65,7 @@ class Batch(ctypes.Structure):
     _fields_ = [("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
                 ("seq_lens", ctypes.c_void_p), ("sink_idx", ctypes.c_void_p),
                 ("ring_idx", ctypes.c_void_p), ("num_seqs", ctypes.c_int32),
-                ("max_seq_len", ctypes.c_int32)]
+                ("max_seq_len", ctypes.c_int32), ("plan_reuse", ctypes.c_int32)]
 
 
 class PagedPool(ctypes.Structure):
@@ -226,12 +226,13 @@ class BatchTensors:
     sink_idx: torch.Tensor    # int32 [B]
     ring_idx: torch.Tensor | None
     max_seq_len: int
+    plan_reuse: bool = False  # use the work list the last call on the workspace left
 
     def struct(self) -> Batch:
         return Batch(self.page_table.data_ptr(), self.page_table.shape[1],
                      self.seq_lens.data_ptr(), self.sink_idx.data_ptr(),
                      0 if self.ring_idx is None else self.ring_idx.data_ptr(),
-                     self.seq_lens.shape[0], int(self.max_seq_len))
+                     self.seq_lens.shape[0], int(self.max_seq_len), int(self.plan_reuse))
 
 
 def workspace_size(cfg: Config, num_seqs: int, max_seq_len: int) -> int:

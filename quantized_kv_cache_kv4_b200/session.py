@@ -55,6 +55,9 @@ class DecodeSession:
         self.step_v = torch.empty_like(self.step_k)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_rows = max_rows_per_call
+        # attention calls reuse the work list the previous call on the shared workspace
+        # left (layers after the first of one decode step: same lengths and paging)
+        self.plan_reuse = False
         ws = self._workspace_size(B, self.max_len)
         if workspace is not None and workspace.numel() >= ws:
             self.workspace = workspace  # shared with other layers (calls run in stream order)
@@ -84,7 +87,7 @@ class DecodeSession:
 
     def batch(self, lens: torch.Tensor) -> kv4.BatchTensors:
         return kv4.BatchTensors(self.page_table, lens, self.sink_idx, self.ring_idx,
-                                self.max_len)
+                                self.max_len, self.plan_reuse)
 
     def _append_rows(self, rows_k, rows_v, counts, lens_after, page_table=None):
         """One append call: rows of all sequences, CSR by `counts`."""

@@ -26,7 +26,7 @@ int main(void) {
   SIZE(kv4_batch);
   OFF(kv4_batch, page_table); OFF(kv4_batch, max_pages); OFF(kv4_batch, seq_lens);
   OFF(kv4_batch, sink_idx); OFF(kv4_batch, ring_idx); OFF(kv4_batch, num_seqs);
-  OFF(kv4_batch, max_seq_len);
+  OFF(kv4_batch, max_seq_len); OFF(kv4_batch, plan_reuse);
   SIZE(kv4_paged_pool);
   OFF(kv4_paged_pool, k); OFF(kv4_paged_pool, v); OFF(kv4_paged_pool, k_scales);
   OFF(kv4_paged_pool, v_scales); OFF(kv4_paged_pool, num_pages);

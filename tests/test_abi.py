@@ -253,7 +253,7 @@ def test_binding_structs_match_the_c_layout(kv4, tmp_path):
             struct, field = name.split(".")
             assert getattr(py[struct], field).offset == val, name
         checked += 1
-    assert checked == 5 + 10 + 5 + 10 + 7 + 5
+    assert checked == 5 + 10 + 5 + 10 + 8 + 5
 
 
 def test_binding_refuses_host_or_strided_tensors(kv4):

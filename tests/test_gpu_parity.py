@@ -304,6 +304,60 @@ def test_lift_overflow_is_redone_without_the_lift():
     sess.check_err()
 
 
+def test_plan_reuse_across_layers():
+    """Two layers of one decode step share a workspace: layer 1's calls reuse the work
+    list layer 0's call left (batch.plan_reuse). Its outputs equal those of building its
+    own work list bit for bit, through kv4_decode_attention and kv4_decode_step alike,
+    over three steps, and match the oracle."""
+    kv4, session, W = _mods()
+    wl = W.custom_workload([700, 2000, 40, 1500, 333], num_sinks=16, num_recent=128, seed=8,
+                           outlier_channels=2, outlier_scale=8.0)
+    l0 = session.DecodeSession(wl, steps=3, layer=0)
+    l1 = session.DecodeSession(wl, steps=3, layer=1, keep_streams=range(5),
+                               workspace=l0.workspace)
+    own = torch.empty_like(l1.out)
+    for s in range(3):
+        l0.fused_step(s)                      # builds the work list
+        l1.plan_reuse = True
+        l1.fused_step(s)                      # append + attention on layer 0's work list
+        torch.cuda.synchronize()
+        reused = l1.out.clone()
+        l1.plan_reuse = False
+        l1.attention_step(s, out=own)         # its own work list
+        torch.cuda.synchronize()
+        assert torch.equal(reused, own), s
+        l0.attention_step(s)                  # layer 0 again, then layer 1's separate call
+        l1.plan_reuse = True
+        l1.attention_step(s)
+        torch.cuda.synchronize()
+        assert torch.equal(l1.out, own), s
+        l1.plan_reuse = False
+        check_attention(l1, range(5), step=s, got=None)
+    l0.check_err()
+    l1.check_err()
+
+
+def test_plan_reuse_with_another_batch_is_flagged_without_faulting():
+    """A reused work list built for 5 sequences, used by a batch of 2: the entries of the
+    missing sequences are skipped and flagged (KV4_DEVERR_WORKSPACE); the call returns and
+    the next call, which builds its own work list, is exact."""
+    kv4, session, W = _mods()
+    wl = W.custom_workload([700, 2000, 40, 1500, 333], num_sinks=16, num_recent=128, seed=9)
+    sess = make_session(wl, keep=range(5))
+    sess.attention_step(0)
+    small = kv4.BatchTensors(sess.page_table[:2].contiguous(), sess.step_lens[0][:2].contiguous(),
+                             sess.sink_idx[:2].contiguous(), sess.ring_idx[:2].contiguous(),
+                             sess.max_len, plan_reuse=True)
+    out = torch.empty((2, wl.num_q_heads, 128), dtype=torch.bfloat16, device="cuda")
+    kv4.decode_attention(sess.cache, small, sess.q[0][:2].contiguous(), out, sess.workspace,
+                         err=sess.err)
+    torch.cuda.synchronize()
+    assert int(sess.err.item()) & 16, kv4.decode_err(int(sess.err.item()))
+    sess.err.zero_()
+    check_attention(sess, range(5))
+    sess.check_err()
+
+
 def test_bounded_wait_gives_up_without_a_fault():
     """The error path of the bounded waits, run on a GPU without any fault: the testing
     hook withholds the first copy of work item 0 (nothing is issued for it, so nothing is
