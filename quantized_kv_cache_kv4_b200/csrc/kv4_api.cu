@@ -274,6 +274,8 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
   take_test_hook(&w);
+  w.check_plan = batch->plan_reuse;
+  const kv4::PlanSig sig = kv4::plan_signature_host(v, w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = batch->plan_reuse ? cudaSuccess : kv4::launch_plan(v, w, err_flag, s);
   if (e == cudaSuccess) e = kv4::launch_prefix(v, w, static_cast<const uint16_t *>(q), err_flag, s);
@@ -282,7 +284,7 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
                           static_cast<uint16_t *>(out), out_f32, lse, w.counter,
-                          kv4::plan_signature_host(v, w), s);
+                          w.check_plan ? &sig : nullptr, s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -303,6 +305,8 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   st = carve_workspace(cfg, v, batch, workspace, ws_bytes, &w);
   if (st != KV4_OK) return st;
   take_test_hook(&w);
+  w.check_plan = batch->plan_reuse;
+  const kv4::PlanSig sig = kv4::plan_signature_host(v, w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // The second stream and its events are not created while the caller's stream is being
   // captured into a graph; a first call made there builds the work list on the caller's
@@ -337,7 +341,7 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
                           static_cast<uint16_t *>(out), out_f32, lse, w.counter,
-                          kv4::plan_signature_host(v, w), s);
+                          w.check_plan ? &sig : nullptr, s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -353,7 +357,7 @@ kv4_status kv4_regional_merge(const float *partials, const int32_t *region_offse
     return KV4_ERR_INVALID_ARG;
   cudaError_t e = kv4::launch_merge(partials, region_offsets, n_units, group,
                                     static_cast<uint16_t *>(out), out_f32, lse, nullptr,
-                                    kv4::PlanSig{}, reinterpret_cast<cudaStream_t>(stream));
+                                    nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 
@@ -403,6 +407,8 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
   if (st != KV4_OK) return st;
   take_test_hook(&w);
   w.heads_per_warp = 1;  // one kv head per warp and entry
+  w.check_plan = batch->plan_reuse;
+  const kv4::PlanSig sig = kv4::plan_signature_host(v, w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = batch->plan_reuse ? cudaSuccess : kv4::launch_plan(v, w, err_flag, s);
   if (e == cudaSuccess)
@@ -410,7 +416,7 @@ kv4_status kv4_baseline_decode_attention(kv4_baseline_format fmt, const kv4_conf
   if (e == cudaSuccess)
     e = kv4::launch_merge(w.partials, w.unit_offsets, batch->num_seqs * v.num_kv_heads, v.gqa,
                           static_cast<uint16_t *>(out), out_f32, lse, w.counter,
-                          kv4::plan_signature_host(v, w), s);
+                          w.check_plan ? &sig : nullptr, s);
   return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA;
 }
 

@@ -1189,50 +1189,36 @@ __device__ __forceinline__ int process_int4(WarpCtx &x, const CacheView &c, cons
       if (!(tok0 + t0 >= tok_lo && tok0 + t0 < tok_hi)) s[0][0] = s[0][1] = -CUDART_INF_F;
       if (!(tok0 + t1 >= tok_lo && tok0 + t1 < tok_hi)) s[1][0] = s[1][1] = -CUDART_INF_F;
     }
-    // ---- online softmax. A page moves a running maximum only if one of its logits
-    // exceeds it; when none does (most pages after an entry's first few), the shuffle
-    // reduction and the rescale are skipped: the same result as the general path's with
-    // an unmoved maximum (alpha = 1). Running maxima are kept as max - lift.
-    const bool raise = fmaxf(s[0][0], s[1][0]) - lift > m[0] ||
-                       fmaxf(s[0][1], s[1][1]) - lift > m[1];
-    if (__any_sync(0xffffffffu, raise)) {
-      float a[2];
-      bool moved = false;
+    // ---- online softmax; the rescale is skipped while no running max moves ----
+    float a[2];
+    bool moved = false;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float t = fmaxf(s[0][e], s[1][e]);
-        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
-        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
-        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
-        const float mn = fmaxf(m[e], t - lift);
-        const bool mv = mn != m[e];
-        a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
-        moved |= mv;
-        m[e] = mn;
-        s[0][e] = fast_exp2(s[0][e] - mn);
-        s[1][e] = fast_exp2(s[1][e] - mn);
-        l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
-      }
-      if (__any_sync(0xffffffffu, moved)) {
-        const float2 a2 = make_float2(a[0], a[1]);
+    for (int e = 0; e < 2; ++e) {
+      float t = fmaxf(s[0][e], s[1][e]);
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+      t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+      const float mn = fmaxf(m[e], t - lift);  // running maximum kept as max - lift
+      const bool mv = mn != m[e];
+      a[e] = mv ? fast_exp2(m[e] - mn) : 1.0f;
+      moved |= mv;
+      m[e] = mn;
+      s[0][e] = fast_exp2(s[0][e] - mn);
+      s[1][e] = fast_exp2(s[1][e] - mn);
+      l[e] = fmaf(l[e], a[e], s[0][e] + s[1][e]);
+    }
+    if (__any_sync(0xffffffffu, moved)) {
+      const float2 a2 = make_float2(a[0], a[1]);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          mt[g][0] *= a[0];
-          mt[g][1] *= a[1];
+      for (int g = 0; g < 4; ++g) {
+        mt[g][0] *= a[0];
+        mt[g][1] *= a[1];
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const float2 u = fmul2(make_float2(o[g][t][0], o[g][t][1]), a2);
-            const float2 v = fmul2(make_float2(o[g][t][2], o[g][t][3]), a2);
-            o[g][t][0] = u.x; o[g][t][1] = u.y; o[g][t][2] = v.x; o[g][t][3] = v.y;
-          }
+        for (int t = 0; t < 2; ++t) {
+          const float2 u = fmul2(make_float2(o[g][t][0], o[g][t][1]), a2);
+          const float2 v = fmul2(make_float2(o[g][t][2], o[g][t][3]), a2);
+          o[g][t][0] = u.x; o[g][t][1] = u.y; o[g][t][2] = v.x; o[g][t][3] = v.y;
         }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        s[0][e] = fast_exp2(s[0][e] - m[e]);
-        s[1][e] = fast_exp2(s[1][e] - m[e]);
-        l[e] = fmaf(l[e], 1.0f, s[0][e] + s[1][e]);
       }
     }
     // ---- P'_g = p * vscale_g as fp16 token pairs; sum p * vmin_g on the side ----
@@ -1718,7 +1704,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
     fence_barrier_init();
   }
   __syncwarp();
-  if (!plan_matches(c, w)) {  // a reused work list of another batch: read none of it
+  if (w.check_plan && !plan_matches(c, w)) {  // a reused list of another batch: read none
     if (x.lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
     return;
   }
@@ -1753,11 +1739,11 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
 __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
                                                     const int32_t *__restrict__ offs, int n_units,
                                                     int G, Outputs o, int32_t *reset,
-                                                    PlanSig want) {
+                                                    PlanSig want, int check) {
   constexpr int kBatch = 4;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (reset != nullptr) {  // the work list must be this call's (see plan_signature)
+  if (check) {  // a reused work list must be this call's (see plan_signature)
     bool ok = true;
 #pragma unroll
     for (int i = 0; i < 8; ++i) ok &= reset[8 + i] == want.v[i];
@@ -1867,7 +1853,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) attn_kernel(Cache
   __syncwarp();
 
   const int H = c.num_kv_heads, G = c.gqa;
-  if (!plan_matches(c, w)) {  // a reused work list of another batch: read none of it
+  if (w.check_plan && !plan_matches(c, w)) {  // a reused list of another batch: read none
     if (x.lane == 0) set_err(err, KV4_DEVERR_WORKSPACE);
     return;
   }
@@ -1909,7 +1895,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) lift_kernel(Cache
                                                                            const uint16_t *__restrict__ q,
                                                                            int32_t *err) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  if (!plan_matches(c, w)) return;  // flagged by the attention kernel
+  if (w.check_plan && !plan_matches(c, w)) return;  // flagged by the attention kernel
   const int n_items = *w.lift_count;
   if (n_items == 0) return;
   WarpCtx x;
@@ -2064,13 +2050,13 @@ cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint1
 
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
                          int32_t group, uint16_t *out, float *out_f32, float *lse,
-                         const int32_t *reset, const PlanSig &want, cudaStream_t s) {
+                         const int32_t *reset, const PlanSig *want, cudaStream_t s) {
   const long long warps = static_cast<long long>(n_units) * group;
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps * 32 + 255) / 256;
   merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
       partials, unit_offsets, n_units, group, Outputs{out, out_f32, lse},
-      const_cast<int32_t *>(reset), want);
+      const_cast<int32_t *>(reset), want ? *want : PlanSig{}, want && reset ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -2116,6 +2102,7 @@ size_t workspace_bytes(int32_t num_seqs, int32_t max_seq_len, int32_t num_kv_hea
     carve->heads_per_warp = heads_per_warp_for(gqa);
     carve->wait_limit = kWaitLimit;
     carve->fault_item = -1;
+    carve->check_plan = 0;
   }
   return off;
 }

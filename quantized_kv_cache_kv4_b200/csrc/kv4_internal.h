@@ -82,6 +82,7 @@ struct Workspace {
   int32_t *lift_count;     // [1] entries on the lift list (small V scales)
   int32_t *lift_counter;   // [1] dynamic work counter of the lift kernel
   int32_t *lift_items;     // [cap_entries] work items on the lift list
+  int32_t check_plan;      // the call reuses a work list: kernels check its signature first
   uint32_t wait_limit;     // attempts of one bounded wait for a copy (kWaitLimit)
   int32_t fault_item;      // testing hook: work item whose first copy is withheld, -1 none
 };
@@ -125,12 +126,13 @@ struct PlanSig {
 PlanSig plan_signature_host(const CacheView &c, const Workspace &w);
 
 // reset: the workspace's counter block (nullptr for a bare merge); the merge, the last
-// kernel of an attention call, checks there that the work list is the call's (want: its
-// signature; else it writes zero outputs) and zeroes the work counters, so that a
-// following call can reuse the work list without the plan kernel.
+// kernel of an attention call, zeroes its work counters there, so that a following call
+// can reuse the work list without the plan kernel. want: the call's signature when it
+// reuses a work list (nullptr otherwise); the merge then checks the list's signature
+// first and writes zero outputs if it is another batch's.
 cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int32_t n_units,
                          int32_t group, uint16_t *out, float *out_f32, float *lse,
-                         const int32_t *reset, const PlanSig &want, cudaStream_t s);
+                         const int32_t *reset, const PlanSig *want, cudaStream_t s);
 
 // Comparison baselines (kv4_baseline.cu): fmt is a kv4_baseline_format. The view's
 // k_codes / v_codes hold the BF16 or INT8 pages, k_params / v_params the KV8 scales.
