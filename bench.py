@@ -278,7 +278,10 @@ def output_check(sess, step, nseq=8, seed=5):
     refs = {}
     for b in seqs:
         L = int(sess.L0[b]) + step
-        k, v = seq_kv(wl, b, L, sess.layer, sess.device)
+        # drawn as the session drew it (the whole stream, then the positions in use): a
+        # stream's values can depend on its drawn length (the Student-t draws)
+        k, v = seq_kv(wl, b, int(sess.L0[b]) + sess.steps, sess.layer, sess.device)
+        k, v = k[:L], v[:L]
         q = sess.q[step, b].float().cpu().numpy()
         refs[b] = O.decode_reference(q, k.float().cpu().numpy(), v.float().cpu().numpy(),
                                      wl.num_sinks, wl.num_recent, sess.demotion)[0]
