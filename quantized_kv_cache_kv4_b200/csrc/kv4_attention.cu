@@ -38,6 +38,8 @@
 //                the kernel behind kv4_regional_merge.
 #include <math_constants.h>
 
+#include <climits>
+
 #include "kv4_attn_common.cuh"
 
 namespace kv4 {
@@ -54,10 +56,10 @@ constexpr int kScanN = 6;            // values scanned together per sequence
 constexpr int kPrefixCols = 16;      // query columns of one prefix entry (two MMA N tiles)
 constexpr int kMaxPrefixPages = 256;  // leading INT4 pages compared for sharing
 
-// Exclusive block-wide scan of kScanN values at once (warp shuffles + one warp over the
-// 32 warp totals per value); totals returned in tot.
+// Exclusive block-wide scan of kScanN values at once (warp shuffles + one warp per value
+// over the warp totals); totals returned in tot. Blocks of 32 to 1024 threads.
 __device__ void block_scan_n(int (&v)[kScanN], int (&tot)[kScanN], int (*warp_sums)[32]) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int x[kScanN];
 #pragma unroll
   for (int i = 0; i < kScanN; ++i) {
@@ -70,14 +72,14 @@ __device__ void block_scan_n(int (&v)[kScanN], int (&tot)[kScanN], int (*warp_su
     if (lane == 31) warp_sums[i][wid] = x[i];
   }
   __syncthreads();
-  if (wid < kScanN) {
-    int t = warp_sums[wid][lane];
+  for (int i = wid; i < kScanN; i += nw) {
+    int t = lane < nw ? warp_sums[i][lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, t, off);
       if (lane >= off) t += y;
     }
-    warp_sums[wid][lane] = t;
+    warp_sums[i][lane] = t;
   }
   __syncthreads();
 #pragma unroll
@@ -115,9 +117,9 @@ __device__ int key_rank(int key, int (*cnt)[33], int *chunk_tot) {
   return rank;
 }
 
-// Inclusive block-wide max-scan of v (1024 threads); warp_max: shared scratch [32].
+// Inclusive block-wide max-scan of v (32 to 1024 threads); warp_max: shared scratch [32].
 __device__ int block_max_scan(int v, int *warp_max) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, v, off);
@@ -126,7 +128,7 @@ __device__ int block_max_scan(int v, int *warp_max) {
   if (lane == 31) warp_max[wid] = v;
   __syncthreads();
   if (wid == 0) {
-    int t = warp_max[lane];
+    int t = lane < nw ? warp_max[lane] : INT_MIN;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, t, off);
@@ -271,15 +273,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     return prefix ? prefix_runs(c, w, base, run_min, run_len, warp_max) : PrefixRun{};
   };
 
-  // pass 1: totals over every sequence. A batch of at most kPlanThreads sequences is
+  // pass 1: totals over every sequence. A batch of at most one block of sequences is
   // one block-wide pass, whose exclusive offsets and key ranks are kept for pass 2.
-  const bool single = B <= kPlanThreads;
+  // Blocks have min(1024, num_seqs rounded up to a warp) threads.
+  const int T = blockDim.x;
+  const bool single = B <= T;
   int tot[kScanN] = {0, 0, 0, 0, 0, 0};
   SeqPlan keep{};
   int keep_off[kScanN] = {0, 0, 0, 0, 0, 0};
   int keep_rank = 0;
   if (threadIdx.x < 32) key_tot[threadIdx.x] = 0;
-  for (int base = 0; base < B; base += kPlanThreads) {
+  for (int base = 0; base < B; base += T) {
     SeqPlan sp = plan_of(base + threadIdx.x, runs_of(base));
     int off[kScanN], t[kScanN];
 #pragma unroll
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(CacheView c, Workspa
     int run[kScanN];
 #pragma unroll
     for (int i = 0; i < kScanN; ++i) run[i] = class_base[i];
-    for (int base = 0; base < my_hi; base += kPlanThreads) {
+    for (int base = 0; base < my_hi; base += T) {
       const int b = base + threadIdx.x;
       const PrefixRun pr = runs_of(base);
       SeqPlan sp = fits ? plan_of(b, pr) : SeqPlan{};
@@ -1950,7 +1954,9 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) lift_kernel(Cache
 cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag,
                         cudaStream_t s) {
   const int ctas = max(1, min(kPlanMaxCtas, (c.num_seqs + kPlanSeqsPerCta - 1) / kPlanSeqsPerCta));
-  plan_kernel<<<ctas, kPlanThreads, 0, s>>>(c, w, err_flag);
+  // small batches: fewer threads (the scans and barriers span only the warps in use)
+  const int threads = min(kPlanThreads, max(32, (c.num_seqs + 31) / 32 * 32));
+  plan_kernel<<<ctas, threads, 0, s>>>(c, w, err_flag);
   return cudaGetLastError();
 }
 
