@@ -244,13 +244,10 @@ kv4_status kv4_decode_attention(const kv4_config *cfg, const kv4_int4_pool *pool
  * total_new = num_seqs; k_new, v_new bf16 [num_seqs][Hkv][128]) followed by
  * kv4_decode_attention, with the same arguments, checks, results and error flags as
  * the two calls made in that order on `stream` (batch->seq_lens are the lengths after
- * the append). The attention's work list depends only on the lengths, so it is built on
- * a second stream, forked from and joined back to `stream` with events, while the
- * append runs; the call stays asynchronous and can be captured in a CUDA graph. The
- * second stream and the two events are created on first use, one set per host thread
- * and device, and live until the process ends; a thread's first call made while the
- * stream is being captured creates nothing and builds the work list on `stream`
- * itself (same results, without the overlap).
+ * the append). The attention's work list depends only on the lengths (and page tables),
+ * which the append does not write, so one kernel launch builds it and appends the tokens;
+ * with batch->plan_reuse set it only appends. Everything runs on `stream`; the call is
+ * asynchronous and allocates nothing.
  */
 kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
                            const kv4_int8_side *side, const kv4_batch *batch,

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkv4.so")
 SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_attention.cu", "kv4_baseline.cu", "kv4_noalloc.cu"]
-HEADERS = ["kv4_device.cuh", "kv4_internal.h", "kv4_attn_common.cuh"]
+HEADERS = ["kv4_device.cuh", "kv4_internal.h", "kv4_attn_common.cuh", "kv4_plan.cuh"]
 
 
 def nvcc() -> str:

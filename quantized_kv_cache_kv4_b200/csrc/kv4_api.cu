@@ -191,36 +191,6 @@ kv4_status carve_workspace(const kv4_config *cfg, const kv4::CacheView &v,
   return ws_bytes < need ? KV4_ERR_WORKSPACE_TOO_SMALL : KV4_OK;
 }
 
-// The second stream and fork/join events of kv4_decode_step: one set per host thread
-// and device, created on first use and kept for the life of the process.
-struct StepStreams {
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-
-// *out = this thread's set for the current device, created unless `create` is false
-// (then nullptr when it does not exist yet).
-cudaError_t step_streams(bool create, StepStreams **out) {
-  constexpr int kMaxDevices = 64;
-  thread_local StepStreams per_device[kMaxDevices];
-  *out = nullptr;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  StepStreams &ss = per_device[dev];
-  if (ss.join == nullptr) {
-    if (!create) return cudaSuccess;
-    if (ss.side == nullptr) e = cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking);
-    if (e == cudaSuccess && ss.fork == nullptr)
-      e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) return e;
-  }
-  *out = &ss;
-  return cudaSuccess;
-}
-
 kv4_status check_attention_args(const kv4_batch *batch, const void *q, const void *out,
                                 const float *out_f32, const void *workspace) {
   if (q == nullptr || out == nullptr || workspace == nullptr) return KV4_ERR_INVALID_ARG;
@@ -308,33 +278,12 @@ kv4_status kv4_decode_step(const kv4_config *cfg, const kv4_int4_pool *pool,
   w.check_plan = batch->plan_reuse;
   const kv4::PlanSig sig = kv4::plan_signature_host(v, w);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The second stream and its events are not created while the caller's stream is being
-  // captured into a graph; a first call made there builds the work list on the caller's
-  // stream (same results, no overlap).
-  cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
-  cudaError_t e = cudaStreamIsCapturing(s, &capturing);
-  if (e != cudaSuccess) return KV4_ERR_CUDA;
-  StepStreams *ss = nullptr;
-  if (!batch->plan_reuse) {  // with a reused work list there is nothing to run beside
-    e = step_streams(capturing == cudaStreamCaptureStatusNone, &ss);
-    if (e != cudaSuccess) return KV4_ERR_CUDA;
-  }
-  if (batch->plan_reuse) {
-    e = cudaSuccess;
-  } else if (ss != nullptr) {  // fork: the work list on the second stream beside the append
-    e = cudaEventRecord(ss->fork, s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->side, ss->fork, 0);
-    if (e == cudaSuccess) e = kv4::launch_plan(v, w, err_flag, ss->side);
-    if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->side);
-  } else {
-    e = kv4::launch_plan(v, w, err_flag, s);
-  }
-  if (e == cudaSuccess)
-    e = kv4::launch_append(v, static_cast<const uint16_t *>(k_new),
-                           static_cast<const uint16_t *>(v_new), nullptr, batch->num_seqs,
-                           err_flag, s);
-  // join, then the attention and the merge behind both
-  if (e == cudaSuccess && ss != nullptr) e = cudaStreamWaitEvent(s, ss->join, 0);
+  const uint16_t *kn = static_cast<const uint16_t *>(k_new);
+  const uint16_t *vn = static_cast<const uint16_t *>(v_new);
+  // the work list and the append are independent: one launch does both
+  cudaError_t e = batch->plan_reuse
+                      ? kv4::launch_append(v, kn, vn, nullptr, batch->num_seqs, err_flag, s)
+                      : kv4::launch_plan_append(v, w, kn, vn, err_flag, s);
   if (e == cudaSuccess) e = kv4::launch_prefix(v, w, static_cast<const uint16_t *>(q), err_flag, s);
   if (e == cudaSuccess)
     e = kv4::launch_attention(v, w, static_cast<const uint16_t *>(q), err_flag, s);

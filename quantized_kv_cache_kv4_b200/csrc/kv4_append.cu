@@ -27,6 +27,7 @@
 // for the fp16 scales.
 #include "kv4_device.cuh"
 #include "kv4_internal.h"
+#include "kv4_plan.cuh"
 
 
 namespace kv4 {
@@ -172,14 +173,12 @@ __device__ __forceinline__ int find_seq_warp(const int32_t *__restrict__ indptr,
   return lo;
 }
 
-// One warp per (new token, kv head): the token's 256 bytes of K and of V are one
-// coalesced load per warp.
-__global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t *__restrict__ k_new,
-                                                     const uint16_t *__restrict__ v_new,
-                                                     const int32_t *__restrict__ new_indptr,
-                                                     int32_t total_new, int32_t *err) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+// Warp `warp` of the single-token append: (new token, kv head) = (warp / H, warp % H); the
+// token's 256 bytes of K and of V are one coalesced load per warp.
+__device__ __forceinline__ void append_warp(const CacheView &c, const uint16_t *__restrict__ k_new,
+                                            const uint16_t *__restrict__ v_new,
+                                            const int32_t *__restrict__ new_indptr,
+                                            int32_t total_new, int32_t *err, int warp, int lane) {
   const int H = c.num_kv_heads;
   if (warp >= total_new * H) return;
   const int h = warp % H;
@@ -204,6 +203,29 @@ __global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t
     return;
   }
   append_token(c, h, b, pos, L, kr, vr, lane, err);
+}
+
+__global__ void __launch_bounds__(256) append_kernel(CacheView c, const uint16_t *__restrict__ k_new,
+                                                     const uint16_t *__restrict__ v_new,
+                                                     const int32_t *__restrict__ new_indptr,
+                                                     int32_t total_new, int32_t *err) {
+  append_warp(c, k_new, v_new, new_indptr, total_new, err,
+              (blockIdx.x * blockDim.x + threadIdx.x) >> 5, threadIdx.x & 31);
+}
+
+// A decode step's two independent first launches as one: blocks [0, n_plan) build the
+// work list (plan_block; it reads the lengths and page tables, which the append does not
+// write), the blocks after them append one token per sequence, blockDim / 32 (token, kv
+// head) warps per block. The block size is the plan's (32 to 1024 threads by batch size).
+__global__ void __launch_bounds__(kPlanThreads) plan_append_kernel(
+    CacheView c, Workspace w, const uint16_t *__restrict__ k_new,
+    const uint16_t *__restrict__ v_new, int32_t *err, int n_plan) {
+  if (static_cast<int>(blockIdx.x) < n_plan) {
+    plan_block(c, w, err, blockIdx.x, n_plan);
+    return;
+  }
+  const int warp = (static_cast<int>(blockIdx.x) - n_plan) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  append_warp(c, k_new, v_new, nullptr, c.num_seqs, err, warp, threadIdx.x & 31);
 }
 
 // ---------------------------------------------------------------------------
@@ -619,6 +641,17 @@ cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint1
     const unsigned blocks = static_cast<unsigned>((warps * 32 + threads - 1) / threads);
     append_kernel<<<blocks, threads, 0, s>>>(c, k_new, v_new, new_indptr, total_new, err_flag);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan_append(const CacheView &c, const Workspace &w, const uint16_t *k_new,
+                               const uint16_t *v_new, int32_t *err_flag, cudaStream_t s) {
+  int n_plan = 0, threads = 0;
+  plan_shape(c.num_seqs, &n_plan, &threads);
+  const long long warps = static_cast<long long>(c.num_seqs) * c.num_kv_heads;
+  const long long per_block = threads / 32;
+  const unsigned blocks = static_cast<unsigned>(n_plan + (warps + per_block - 1) / per_block);
+  plan_append_kernel<<<blocks, threads, 0, s>>>(c, w, k_new, v_new, err_flag, n_plan);
   return cudaGetLastError();
 }
 

@@ -110,6 +110,11 @@ cudaError_t launch_append(const CacheView &c, const uint16_t *k_new, const uint1
 cudaError_t launch_plan(const CacheView &c, const Workspace &w, int32_t *err_flag,
                         cudaStream_t s);
 
+// The work list of w and the append of one token per sequence (k_new, v_new: bf16
+// [num_seqs][num_kv_heads][128]) in one launch; the two are independent.
+cudaError_t launch_plan_append(const CacheView &c, const Workspace &w, const uint16_t *k_new,
+                               const uint16_t *v_new, int32_t *err_flag, cudaStream_t s);
+
 cudaError_t launch_attention(const CacheView &c, const Workspace &w, const uint16_t *q,
                              int32_t *err_flag, cudaStream_t s);
 

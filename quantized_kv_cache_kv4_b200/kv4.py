@@ -271,8 +271,8 @@ def decode_step(cache: Cache, batch: BatchTensors, k_new: torch.Tensor, v_new: t
                 out_f32: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                 err: torch.Tensor | None = None, stream=None):
     """One decode step: quantize_append of one token per sequence (k_new, v_new bf16
-    [B, Hkv, 128]) then decode_attention, in one library call (the attention's work list
-    is built on a second stream while the append runs). batch.lens: lengths after the
+    [B, Hkv, 128]) then decode_attention, in one library call (one launch builds the
+    attention's work list and appends the tokens). batch.lens: lengths after the
     append."""
     pool, side, bs = cache.pool_struct(), cache.side_struct(), batch.struct()
     st = _lib.kv4_decode_step(ctypes.byref(cache.cfg), ctypes.byref(pool), ctypes.byref(side),
