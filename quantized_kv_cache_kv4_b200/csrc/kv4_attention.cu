@@ -277,10 +277,10 @@ __device__ __forceinline__ int process_protected(WarpCtx &x, const CacheView &c,
       float *r = rec + j * kRecordFloats;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc)  // rows: dim 16cc+2gid (c0/c1) and +1 (c2/c3)
-        *reinterpret_cast<float2 *>(r + 16 * cc + 2 * gid) = make_float2(o[cc][e], o[cc][2 + e]);
+        st_rec(reinterpret_cast<float2 *>(r + 16 * cc + 2 * gid), make_float2(o[cc][e], o[cc][2 + e]));
       if (gid == 0) {
-        r[kHeadDim] = m[e] * kLn2;
-        r[kHeadDim + 1] = l[e];
+        st_rec(r + kHeadDim, m[e] * kLn2);
+        st_rec(r + kHeadDim + 1, l[e]);
       }
     }
   }
@@ -581,10 +581,11 @@ __device__ __forceinline__ int process_protected_pair(WarpCtx &x, const CacheVie
         float *rr = rec + j * kRecordFloats;
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)  // rows: dim 16cc+2gid (c0/c1) and +1 (c2/c3)
-          *reinterpret_cast<float2 *>(rr + 16 * cc + 2 * gid) = make_float2(o[cc][e], o[cc][2 + e]);
+          st_rec(reinterpret_cast<float2 *>(rr + 16 * cc + 2 * gid),
+                 make_float2(o[cc][e], o[cc][2 + e]));
         if (gid == 0) {
-          rr[kHeadDim] = m[e] * kLn2;
-          rr[kHeadDim + 1] = l[e];
+          st_rec(rr + kHeadDim, m[e] * kLn2);
+          st_rec(rr + kHeadDim + 1, l[e]);
         }
       }
     }
@@ -957,11 +958,11 @@ __device__ __forceinline__ int process_int4(WarpCtx &x, const CacheView &c, cons
                                        fmaf(o[g][0][2 + e], kUnscaleV1, mt[g][e]),
                                        fmaf(o[g][1][e], kUnscaleV, mt[g][e]),
                                        fmaf(o[g][1][2 + e], kUnscaleV1, mt[g][e]));
-          *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
+          st_rec(reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid), v);
         }
         if (gid == 0) {
-          rr[kHeadDim] = m[e] * kLn2;
-          rr[kHeadDim + 1] = l[e];
+          st_rec(rr + kHeadDim, m[e] * kLn2);
+          st_rec(rr + kHeadDim + 1, l[e]);
         }
       }
     }
@@ -1334,11 +1335,11 @@ __device__ __forceinline__ bool process_prefix(WarpCtx &x, const CacheView &c, c
                                      fmaf(o[g][0][t][2 + e], kUnscaleV1, mt[g][t][e]),
                                      fmaf(o[g][1][t][e], kUnscaleV, mt[g][t][e]),
                                      fmaf(o[g][1][t][2 + e], kUnscaleV1, mt[g][t][e]));
-        *reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid) = v;
+        st_rec(reinterpret_cast<float4 *>(rr + 32 * g + 4 * gid), v);
       }
       if (gid == 0) {
-        rr[kHeadDim] = m[t][e] * kLn2;
-        rr[kHeadDim + 1] = l[t][e];
+        st_rec(rr + kHeadDim, m[t][e] * kLn2);
+        st_rec(rr + kHeadDim + 1, l[t][e]);
       }
     }
   return false;
@@ -1440,12 +1441,12 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
     float4 a[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i)
-      if (i < cnt) a[i] = __ldcg(reinterpret_cast<const float4 *>(rec_of(base + i)) + lane);
+      if (i < cnt) a[i] = __ldcs(reinterpret_cast<const float4 *>(rec_of(base + i)) + lane);
     float mr = -CUDART_INF_F, lr = 0.f;
     if (lane < cnt) {
       const float *rec = rec_of(base + lane);
-      lr = __ldcg(rec + kHeadDim + 1);
-      mr = lr > 0.f ? __ldcg(rec + kHeadDim) : -CUDART_INF_F;
+      lr = __ldcs(rec + kHeadDim + 1);
+      mr = lr > 0.f ? __ldcs(rec + kHeadDim) : -CUDART_INF_F;
     }
     float bm = mr;
 #pragma unroll

@@ -215,10 +215,10 @@ __device__ __forceinline__ bool withheld_item(const Workspace &w, int item) {
 __device__ inline void write_empty(float *rec, int G, int lane) {
   for (int j = 0; j < G; ++j) {
     float *r = rec + j * kRecordFloats;
-    reinterpret_cast<float4 *>(r)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    st_rec(reinterpret_cast<float4 *>(r) + lane, make_float4(0.f, 0.f, 0.f, 0.f));
     if (lane == 0) {
-      r[kHeadDim] = -CUDART_INF_F;
-      r[kHeadDim + 1] = 0.0f;
+      st_rec(r + kHeadDim, -CUDART_INF_F);
+      st_rec(r + kHeadDim + 1, 0.0f);
     }
   }
 }

@@ -83,6 +83,30 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
       : "memory");
 }
 
+// Stores of partial records: written by the attention kernels and read back by the merge
+// (with evict-first loads) right after, so they are stored with the L2 evict_last
+// priority and stay in L2 while the pages stream past (measured: the call 1.5-2 us
+// faster on every batch; an evict_first hint on the page copies was slower).
+__device__ __forceinline__ uint64_t l2_keep_policy() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_rec(float *p, float v) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(l2_keep_policy())
+               : "memory");
+}
+__device__ __forceinline__ void st_rec(float2 *p, float2 v) {
+  asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y),
+               "l"(l2_keep_policy())
+               : "memory");
+}
+__device__ __forceinline__ void st_rec(float4 *p, float4 v) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(l2_keep_policy())
+               : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // warp-level tensor cores: D(16x8, f32) += A(16x16, f16, row) * B(16x8, f16, col)
 // Fragment ownership, lane = 4*gid + tig:
