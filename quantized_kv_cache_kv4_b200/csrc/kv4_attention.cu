@@ -1390,16 +1390,32 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) prefix_kernel(Cac
 //   M = max m_r, Lambda = sum l_r e^(m_r - M), O = sum acc_r e^(m_r - M) / Lambda,
 //   lse = M + ln Lambda, over live regions (l_r > 0); no live region gives O = 0,
 //   lse = -inf.
-// Regions are taken in batches of 4: the lanes first issue every load of the batch (the
-// region maxima and sums spread over the lanes, each lane's 4 dims of every record),
-// then the batch's weights are formed and added in region order. The arithmetic order
-// is fixed, so the result is deterministic; M is the running maximum over the batches
-// (with a rescale between batches, as in the online softmax). Batches of 4 rather than
-// 8 keep the registers low enough for 40 resident warps per SM (measured in graphs:
-// 13.4 against 17.4 us on the 1024-sequence batch, 7.0 against 8.4 us on 128 x 16384).
-__global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ partials,
+// Regions are taken in batches of 4: every lane loads its 4 dims of each record of the
+// batch and, with one broadcast load per record, the record's (m, l); each lane then
+// forms the batch's maximum and weights itself (no shuffles) and adds the records in
+// region order. The arithmetic order is fixed, so the result is deterministic; M is the
+// running maximum over the batches (with a rescale between batches, as in the online
+// softmax). e^x is evaluated as 2^(x log2 e) with x = m_r - M formed first, so the
+// rounding of the scaling is relative to the difference (weights and Lambda to a few
+// 1e-7 relative for the differences that carry weight); 1/Lambda and ln Lambda use the
+// hardware reciprocal and base-2 logarithm (1-2 ulp). Against per-lane gathers with
+// shuffle reductions, IEEE division and the library exp/log (292 instructions per row)
+// this takes a third of the instructions. Batches of 4 rather than 8 keep the registers
+// low enough for 40 resident warps per SM.
+__device__ __forceinline__ float fast_log2(float x) {
+  float y;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(256, 5) merge_kernel(const float *__restrict__ partials,
                                                     const int32_t *__restrict__ offs, int n_units,
-                                                    int G, Outputs o, int32_t *reset,
+                                                    int G, int g_shift, Outputs o, int32_t *reset,
                                                     PlanSig want, int check) {
   constexpr int kBatch = 4;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -1429,46 +1445,46 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
     reset[5] = 0;
   }
   if (warp >= n_units * G) return;
-  const int u = warp / G, j = warp - u * G;
+  const int u = g_shift >= 0 ? warp >> g_shift : warp / G;
+  const int j = warp - u * G;
   const int r0 = offs[u], n = offs[u + 1] - r0;
-  auto rec_of = [&](int r) {
-    return partials + (static_cast<size_t>(r0 + r) * G + j) * kRecordFloats;
-  };
+  const int stride = G * kRecordFloats;  // floats from one region's record to the next
+  const float *rec = partials + (static_cast<size_t>(r0) * G + j) * kRecordFloats;
   float M = -CUDART_INF_F, lam = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int base = 0; base < n; base += kBatch) {
+  for (int base = 0; base < n; base += kBatch, rec += kBatch * stride) {
     const int cnt = min(kBatch, n - base);
     float4 a[kBatch];
+    float2 ml[kBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-      if (i < cnt) a[i] = __ldcs(reinterpret_cast<const float4 *>(rec_of(base + i)) + lane);
-    float mr = -CUDART_INF_F, lr = 0.f;
-    if (lane < cnt) {
-      const float *rec = rec_of(base + lane);
-      lr = __ldcs(rec + kHeadDim + 1);
-      mr = lr > 0.f ? __ldcs(rec + kHeadDim) : -CUDART_INF_F;
+    for (int i = 0; i < kBatch; ++i) {
+      a[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      ml[i] = make_float2(-CUDART_INF_F, 0.f);
+      if (i < cnt) {
+        a[i] = __ldcs(reinterpret_cast<const float4 *>(rec + i * stride) + lane);
+        ml[i] = __ldcs(reinterpret_cast<const float2 *>(rec + i * stride + kHeadDim));
+      }
     }
-    float bm = mr;
+    float mr[kBatch];
+    float bm = -CUDART_INF_F;
 #pragma unroll
-    for (int off = 4; off; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-    bm = __shfl_sync(0xffffffffu, bm, 0);  // max over the batch (lanes 0..3; 4..7 hold -inf)
-    if (bm == -CUDART_INF_F) continue;     // no live region in this batch
+    for (int i = 0; i < kBatch; ++i) {
+      mr[i] = ml[i].y > 0.f ? ml[i].x : -CUDART_INF_F;  // only live regions carry weight
+      bm = fmaxf(bm, mr[i]);
+    }
+    if (bm == -CUDART_INF_F) continue;  // no live region in this batch
     const float Mn = fmaxf(M, bm);
-    if (Mn != M) {  // rescale what was accumulated under the old maximum
-      const float sc = expf(M - Mn);
+    if (Mn != M) {  // rescale what was accumulated under the old maximum (0 at the start)
+      const float sc = fast_exp2((M - Mn) * kLog2e);
       acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
       lam *= sc;
       M = Mn;
     }
-    const float wl = lr > 0.f ? expf(mr - M) : 0.f;  // this lane's region weight
-    float ls = lr * wl;
-#pragma unroll
-    for (int off = 4; off; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-    lam += __shfl_sync(0xffffffffu, ls, 0);
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const float wgt = __shfl_sync(0xffffffffu, wl, i);
-      if (i < cnt && wgt > 0.f) {
+      const float wgt = fast_exp2((mr[i] - M) * kLog2e);  // 0 for a dead or absent region
+      if (wgt > 0.f) {  // a skipped region's acc is never read into the sum
+        lam = fmaf(ml[i].y, wgt, lam);
         acc.x = fmaf(a[i].x, wgt, acc.x);
         acc.y = fmaf(a[i].y, wgt, acc.y);
         acc.z = fmaf(a[i].z, wgt, acc.z);
@@ -1476,7 +1492,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
       }
     }
   }
-  const float inv = lam > 0.f ? 1.0f / lam : 0.f;
+  const float inv = lam > 0.f ? fast_rcp(lam) : 0.f;
   const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   const size_t row = static_cast<size_t>(u) * G + j;
   __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
@@ -1485,7 +1501,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const float *__restrict__ pa
   packed.y = *reinterpret_cast<uint32_t *>(&hi);
   *reinterpret_cast<uint2 *>(o.out + row * kHeadDim + 4 * lane) = packed;
   if (o.out_f32) *reinterpret_cast<float4 *>(o.out_f32 + row * kHeadDim + 4 * lane) = v;
-  if (o.lse && lane == 0) o.lse[row] = lam > 0.f ? M + logf(lam) : -CUDART_INF_F;
+  if (o.lse && lane == 0) o.lse[row] = lam > 0.f ? M + fast_log2(lam) * kLn2 : -CUDART_INF_F;
 }
 
 
@@ -1716,8 +1732,9 @@ cudaError_t launch_merge(const float *partials, const int32_t *unit_offsets, int
   const long long warps = static_cast<long long>(n_units) * group;
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps * 32 + 255) / 256;
+  const int g_shift = (group & (group - 1)) == 0 ? __builtin_ctz(group) : -1;
   merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      partials, unit_offsets, n_units, group, Outputs{out, out_f32, lse},
+      partials, unit_offsets, n_units, group, g_shift, Outputs{out, out_f32, lse},
       const_cast<int32_t *>(reset), want ? *want : PlanSig{}, want && reset ? 1 : 0);
   return cudaGetLastError();
 }
