@@ -464,7 +464,7 @@ def run_gpu(args, rank, world, local_rank):
         return ev[0].elapsed_time(ev[1]), [a.elapsed_time(b) for a, b in att]
 
     # A timed step is one kv4_decode_step call per layer (append + attention in one call,
-    # the attention's work list built beside the append); the attention calls are also
+    # the work list and the append in one launch); the attention calls are also
     # timed on their own, as the separate kv4_decode_attention call, for the roofline.
     # eager: every call launches its kernels from the host
     with ClockSampler(local_rank) as clocks_eager:
@@ -551,7 +551,7 @@ def run_gpu(args, rank, world, local_rank):
             "data": "synthetic",
             "config": bench_config(wl, args.cache, world),
             "method": {"step": "one kv4_decode_step call per layer (append + attention; "
-                               "the work list built on a second stream beside the append"
+                               "the work list and the append in one launch"
                                + ("; layers after the first reuse the first layer's work list"
                                   if nl > 1 and args.plan_reuse == "on" else "") + ")",
                        "launch": {"graph": "cuda graph per call, replayed (each layer's "

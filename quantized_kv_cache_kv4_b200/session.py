@@ -186,7 +186,7 @@ class DecodeSession:
 
     def step_call(self, batch, k, v, q, out, out_f32=None, lse=None, stream=None):
         """One decode step (one new token per sequence) as one kv4.decode_step call:
-        append + attention, the attention's work list built beside the append."""
+        append + attention; one launch builds the work list and appends the tokens."""
         kv4.decode_step(self.cache, batch, k, v, q, out, self.workspace, out_f32, lse,
                         self.err, stream=stream)
 

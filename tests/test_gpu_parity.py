@@ -464,7 +464,7 @@ def test_bulk_append_across_empty_sequences():
 
 
 def test_decode_step_matches_separate_calls():
-    """kv4_decode_step (append + attention, the work list built on a second stream) gives
+    """kv4_decode_step (append + attention, its work list and the append in one launch) gives
     the same cache and the same outputs, bit for bit, as the two calls in order; also
     when captured in a CUDA graph, including a new thread's first call; and its outputs
     match the oracle."""
