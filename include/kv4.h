@@ -103,9 +103,11 @@ typedef struct {
   int32_t num_sinks;    /* S >= 0 */
   int32_t num_recent;   /* R >= 0, S + R <= 144 */
   int32_t chunk_pages;  /* split-K chunk length in pages for the INT4 region, 1..64; 0 = chosen
-                           per call from num_seqs and max_seq_len: 64 for large batches, down
-                           to 8 when long chunks would leave the GPU's warps idle (and 64
-                           whenever the workspace passed is too small for the finer split) */
+                           per call from num_seqs and max_seq_len: the length in 8..64 with
+                           the shortest estimated attention time on the GPU's resident warps
+                           (64 for large batches, shorter where long chunks would leave
+                           warps idle; 64 whenever the workspace passed is too small for
+                           the finer split) */
   int32_t demotion;     /* where a position's INT4 copy comes from: 0 = the bf16 input, at
                            append (reading A, the default); 1 = the position's INT8 copy,
                            dequantised (reading B: what demotion out of the recent window

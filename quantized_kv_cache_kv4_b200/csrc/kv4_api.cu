@@ -27,27 +27,54 @@ kv4_status check_config(const kv4_config *cfg) {
   return KV4_OK;
 }
 
-// Automatic chunk length (chunk_pages == 0): the longest chunk in kAutoChunks that still
-// gives the persistent attention grid about one entry per resident warp (148 SMs x 3
-// CTAs x 4 warps) for num_seqs sequences of max_seq_len tokens. Large batches get 64-page
-// chunks (fewest partial states to merge); small batches are split finer so every warp
-// has work.
-constexpr int kAutoChunks[] = {64, 48, 32, 24, 16, 12, 8};
-constexpr long long kAutoTargetEntries = 148LL * 3 * 4;
+// Automatic chunk length (chunk_pages == 0), from num_seqs and max_seq_len only (the
+// lengths themselves are on the device): the C in [8, 64] with the shortest estimated
+// attention time, in units of one INT4 page of one warp, on the W = 148 SMs x 3 CTAs x 4
+// warps resident warps of the persistent grid:
+//   T(C) = max(C + e, work(C) / W) + (entries(C) > W ? (C + e) / 2 : 0),
+// where an entry costs its pages plus e (its set-up, the ramp of its first copies, its
+// record and its share of the merge), a protected-set entry kProtEntryPages, and work is
+// the sum over all entries. One round of entries (entries <= W) ends with its longest
+// entry; with more, the second term is the imbalance of the last round. Of the C within
+// kAutoSlack of the best estimate the longest is taken (fewest partial states). The
+// constants fit calls measured at forced chunk lengths: one round at the shortest C
+// reaching it on 64 x 2048 and 32 x 4096 (C = 24, 21), 24- to 32-page chunks on
+// 256 x 1024, 64 on the 1024-sequence rollout batch and on 128 x 16384 (32 and 48 there
+// 1-5 % slower).
+constexpr int kAutoMinChunk = 8;
+constexpr double kAutoWarps = 148.0 * 3 * 4;
+constexpr double kEntryPages = 8.0;
+constexpr double kProtEntryPages = 12.0;
+constexpr double kAutoSlack = 1.03;  // the longest C within 3 % of the best estimate
 
 int chunk_of(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
   if (cfg->chunk_pages > 0) return cfg->chunk_pages;
   const int H = cfg->num_kv_heads;
   const int hpw = kv4::heads_per_warp_for(cfg->num_q_heads / H);
-  const long long nslots = (H + hpw - 1) / hpw;
-  const int protect = cfg->num_sinks + cfg->num_recent;
-  const long long int4_pages = (std::max(0, max_seq_len - protect) + kv4::kPage - 1) / kv4::kPage + 1;
-  const long long prot_entries = protect > 0 ? nslots : 0;
-  for (int C : kAutoChunks) {
-    const long long entries = num_seqs * (nslots * ((int4_pages + C - 1) / C) + prot_entries);
-    if (entries >= kAutoTargetEntries) return C;
+  const double slots = static_cast<double>(num_seqs) * ((H + hpw - 1) / hpw);
+  const int S = cfg->num_sinks, R = cfg->num_recent;
+  // pages of the INT4 range [S, L - R) at L = max_seq_len
+  const long long int4_pages =
+      max_seq_len - R > S ? (max_seq_len - R - 1) / kv4::kPage - S / kv4::kPage + 1 : 0;
+  const double prot_entries = S + R > 0 ? slots : 0.0;
+  double t[kv4::kMaxChunkPages + 1];
+  double t_min = 0.0;
+  for (int C = kAutoMinChunk; C <= kv4::kMaxChunkPages; ++C) {
+    const double n_c = static_cast<double>((int4_pages + C - 1) / C);
+    const double entries = slots * n_c + prot_entries;
+    const double work = slots * (static_cast<double>(int4_pages) + n_c * kEntryPages) +
+                        prot_entries * kProtEntryPages;
+    t[C] = std::max(C + kEntryPages, work / kAutoWarps);
+    if (entries > kAutoWarps) t[C] += 0.5 * (C + kEntryPages);
+    if (C == kAutoMinChunk || t[C] < t_min) t_min = t[C];
   }
-  return kAutoChunks[sizeof(kAutoChunks) / sizeof(kAutoChunks[0]) - 1];
+  int best = kAutoMinChunk;
+  for (int C = kv4::kMaxChunkPages; C >= kAutoMinChunk; --C)
+    if (t[C] <= kAutoSlack * t_min) {
+      best = C;
+      break;
+    }
+  return best;
 }
 
 bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
