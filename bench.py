@@ -574,12 +574,13 @@ def run_gpu(args, rank, world, local_rank):
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                     "host_issue_ms_per_step": host_ms / K},
             "output_check": check,
-            # per step and layer: plan, append, attention, merge (+ the lift kernel, and the
-            # prefix kernel with the shared-prefix read) for KV4-RL; plan, append,
-            # attention, merge for a comparison cache
-            "gpu_launches": ((4 + (1 if args.cache == "kv4" else 0)
-                              + (1 if args.cache == "kv4" and args.prefix == "shared" else 0))
-                             * nl - (nl - 1 if nl > 1 and args.plan_reuse == "on" else 0)) * K,
+            # per step and layer for KV4-RL: the work list and the append in one launch (the
+            # append alone with a reused list), attention, lift, merge (+ the prefix kernel
+            # with the shared-prefix read); for a comparison cache: append, plan (none
+            # with a reused list), attention, merge
+            "gpu_launches": ((4 + (1 if args.prefix == "shared" else 0)) * nl
+                             if args.cache == "kv4" else
+                             4 * nl - (nl - 1 if nl > 1 and args.plan_reuse == "on" else 0)) * K,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
