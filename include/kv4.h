@@ -178,6 +178,14 @@ typedef struct {
 size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len);
 
 /*
+ * The split-K chunk length in pages that kv4_decode_attention and kv4_workspace_size use
+ * for a batch of num_seqs sequences no longer than max_seq_len: cfg->chunk_pages when it
+ * is set, else the automatic choice (see kv4_config.chunk_pages). Returns -1 for invalid
+ * arguments. (Infrastructure of this library: no passage of the pages defines it.)
+ */
+int32_t kv4_chunk_pages_for(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len);
+
+/*
  * Quantise and append new tokens' K/V: the per-step write path (with n = 1 per
  * sequence), also usable for bulk prefill.
  * Defined by: the whole context kept in calibration-free INT4 in a paged format, with

@@ -239,6 +239,11 @@ size_t kv4_workspace_size(const kv4_config *cfg, int32_t num_seqs, int32_t max_s
                               nullptr);
 }
 
+int32_t kv4_chunk_pages_for(const kv4_config *cfg, int32_t num_seqs, int32_t max_seq_len) {
+  if (check_config(cfg) != KV4_OK || num_seqs < 0 || max_seq_len < 0) return -1;
+  return chunk_of(cfg, num_seqs, max_seq_len);
+}
+
 kv4_status kv4_quantize_append(const kv4_config *cfg, const kv4_int4_pool *pool,
                                const kv4_int8_side *side, const kv4_batch *batch,
                                const void *k_new, const void *v_new, const int32_t *new_indptr,

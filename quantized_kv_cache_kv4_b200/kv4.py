@@ -28,8 +28,9 @@ HEAD_DIM = 128
 PAGE = 16
 GROUP = 32
 
-EXPORTS = ("kv4_workspace_size", "kv4_quantize_append", "kv4_decode_attention",
-           "kv4_decode_step", "kv4_regional_merge", "kv4_status_string", "kv4_version",
+EXPORTS = ("kv4_workspace_size", "kv4_chunk_pages_for", "kv4_quantize_append",
+           "kv4_decode_attention", "kv4_decode_step", "kv4_regional_merge",
+           "kv4_status_string", "kv4_version",
            "kv4_decode_attention_noalloc", "kv4_noalloc_scratch_bytes",
            "kv4_baseline_append", "kv4_baseline_workspace_size",
            "kv4_baseline_decode_attention", "kv4_test_withhold_copy")
@@ -82,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P = ctypes.c_void_p
     lib.kv4_workspace_size.restype = ctypes.c_size_t
     lib.kv4_workspace_size.argtypes = [ctypes.POINTER(Config), ctypes.c_int32, ctypes.c_int32]
+    lib.kv4_chunk_pages_for.restype = ctypes.c_int32
+    lib.kv4_chunk_pages_for.argtypes = [ctypes.POINTER(Config), ctypes.c_int32, ctypes.c_int32]
     lib.kv4_quantize_append.restype = ctypes.c_int
     lib.kv4_quantize_append.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Int4Pool),
                                         ctypes.POINTER(Int8Side), ctypes.POINTER(Batch),
@@ -239,6 +242,14 @@ def workspace_size(cfg: Config, num_seqs: int, max_seq_len: int) -> int:
     n = _lib.kv4_workspace_size(ctypes.byref(cfg), num_seqs, max_seq_len)
     if n == 0 and num_seqs > 0:
         raise KV4Error("kv4_workspace_size: invalid arguments")
+    return n
+
+
+def chunk_pages_for(cfg: Config, num_seqs: int, max_seq_len: int) -> int:
+    """The INT4 chunk length (pages) the library uses for such a batch."""
+    n = _lib.kv4_chunk_pages_for(ctypes.byref(cfg), num_seqs, max_seq_len)
+    if n < 0:
+        raise KV4Error("kv4_chunk_pages_for: invalid arguments")
     return n
 
 

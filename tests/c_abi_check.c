@@ -45,6 +45,14 @@ int main(void) {
   kv4_config too_wide = config(32, 8, 100, 100, 0);
   CHECK(kv4_workspace_size(&too_wide, 64, 2048) == 0);
 
+  /* chunk lengths: the configured one, an automatic one in 8..64, -1 when rejected */
+  CHECK(kv4_chunk_pages_for(&c, 64, 2048) == 32);
+  kv4_config autoc = config(32, 8, 16, 128, 0);
+  int32_t ch = kv4_chunk_pages_for(&autoc, 64, 2048);
+  CHECK(ch >= 8 && ch <= 64);
+  CHECK(kv4_chunk_pages_for(&autoc, 1024, 16384) == 64);
+  CHECK(kv4_chunk_pages_for(&too_wide, 64, 2048) == -1);
+
   /* argument checks answer before any launch */
   kv4_int4_pool pool;
   kv4_int8_side side;

@@ -147,6 +147,33 @@ def test_automatic_chunk_splits_small_batches_finer(kv4):
     assert kv4.workspace_size(auto, 1024, 14348) == kv4.workspace_size(c64, 1024, 14348)
 
 
+def test_automatic_chunk_length(kv4):
+    """The automatic chunk length (kv4_chunk_pages_for): within 8..64; the configured length
+    when one is set; 64 pages for large batches; for batches whose entries fit one round of
+    the 1776 resident warps of the persistent grid, the shortest length that keeps them in
+    one round (64 x 2048: 120 INT4 pages per kv-head pair -> 5 chunks of 24; 32 x 4096:
+    248 pages -> 12 chunks of 21); the shortest length for a handful of sequences."""
+    c = _cfg(kv4)
+    assert kv4.chunk_pages_for(_cfg(kv4, chunk_pages=32), 2, 1000) == 32
+    assert kv4.chunk_pages_for(c, 64, 2049) == 24
+    assert kv4.chunk_pages_for(c, 32, 4097) == 21
+    assert kv4.chunk_pages_for(c, 1024, 14349) == 64
+    assert kv4.chunk_pages_for(c, 128, 16385) == 64
+    assert kv4.chunk_pages_for(c, 2, 1000) == 8
+    for B in (1, 7, 100, 600, 3000):
+        for L in (0, 150, 5000, 100000):
+            assert 8 <= kv4.chunk_pages_for(c, B, L) <= 64, (B, L)
+    # one round: the entries (two kv heads per warp: 4 slots per sequence, one protected
+    # entry per slot) at the chosen length fit the resident warps, one page shorter not
+    for B, L in ((64, 2049), (32, 4097), (16, 8193)):
+        pages = (L - 128 - 1) // 16 - 16 // 16 + 1
+        C = kv4.chunk_pages_for(c, B, L)
+        entries = lambda C: B * 4 * (-(-pages // C)) + B * 4
+        assert entries(C) <= 1776 < entries(C - 1), (B, L, C)
+    bad = _cfg(kv4, num_sinks=100, num_recent=100)
+    assert kv4._lib.kv4_chunk_pages_for(ctypes.byref(bad), 4, 100) == -1
+
+
 def test_workspace_too_small_is_reported(kv4):
     c = _cfg(kv4)
     # too small even for 64-page chunks, the fallback of the automatic choice
