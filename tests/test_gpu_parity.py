@@ -463,6 +463,50 @@ def test_bulk_append_across_empty_sequences():
     check_cache(sess, [b for b in range(wl.num_seqs) if counts[b] > 0])
 
 
+STEP_CASES = [
+    # name, lens, Hq, Hkv, S, R, prompt_len, group_seqs, prefix
+    # fewer sequences than a warp: blocks of 32 threads for the plan and the append
+    ("three-seqs", [150, 700, 33], 8, 2, 4, 32, 0, 1, "off"),
+    # more sequences than a block: the plan's multi-pass path in every plan block
+    ("1100-seqs", [40 + (37 * i) % 400 for i in range(1100)], 8, 2, 4, 32, 0, 1, "off"),
+    # the shared-prefix read: the plan blocks also compare page tables
+    ("shared-prefix", [700, 900, 410, 1300, 260, 2000, 520, 640], 32, 8, 16, 128, 256, 4,
+     "shared"),
+]
+
+
+@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,P,grp,prefix", STEP_CASES,
+                         ids=[c[0] for c in STEP_CASES])
+def test_decode_step_shapes(name, lens, Hq, Hkv, S, R, P, grp, prefix):
+    """kv4_decode_step (one launch for the work list and the append, then the attention)
+    against kv4_quantize_append followed by kv4_decode_attention: the same outputs, bit for
+    bit, over two steps, for a batch under one warp, one over 1024 sequences and one with
+    the shared-prefix read; sampled sequences also against the oracle."""
+    _, session, W = _mods()
+    wl = W.custom_workload(lens, num_q_heads=Hq, num_kv_heads=Hkv, num_sinks=S, num_recent=R,
+                           prompt_len=P, group_seqs=grp,
+                           seed=zlib.crc32(name.encode()) & 0xFFFF)
+    keep = sorted(set([0, len(lens) // 2, len(lens) - 1]))
+    sa = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix)
+    sb = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix)
+    B = wl.num_seqs
+    dev = torch.device("cuda")
+    for s in range(2):
+        o = [(torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev),
+              torch.empty((B, Hq, 128), dtype=torch.float32, device=dev),
+              torch.empty((B, Hq), dtype=torch.float32, device=dev)) for _ in range(2)]
+        sa.append_step(s)
+        sa.attention_step(s, out=o[0][0], out_f32=o[0][1], lse=o[0][2])
+        sb.fused_step(s, out=o[1][0], out_f32=o[1][1], lse=o[1][2])
+        torch.cuda.synchronize()
+        for x, y in zip(o[0], o[1]):
+            assert torch.equal(x, y), (name, s)
+        check_attention(sb, keep, step=s, got=(o[1][0].float().cpu().numpy(),
+                                                o[1][1].cpu().numpy(), o[1][2].cpu().numpy()))
+    sa.check_err()
+    sb.check_err()
+
+
 def test_decode_step_matches_separate_calls():
     """kv4_decode_step (append + attention, its work list and the append in one launch) gives
     the same cache and the same outputs, bit for bit, as the two calls in order; also
@@ -502,8 +546,7 @@ def test_decode_step_matches_separate_calls():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(oa, ob) and torch.equal(fa, fb) and torch.equal(la, lb)
-    # step 3: the first call of a new host thread, made while capturing (the library
-    # creates nothing then and builds the work list on the captured stream)
+    # step 3: the first call of a new host thread, made while capturing
     import threading
     oa, fa, la = outs()
     ob, fb, lb = outs()
