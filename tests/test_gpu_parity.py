@@ -464,31 +464,36 @@ def test_bulk_append_across_empty_sequences():
 
 
 STEP_CASES = [
-    # name, lens, Hq, Hkv, S, R, prompt_len, group_seqs, prefix
+    # name, lens, Hq, Hkv, S, R, prompt_len, group_seqs, prefix, demotion reading
     # fewer sequences than a warp: blocks of 32 threads for the plan and the append
-    ("three-seqs", [150, 700, 33], 8, 2, 4, 32, 0, 1, "off"),
+    ("three-seqs", [150, 700, 33], 8, 2, 4, 32, 0, 1, "off", "A"),
     # more sequences than a block: the plan's multi-pass path in every plan block
-    ("1100-seqs", [40 + (37 * i) % 400 for i in range(1100)], 8, 2, 4, 32, 0, 1, "off"),
+    ("1100-seqs", [40 + (37 * i) % 400 for i in range(1100)], 8, 2, 4, 32, 0, 1, "off", "A"),
     # the shared-prefix read: the plan blocks also compare page tables
     ("shared-prefix", [700, 900, 410, 1300, 260, 2000, 520, 640], 32, 8, 16, 128, 256, 4,
-     "shared"),
+     "shared", "A"),
+    # demotion reading B: the INT4 copy quantised from the INT8 copy
+    ("reading-b", [300, 45, 1000, 129, 17], 8, 2, 4, 32, 0, 1, "off", "B"),
 ]
 
 
-@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,P,grp,prefix", STEP_CASES,
+@pytest.mark.parametrize("name,lens,Hq,Hkv,S,R,P,grp,prefix,demotion", STEP_CASES,
                          ids=[c[0] for c in STEP_CASES])
-def test_decode_step_shapes(name, lens, Hq, Hkv, S, R, P, grp, prefix):
+def test_decode_step_shapes(name, lens, Hq, Hkv, S, R, P, grp, prefix, demotion):
     """kv4_decode_step (one launch for the work list and the append, then the attention)
-    against kv4_quantize_append followed by kv4_decode_attention: the same outputs, bit for
-    bit, over two steps, for a batch under one warp, one over 1024 sequences and one with
-    the shared-prefix read; sampled sequences also against the oracle."""
+    against kv4_quantize_append followed by kv4_decode_attention: the same outputs and the
+    same cache bytes, bit for bit, over two steps, for a batch under one warp, one over 1024
+    sequences, one with the shared-prefix read and one in demotion reading B; sampled
+    sequences also against the oracle."""
     _, session, W = _mods()
     wl = W.custom_workload(lens, num_q_heads=Hq, num_kv_heads=Hkv, num_sinks=S, num_recent=R,
                            prompt_len=P, group_seqs=grp,
                            seed=zlib.crc32(name.encode()) & 0xFFFF)
     keep = sorted(set([0, len(lens) // 2, len(lens) - 1]))
-    sa = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix)
-    sb = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix)
+    sa = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix,
+                               demotion=demotion)
+    sb = session.DecodeSession(wl, steps=2, keep_streams=keep, prefix=prefix,
+                               demotion=demotion)
     B = wl.num_seqs
     dev = torch.device("cuda")
     for s in range(2):
@@ -503,6 +508,11 @@ def test_decode_step_shapes(name, lens, Hq, Hkv, S, R, P, grp, prefix):
             assert torch.equal(x, y), (name, s)
         check_attention(sb, keep, step=s, got=(o[1][0].float().cpu().numpy(),
                                                 o[1][1].cpu().numpy(), o[1][2].cpu().numpy()))
+    # the caches the two paths wrote, byte for byte (INT4 pages of the new positions
+    # included, which no attention of these steps reads yet)
+    for f in ("k_codes", "v_codes", "k_params", "v_params", "sink_k", "sink_v", "sink_ks",
+              "sink_vs", "ring_k", "ring_v", "ring_ks", "ring_vs"):
+        assert torch.equal(getattr(sa.cache, f), getattr(sb.cache, f)), (name, f)
     sa.check_err()
     sb.check_err()
 
